@@ -1,0 +1,28 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+    config.addinivalue_line("markers", "slow: large workloads (minutes of oracle time)")
+
+
+def pytest_collection_modifyitems(config, items):
+    # GPU tests need the device; without one they are skipped rather than failed
+    # only when the run did not select them explicitly with -m gpu.
+    import torch
+    if torch.cuda.is_available():
+        return
+    sel = config.getoption("-m") or ""
+    if "gpu" in sel and "not gpu" not in sel:
+        return
+    skip = pytest.mark.skip(reason="no CUDA device")
+    for it in items:
+        if "gpu" in it.keywords:
+            it.add_marker(skip)
