@@ -1,0 +1,415 @@
+"""LatentMoE layer forward benchmark: tokens/s on B200 and the dominant kernel's roofline fraction.
+
+One step = one full layer forward (router GEMM, top-K' + softmax, counting
+sort, expert up / down GEMMs, combine, up-projection + residual) over one
+batch of seeded synthetic tokens, with weights and inputs resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank runs an
+independent replica of the layer on its own tokens (the layer shards by
+tokens with no exchange step), so per-GPU work is fixed: weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from latent_mixture_experts_gemm_b200 import lmoe, synth  # noqa: E402
+
+METRIC = "LatentMoE layer tokens/s at 1 B200 (prefill & decode); % of BF16/HBM roofline"
+DEFAULT_WORKLOAD = "nemotron_decode"
+SECONDARY_WORKLOAD = "nemotron_prefill"
+N_INPUT_BATCHES = 4  # distinct token batches cycled through the steps
+SMALL_ROWS = 8       # the library's default split: experts with <= 8 rows take the weight-streaming path
+
+
+# ----------------------------------------------------------------------------- peaks
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _smi_id(device: int) -> str:
+    """nvidia-smi --id for a torch device (its UUID; CUDA_VISIBLE_DEVICES may renumber indices)."""
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(device)
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def layer_work(cfg, stats, T):
+    """F (FLOPs) and B (bytes) of one forward from its actual routing."""
+    g = 2 if cfg.gated else 1
+    R, E = stats["ffn_rows"], stats["experts_touched"]
+    d, L, m, nt = cfg.d, cfg.latent, cfg.m, cfg.n_total
+    if cfg.has_proj:
+        F = 2 * T * (2 * d * L + d * nt) + 2 * (g + 1) * L * m * R
+        B = 2 * ((g + 1) * L * m * E + 2 * d * L + d * nt) + 2 * 2 * T * d
+    else:
+        F = 2 * T * d * nt + 2 * (g + 1) * d * m * R
+        B = 2 * ((g + 1) * d * m * E + d * nt) + 4 * T * d
+    return float(F), float(B)
+
+
+def phase_units(cfg, stats, T, phase):
+    """Algorithmic (flops, bytes) of one launch of a phase's kernel."""
+    g = 2 if cfg.gated else 1
+    d, L, m, nt = cfg.d, cfg.latent, cfg.m, cfg.n_total
+    fin = L  # expert input width (== d for the standard MoE)
+    rows_tc = stats.get("tc_rows", 0)
+    rows_st = stats.get("stream_rows", 0)
+    e_tc = stats.get("tc_experts", 0)
+    e_st = stats.get("stream_experts", 0)
+    if phase == "expert_up_gemm":
+        return 2.0 * rows_tc * fin * g * m, 2.0 * (g * m * fin * e_tc + rows_tc * fin + rows_tc * m)
+    if phase == "expert_down_gemm":
+        return 2.0 * rows_tc * m * fin, 2.0 * (fin * m * e_tc + rows_tc * m + rows_tc * fin)
+    if phase == "expert_up_stream":
+        return 2.0 * rows_st * fin * g * m, 2.0 * (g * m * fin * e_st + rows_st * fin + rows_st * m)
+    if phase == "expert_down_stream":
+        return 2.0 * rows_st * m * fin, 2.0 * (fin * m * e_st + rows_st * m + rows_st * fin)
+    if phase == "router_proj_gemm":
+        n_out = (L if cfg.has_proj else 0) + nt
+        return 2.0 * T * d * n_out, 2.0 * (n_out * d + T * d) + T * (L * 2 if cfg.has_proj else 0) + 4.0 * T * nt
+    if phase == "up_proj_gemm":
+        return 2.0 * T * L * d, 2.0 * (d * L + T * L + 2 * T * d)
+    if phase == "combine":
+        return 2.0 * T * cfg.top_k * L, 2.0 * (rows_tc + rows_st) * L + 2.0 * T * L
+    return 0.0, 0.0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def setup_layer(cfg, rank, device):
+    layer = synth.make_layer(cfg)
+    xs = [synth.make_tokens(cfg, cfg.tokens, seed=1000 * (rank + 1) + i) for i in range(N_INPUT_BATCHES)]
+    return layer, xs
+
+
+def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_clocks=True):
+    torch.cuda.set_device(device)
+    layer, xs = setup_layer(cfg, rank, device)
+    T = cfg.tokens
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=T, device=f"cuda:{device}")
+    xd = [x.to(f"cuda:{device}") for x in xs]
+    yd = torch.empty_like(xd[0])
+    stream = torch.cuda.current_stream()
+
+    # routing statistics averaged over the input batches (path split for the per-kernel work)
+    acc = {}
+    for xb in xd:
+        _, dbg = mod.forward(xb, yd, debug=True)
+        torch.cuda.synchronize()
+        st = lmoe.lmoe_routing_stats(mod.h)
+        counts = dbg["counts"].cpu().numpy()[: cfg.n_ffn]
+        tc_mask = counts > SMALL_ROWS
+        st_mask = (counts > 0) & ~tc_mask
+        st.update(tc_rows=int(counts[tc_mask].sum()), stream_rows=int(counts[st_mask].sum()),
+                  tc_experts=int(tc_mask.sum()), stream_experts=int(st_mask.sum()))
+        for k, v in st.items():
+            acc[k] = acc.get(k, 0) + v / len(xd)
+    stats = acc
+
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+
+    def barrier():
+        if dist:
+            tdist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if not dist:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=f"cuda:{device}")
+        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+        return float(t.item())
+
+    for i in range(warmup):
+        mod.forward(xd[i % N_INPUT_BATCHES], yd)
+    torch.cuda.synchronize()
+    status = mod.last_error()
+    if status != 0:
+        raise RuntimeError(f"device error during warm-up: {lmoe.lmoe_status_string(status)}")
+
+    # ---------------------------------------------------------------- device-timed region
+    lmoe.lmoe_set_profiling(mod.h, True, steps)
+    clocks = ClockSampler(_smi_id(device)) if with_clocks else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(steps):
+        mod.forward(xd[i % N_INPUT_BATCHES], yd)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop() if clocks else None
+    phases = lmoe.lmoe_phase_times(mod.h)
+    lmoe.lmoe_set_profiling(mod.h, False)
+    status = mod.last_error()
+    if status != 0:
+        raise RuntimeError(f"device error in the timed region: {lmoe.lmoe_status_string(status)}")
+    ms_max = max_over_ranks(ms)
+
+    # ---------------------------------------------------------------- end to end through host buffers
+    e2e = None
+    if with_e2e:
+        xh = [x.pin_memory() for x in xs]
+        yh = torch.empty_like(xh[0]).pin_memory()
+        for i in range(warmup):
+            mod.forward_host(xh[i % N_INPUT_BATCHES], yh)
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(steps):
+            mod.forward_host(xh[i % N_INPUT_BATCHES], yh)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(ev0.elapsed_time(ev1))
+        e2e = {"value": world * T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
+               "d2h_bytes_per_step": int(yh.numel() * yh.element_size()), "ms_per_step": e2e_ms / steps}
+
+    # ---------------------------------------------------------------- roofline of the dominant kernel
+    launches = sum(n for _, n in phases.values())
+    dom = max(phases, key=lambda k: phases[k][0])
+    dom_ms, dom_n = phases[dom]
+    flops, nbytes = phase_units(cfg, stats, T, dom)
+    per_launch_ms = dom_ms / max(dom_n, 1)
+    intensity = flops / max(nbytes, 1.0)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if "gemm" in dom and intensity >= ridge:
+        roof = {"bound": "tensor", "achieved": flops / (per_launch_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": nbytes / (per_launch_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["launch_ms"] = per_launch_ms
+    roof["algorithmic_per_launch"] = {"flops": flops, "bytes": nbytes}
+    roof["traffic"] = None
+    roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "")
+
+    F, B = layer_work(cfg, stats, T)
+    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+    layer_roof = {"flops": F, "bytes": B, "t_roof_us": t_roof * 1e6, "t_step_us": ms_max / steps * 1e3,
+                  "frac": t_roof / (ms_max / steps / 1e3),
+                  "bound": "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+    mod.close()
+    return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
+            "e2e": e2e, "clocks": clk, "stats": stats}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU) arm
+def oracle_rate(cfg, layer, budget_s: float, max_tokens: int):
+    """Tokens/s of the fp64 oracle on a bounded sample of the workload's tokens."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.forward(cfg, layer, x=layer["x"][:1], want=("y",))
+    one = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(max_tokens, budget_s / one * oracle.num_threads() * 0.8)))
+    t0 = time.perf_counter()
+    oracle.forward(cfg, layer, x=layer["x"][:n], want=("y",))
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, oracle.num_threads()
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    layer = synth.make_layer(cfg)
+    rate, n, dt, cores = oracle_rate(cfg, layer, budget_s, cfg.tokens)
+    return {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of the {cfg.tokens} tokens of {cfg.name}, fp64, {dt:.1f} s"}
+
+
+def run_reference(args, cfg, rank, world):
+    """The fp64 oracle as it stands, timed on the host cores (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    layer = synth.make_layer(cfg)
+    total_budget = 150.0
+    t0 = time.perf_counter()
+    oracle.forward(cfg, layer, x=layer["x"][:1], want=("y",))
+    one = max(time.perf_counter() - t0, 1e-4)
+    per_step = total_budget / max(args.steps + args.warmup, 1)
+    n = int(max(1, min(cfg.tokens, per_step / one * oracle.num_threads() * 0.8)))
+    for _ in range(args.warmup):
+        oracle.forward(cfg, layer, x=layer["x"][:n], want=("y",))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.forward(cfg, layer, x=layer["x"][:n], want=("y",))
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{n} of the {cfg.tokens} tokens of {cfg.name} per step, fp64"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def workload_config(cfg):
+    return {"workload": cfg.name, "tokens": cfg.tokens, "d": cfg.d, "latent": cfg.latent, "m": cfg.m,
+            "experts": cfg.n_ffn, "bypass_experts": [cfg.n_zero, cfg.n_copy, cfg.n_const], "top_k": cfg.top_k,
+            "act": ["relu2", "swiglu", "identity"][cfg.act], "projection": bool(cfg.has_proj),
+            "l2": "inputs larger than L2 (the touched expert weights, read every step, exceed the 126 MB L2)",
+            "parallelism": "replicas (tokens shard with no exchange)"}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="lmoe", choices=["lmoe", "reference"])
+    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    cfg = synth.WORKLOADS[args.workload]
+
+    if args.impl == "reference":
+        line = run_reference(args, cfg, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device(f"cuda:{local}"))
+    peaks = load_peaks()
+    try:
+        res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks)
+        secondary = None
+        if not args.no_secondary and args.workload != SECONDARY_WORKLOAD:
+            sc = synth.WORKLOADS[SECONDARY_WORKLOAD]
+            s_steps = max(3, min(args.steps, 20))
+            r2 = run_gpu(sc, s_steps, args.warmup, rank, world, local, peaks, with_e2e=False, with_clocks=False)
+            secondary = {"workload": sc.name, "tokens_per_s": world * sc.tokens * s_steps / (r2["ms"] / 1e3),
+                         "ms_per_step": r2["ms"] / s_steps, "roofline": r2["roofline"],
+                         "layer_roofline": r2["layer_roofline"],
+                         "phases_ms_per_step": {k: v[0] / s_steps for k, v in r2["phases"].items()}}
+    finally:
+        pass
+    if rank == 0:
+        T = cfg.tokens
+        value = world * T * args.steps / (res["ms"] / 1e3)
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": workload_config(cfg), "roofline": res["roofline"],
+                "layer_roofline": res["layer_roofline"], "e2e": res["e2e"], "gpu_launches": res["launches"],
+                "clocks": res["clocks"],
+                "phases_ms_per_step": {k: v[0] / args.steps for k, v in res["phases"].items()},
+                "routing": res["stats"]}
+        if secondary is not None:
+            line["secondary"] = secondary
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+        tdist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

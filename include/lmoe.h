@@ -1,0 +1,204 @@
+/*
+ * lmoe.h -- C ABI of the LatentMoE layer forward for NVIDIA B200 (sm_100a).
+ *
+ * The layer (per token t, tokens independent):
+ *   1. router logits l = W_r f_t (+ bias), f = x_t: the gate stays at the full
+ *      width d ("LatentMoE: How MoE Made a Key Paradigm Leap in 2026", section 2,
+ *      closing note); with latent_router = 1 the gate reads z_t instead
+ *      (the same section's step 2 reading "routing happens in the latent").
+ *   2. the top-K' logits (ties to the lower expert id) and their renormalised
+ *      softmax weights w.
+ *   3. z_t = W_down x_t, d -> latent ("How LatentMoE Works", step 1;
+ *      Nemotron-3 article section 2.2, Figure 3b).
+ *   4. per selected FFN expert e, in the latent width: o = W2_e act(W1_e z_t),
+ *      act = relu(u)^2 or silu(gate) * up ("How LatentMoE Works", step 2);
+ *      MoE++ zero / copy / constant experts return 0 / z_t / v_c without a GEMM
+ *      (Nemotron-3 article section 3.2, Figure 1).
+ *   5. yl_t = sum_k w_k o_k, aggregated in the latent width (Figure 3b).
+ *   6. y_t = x_t + W_up yl_t, latent -> d ("How LatentMoE Works", step 3).
+ * With has_proj = 0 (latent == d) there is no W_down / W_up: the standard MoE
+ * of Figure 3a, y_t = x_t + yl_t.
+ *
+ * Conventions for every entry point:
+ *   - all matrices are row-major; bf16 tensors are passed as `void *` (IEEE
+ *     bfloat16 bit patterns), fp32 as `float *`, ids as `int32_t *`;
+ *   - "device" pointers are CUDA global-memory addresses of the current
+ *     device; "host" pointers are ordinary (preferably pinned) host memory;
+ *   - every device pointer must be 16-byte aligned;
+ *   - the caller owns every buffer; the library never allocates device memory
+ *     and borrows the weights and the workspace for the handle's lifetime;
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream); work is
+ *     enqueued asynchronously, nothing in lmoe_forward synchronises the host;
+ *   - return values: LMOE_OK (0) or a negative LMOE_ERR_* status; a rejected
+ *     call enqueues no work.
+ */
+#ifndef LMOE_H
+#define LMOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LMOE_API __attribute__((visibility("default")))
+#else
+#define LMOE_API
+#endif
+
+#define LMOE_OK 0
+#define LMOE_ERR_INVALID_ARG (-1)       /* null / misaligned pointer, bad enum, x aliases y */
+#define LMOE_ERR_UNSUPPORTED_SHAPE (-2) /* see lmoe_config */
+#define LMOE_ERR_TOO_MANY_TOKENS (-3)   /* T > max_tokens, or T < 0 */
+#define LMOE_ERR_CUDA (-4)              /* a CUDA runtime / driver call failed */
+#define LMOE_ERR_TIMEOUT (-5)           /* device: a bounded wait inside a kernel gave up */
+#define LMOE_ERR_BAD_INDEX (-6)         /* device: an expert id outside [0, n_total) */
+#define LMOE_ERR_WORKSPACE (-7)         /* workspace missing or smaller than lmoe_workspace_bytes */
+
+#define LMOE_ACT_RELU2 0    /* h = relu(u)^2 (non-gated) */
+#define LMOE_ACT_SWIGLU 1   /* W1_e rows [0,m) gate, [m,2m) up: h = silu(gate) * up */
+#define LMOE_ACT_IDENTITY 2 /* h = u (test use) */
+
+/*
+ * Layer shape.  Constraints (else LMOE_ERR_UNSUPPORTED_SHAPE): d, latent and m
+ * multiples of 64 and at most 16384; 1 <= top_k <= min(32, n_total);
+ * n_total = n_experts + n_zero + n_copy + n_const <= 1024; n_experts >= 1;
+ * max_tokens >= 1; has_proj == 0 requires latent == d.
+ */
+typedef struct lmoe_config {
+    int32_t d;             /* model width */
+    int32_t latent;        /* latent width l (== d without projections) */
+    int32_t m;             /* expert hidden width */
+    int32_t n_experts;     /* routed FFN experts N' (ids 0 .. N'-1) */
+    int32_t top_k;         /* experts per token K' */
+    int32_t max_tokens;    /* largest T a forward may be called with */
+    int32_t act;           /* LMOE_ACT_* */
+    int32_t n_zero;        /* MoE++ zero experts (ids N' ..) */
+    int32_t n_copy;        /* MoE++ copy experts (ids after the zero experts) */
+    int32_t n_const;       /* MoE++ constant experts (last ids) */
+    int32_t has_proj;      /* 1: LatentMoE with W_down / W_up; 0: standard MoE */
+    int32_t latent_router; /* 1: the gate reads z (latent) instead of x (d) */
+} lmoe_config;
+
+/* Device pointers to the layer's weights (bf16 unless stated).  n_total as above. */
+typedef struct lmoe_weights {
+    const void *w_router;     /* [n_total, d], or [n_total, latent] with latent_router */
+    const float *router_bias; /* fp32 [n_total], added to the logits before selection; may be NULL */
+    const void *w_down;       /* [latent, d]; NULL when has_proj == 0 */
+    const void *w_up;         /* [d, latent]; NULL when has_proj == 0 */
+    const void *w1;           /* [n_experts, g*m, latent], g = 2 for SwiGLU else 1 */
+    const void *w2;           /* [n_experts, latent, m] */
+    const void *const_vecs;   /* [n_const, latent]; may be NULL when n_const == 0 */
+} lmoe_weights;
+
+/*
+ * Optional device buffers that receive copies of intermediate results after a
+ * forward (enqueued on the same stream).  Every field may be NULL.
+ */
+typedef struct lmoe_debug {
+    int32_t *topk_idx; /* [T, top_k] expert ids, slot order */
+    float *topk_w;     /* [T, top_k] renormalised weights */
+    int32_t *counts;   /* [n_total] tokens per expert */
+    int32_t *offsets;  /* [n_total + 1] exclusive scan of counts */
+    int32_t *perm;     /* [T * top_k] slot index t*K'+k at each sorted position */
+    void *z;           /* bf16 [T, latent] latent tokens (has_proj == 1) */
+    void *yl;          /* bf16 [T, latent] combined latent output (has_proj == 1) */
+    float *logits;     /* fp32 [T, n_total] router logits, bias not included */
+} lmoe_debug;
+
+typedef struct lmoe_handle lmoe_handle;
+
+/* Bytes of device workspace a handle for `cfg` needs (0 if cfg is invalid). */
+LMOE_API size_t lmoe_workspace_bytes(const lmoe_config *cfg);
+
+/*
+ * Validate `cfg`, record the weight pointers, carve `workspace` (device,
+ * 256-byte aligned, at least lmoe_workspace_bytes(cfg) bytes) and build the
+ * TMA descriptors of the weights.  Uses the current CUDA device.  On success
+ * *out receives a handle (host memory owned by the library until
+ * lmoe_destroy).
+ */
+LMOE_API int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *workspace, size_t workspace_bytes,
+                lmoe_handle **out);
+
+/*
+ * y = LatentMoE(x) for T tokens: x, y device bf16 [T, d], must not overlap.
+ * 0 <= T <= max_tokens (T == 0 enqueues nothing and accepts NULL x / y).  Asynchronous on `stream`;
+ * concurrent forwards on one handle share its workspace and must be ordered
+ * by the caller (same stream).  Device-side faults (a bounded wait that gave
+ * up, a bad expert id) are reported by lmoe_last_error after the stream is
+ * synchronised.  Output is bit-identical from run to run.  `dbg` may be NULL.
+ */
+LMOE_API int lmoe_forward(lmoe_handle *h, const void *x, void *y, int32_t T, void *stream, const lmoe_debug *dbg);
+
+/*
+ * The same forward on HOST buffers: copies x_host [T, d] into the workspace,
+ * runs the layer and copies y back to y_host [T, d], all on `stream`.  The
+ * host buffers should be pinned for the copies to be asynchronous; the caller
+ * synchronises the stream before reading y_host.
+ */
+LMOE_API int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t T, void *stream);
+
+/*
+ * Read and clear the device error word of the handle's workspace (blocking
+ * copy; synchronise the forward's stream first).  Returns LMOE_OK,
+ * LMOE_ERR_TIMEOUT or LMOE_ERR_BAD_INDEX (the first set, in that order), or
+ * LMOE_ERR_CUDA if the read failed.
+ */
+LMOE_API int lmoe_last_error(lmoe_handle *h);
+
+/* Release the handle (not the caller's buffers).  NULL is ignored. */
+LMOE_API void lmoe_destroy(lmoe_handle *h);
+
+/* Static English text of a status code. */
+LMOE_API const char *lmoe_status_string(int status);
+
+/*
+ * Kernel-phase timing.  With profiling on, every forward records CUDA events
+ * around each phase on its stream (at most `max_forwards` forwards are kept).
+ * lmoe_phase_times writes, for each phase, the summed milliseconds and the
+ * number of kernel launches over the kept forwards into ms[i] / launches[i]
+ * (arrays of lmoe_num_phases() entries; either may be NULL), then forgets
+ * them.  Synchronise the stream(s) first.  The phase names are static.
+ */
+LMOE_API int lmoe_set_profiling(lmoe_handle *h, int enable, int max_forwards);
+LMOE_API int lmoe_phase_times(lmoe_handle *h, float *ms, int32_t *launches);
+LMOE_API int lmoe_num_phases(void);
+LMOE_API const char *lmoe_phase_name(int phase);
+
+/*
+ * Sizes of the last forward's routing, read back from the device (blocking;
+ * synchronise first): out[0] = rows routed to FFN experts, out[1] = FFN
+ * experts with at least one row, out[2] = tensor-core M-tiles, out[3] =
+ * experts served by the weight-streaming path.  Used to compute the
+ * algorithmic work of a forward.
+ */
+LMOE_API int lmoe_routing_stats(lmoe_handle *h, int32_t *out4);
+
+/*
+ * Routing threshold: FFN experts with at most `rows` routed rows take the
+ * weight-streaming path (default 8, the maximum), the others the tensor-core
+ * grouped GEMM; 0 sends every expert to the tensor cores.
+ */
+LMOE_API int lmoe_set_small_rows(lmoe_handle *h, int32_t rows);
+
+/* Bound of every in-kernel wait, nanoseconds (default 1e9). */
+LMOE_API int lmoe_set_wait_timeout(lmoe_handle *h, uint64_t ns);
+
+/*
+ * Plain GEMM on the layer's tensor-core kernel: C[M,N] = A[M,K] * B[N,K]^T,
+ * bf16 in (device, row-major, K-major both), fp32 accumulate, bf16 out.
+ * K a multiple of 64 (<= 65536), N a multiple of 64, M >= 0.  `err_word` is a
+ * device int that collects device error bits (may be NULL: errors are then
+ * not reported).  Asynchronous on `stream`.
+ */
+LMOE_API int lmoe_gemm_bf16(const void *A, const void *B, void *C, int32_t M, int32_t N, int32_t K, void *stream,
+                   int *err_word);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LMOE_H */

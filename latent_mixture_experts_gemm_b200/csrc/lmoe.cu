@@ -1,0 +1,642 @@
+// lmoe.cu -- host side of the LatentMoE layer forward: argument checks, the
+// workspace plan, TMA descriptors and the launch sequence.  The C ABI is
+// declared in include/lmoe.h.
+//
+// Launch sequence of one forward (all on the caller's stream):
+//   router/projection GEMM (tcgen05) -> top-K' + softmax -> counting sort
+//   (bitmap, per-expert prefix, offsets + tile lists, scatter/gather) ->
+//   up GEMM + activation (tcgen05 grouped; weight streaming for experts with
+//   few rows) -> down GEMM (same split) -> combine in the latent width ->
+//   up-projection GEMM with the residual add (tcgen05).
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/lmoe.h"
+#include "moe_kernels.cuh"
+#include "tc_gemm.cuh"
+
+using namespace lmoe;
+
+namespace {
+
+// ------------------------------------------------------------------ driver entry point for TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool load_encode() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// bf16 matrix [rows, cols] with row pitch `ld` elements, box = box_rows x 64, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_rows) {
+    if (!load_encode() || rows == 0) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+int n_total(const lmoe_config& c) { return c.n_experts + c.n_zero + c.n_copy + c.n_const; }
+
+bool config_ok(const lmoe_config& c) {
+    auto dim_ok = [](int v) { return v >= 64 && v <= 16384 && v % 64 == 0; };
+    if (!dim_ok(c.d) || !dim_ok(c.latent) || !dim_ok(c.m)) return false;
+    if (c.n_experts < 1 || c.n_zero < 0 || c.n_copy < 0 || c.n_const < 0) return false;
+    const int nt = n_total(c);
+    if (nt > 1024) return false;
+    if (c.top_k < 1 || c.top_k > 32 || c.top_k > nt) return false;
+    if (c.max_tokens < 1 || static_cast<long long>(c.max_tokens) * c.top_k > (1LL << 30)) return false;
+    if (c.act < 0 || c.act > 2) return false;
+    if (c.has_proj != 0 && c.has_proj != 1) return false;
+    if (c.latent_router != 0 && c.latent_router != 1) return false;
+    if (!c.has_proj && c.latent != c.d) return false;
+    return true;
+}
+
+struct Plan {
+    size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
+        xin, yout, total;
+    int ld_logits, nwords, mt_max;
+};
+
+Plan make_plan(const lmoe_config& c) {
+    Plan p{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += round_up(bytes > 0 ? bytes : 1, 256);
+        return o;
+    };
+    const size_t T = c.max_tokens, K = c.top_k, L = c.latent, d = c.d, m = c.m;
+    const size_t nt = n_total(c);
+    const size_t R = T * K;
+    p.ld_logits = static_cast<int>(round_up(nt, 64));
+    p.nwords = static_cast<int>((T + 31) / 32);
+    p.mt_max = static_cast<int>((R + 127) / 128 + c.n_experts);
+    p.hdr = take(HDR_WORDS * 4);
+    p.logits = take(T * p.ld_logits * 4);
+    p.z = c.has_proj ? take(T * L * 2) : 0;
+    p.idx = take(T * K * 4);
+    p.w = take(T * K * 4);
+    p.bitmap = take(static_cast<size_t>(p.nwords) * nt * 4);
+    p.prefix = take(static_cast<size_t>(p.nwords) * nt * 4);
+    p.counts = take(nt * 4);
+    p.offsets = take((nt + 1) * 4);
+    p.perm = take(R * 4);
+    p.inv = take(R * 4);
+    p.mt_list = take(static_cast<size_t>(p.mt_max) * 16);
+    p.small_list = take(static_cast<size_t>(c.n_experts) * 16);
+    p.rows = take(R * L * 2);  // gathered expert inputs, then (reused) expert outputs
+    p.hbuf = take(R * m * 2);
+    p.yl = c.has_proj ? take(T * L * 2) : 0;
+    p.xin = take(T * d * 2);
+    p.yout = take(T * d * 2);
+    p.total = off;
+    return p;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+enum Phase : int { PH_ROUTER = 0, PH_TOPK, PH_DISPATCH, PH_UP_TC, PH_UP_STREAM, PH_DOWN_TC, PH_DOWN_STREAM, PH_COMBINE,
+                   PH_WUP, PH_COUNT };
+const char* kPhaseNames[PH_COUNT] = {"router_proj_gemm", "topk_softmax", "dispatch", "expert_up_gemm",
+                                     "expert_up_stream", "expert_down_gemm", "expert_down_stream", "combine",
+                                     "up_proj_gemm"};
+
+template <int BN, int EPI>
+bool set_smem_attr() {
+    return cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GemmCfg<BN>::SMEM_BYTES) == cudaSuccess;
+}
+
+bool set_all_smem_attrs() {
+    bool ok = true;
+    ok &= set_smem_attr<64, EPI_BF16>();
+    ok &= set_smem_attr<256, EPI_BF16>();
+    ok &= set_smem_attr<64, EPI_RESID>();
+    ok &= set_smem_attr<256, EPI_RESID>();
+    ok &= set_smem_attr<64, EPI_PROJ_ROUTER>();
+    ok &= set_smem_attr<256, EPI_PROJ_ROUTER>();
+    ok &= set_smem_attr<256, EPI_RELU2>();
+    ok &= set_smem_attr<256, EPI_SWIGLU>();
+    return ok;
+}
+
+template <int BN, int EPI>
+void launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args, int grid,
+                 cudaStream_t s) {
+    tc_gemm_kernel<BN, EPI><<<grid, 192, GemmCfg<BN>::SMEM_BYTES, s>>>(a, b, b2, args);
+}
+
+}  // namespace
+
+// ====================================================================== handle
+struct lmoe_handle {
+    lmoe_config c{};
+    lmoe_weights w{};
+    uint8_t* ws = nullptr;
+    Plan p{};
+    int n_tot = 0, g = 1, num_sms = 148, small_max = SMALL_MAX, device = 0;
+    unsigned long long timeout_ns = 1000000000ull;
+    // weight descriptors: router/projection operands for both column tiles, expert weights, workspace operands
+    CUtensorMap wdown64{}, wdown256{}, wr64{}, wr256{}, wup64{}, wup256{}, w1{}, w2{};
+    CUtensorMap a_rows{}, a_h{}, a_yl{}, a_z{};
+    // profiling
+    bool prof = false;
+    int prof_max = 0, prof_n = 0;
+    std::vector<cudaEvent_t> ev;
+    std::vector<int> launches;
+    template <typename T>
+    T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+};
+
+namespace {
+
+struct PhaseScope {
+    lmoe_handle* h;
+    int ph;
+    cudaStream_t s;
+    int n_launch;
+    bool on;
+    PhaseScope(lmoe_handle* h_, int ph_, cudaStream_t s_, int n) : h(h_), ph(ph_), s(s_), n_launch(n) {
+        on = h->prof && h->prof_n < h->prof_max;
+        if (on) cudaEventRecord(h->ev[(static_cast<size_t>(h->prof_n) * PH_COUNT + ph) * 2], s);
+    }
+    ~PhaseScope() {
+        if (on) {
+            cudaEventRecord(h->ev[(static_cast<size_t>(h->prof_n) * PH_COUNT + ph) * 2 + 1], s);
+            h->launches[static_cast<size_t>(h->prof_n) * PH_COUNT + ph] = n_launch;
+        }
+    }
+};
+
+void free_events(lmoe_handle* h) {
+    for (cudaEvent_t e : h->ev)
+        if (e) cudaEventDestroy(e);
+    h->ev.clear();
+    h->launches.clear();
+    h->prof_max = h->prof_n = 0;
+}
+
+int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, const lmoe_debug* dbg) {
+    const lmoe_config& c = h->c;
+    const Plan& p = h->p;
+    const int K = c.top_k, L = c.latent, d = c.d, m = c.m, nt = h->n_tot;
+    const bool proj = c.has_proj != 0;
+    int* hdr = h->at<int>(p.hdr);
+    float* logits = h->at<float>(p.logits);
+    __nv_bfloat16* z = proj ? h->at<__nv_bfloat16>(p.z) : nullptr;
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(y);
+    const __nv_bfloat16* feat = proj ? z : xb;  // what the experts read (latent z, or x for the standard MoE)
+    int32_t* idx = h->at<int32_t>(p.idx);
+    float* wts = h->at<float>(p.w);
+    __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
+    __nv_bfloat16* hbuf = h->at<__nv_bfloat16>(p.hbuf);
+    int4* mt_list = h->at<int4>(p.mt_list);
+    int4* small_list = h->at<int4>(p.small_list);
+
+    CUtensorMap a_x;
+    if (!make_map(&a_x, x, T, d, d, 128)) return LMOE_ERR_CUDA;
+    const int m_tiles = (T + 127) / 128;
+
+    GemmArgs base{};
+    base.err = hdr + HDR_ERR;
+    base.timeout_ns = h->timeout_ns;
+
+    // ---------------------------------------------------------------- router (+ W_down)
+    {
+        const bool fused = proj && !c.latent_router;
+        const int n256 = (fused ? (L + 255) / 256 : 0) + (nt + 255) / 256;
+        const bool big = m_tiles * n256 >= h->num_sms;
+        const int n_gemm = (proj && c.latent_router) ? 2 : 1;
+        PhaseScope ps(h, PH_ROUTER, s, n_gemm);
+        if (proj && c.latent_router) {
+            GemmArgs a = base;
+            a.M = T;
+            a.K = d;
+            a.N0 = L;
+            a.out0 = z;
+            a.ld0 = L;
+            if (big) {
+                a.n_tiles = (L + 255) / 256;
+                launch_gemm<256, EPI_BF16>(a_x, h->wdown256, h->wdown256, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+            } else {
+                a.n_tiles = (L + 63) / 64;
+                launch_gemm<64, EPI_BF16>(a_x, h->wdown64, h->wdown64, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+            }
+        }
+        GemmArgs a = base;
+        a.M = T;
+        a.K = c.latent_router ? L : d;
+        a.N0 = fused ? L : 0;
+        a.N1 = nt;
+        a.out0 = z;
+        a.ld0 = L;
+        a.out1 = logits;
+        a.ld1 = p.ld_logits;
+        const CUtensorMap& A = (proj && c.latent_router) ? h->a_z : a_x;
+        if (big) {
+            a.n_tiles0 = fused ? (L + 255) / 256 : 0;
+            a.n_tiles = a.n_tiles0 + (nt + 255) / 256;
+            launch_gemm<256, EPI_PROJ_ROUTER>(A, fused ? h->wdown256 : h->wr256, h->wr256, a,
+                                              std::min(h->num_sms, m_tiles * a.n_tiles), s);
+        } else {
+            a.n_tiles0 = fused ? (L + 63) / 64 : 0;
+            a.n_tiles = a.n_tiles0 + (nt + 63) / 64;
+            launch_gemm<64, EPI_PROJ_ROUTER>(A, fused ? h->wdown64 : h->wr64, h->wr64, a,
+                                             std::min(h->num_sms, m_tiles * a.n_tiles), s);
+        }
+    }
+    // ---------------------------------------------------------------- top-K' + softmax
+    {
+        PhaseScope ps(h, PH_TOPK, s, 1);
+        const int npl = (nt + 31) / 32;
+        const dim3 grid((T + 7) / 8), block(256);
+        const float* bias = h->w.router_bias;
+        if (npl <= 1) topk_softmax_kernel<1><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
+        else if (npl <= 2) topk_softmax_kernel<2><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
+        else if (npl <= 4) topk_softmax_kernel<4><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
+        else if (npl <= 8) topk_softmax_kernel<8><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
+        else if (npl <= 16) topk_softmax_kernel<16><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
+        else topk_softmax_kernel<32><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
+    }
+    // ---------------------------------------------------------------- counting sort by expert
+    {
+        PhaseScope ps(h, PH_DISPATCH, s, 4);
+        const int nwords = (T + 31) / 32;
+        uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
+        uint32_t* prefix = h->at<uint32_t>(p.prefix);
+        int* counts = h->at<int>(p.counts);
+        int* offsets = h->at<int>(p.offsets);
+        dispatch_bitmap_kernel<<<(nwords + 7) / 8, 256, 8 * nt * 4, s>>>(idx, T, K, nt, bitmap, hdr);
+        dispatch_expert_scan_kernel<<<(nt + 7) / 8, 256, 0, s>>>(bitmap, T, nt, prefix, counts);
+        dispatch_offsets_kernel<<<1, 1024, 0, s>>>(counts, nt, c.n_experts, h->small_max, offsets, mt_list, small_list,
+                                                   hdr);
+        const long slots = static_cast<long>(T) * K;
+        dispatch_scatter_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
+            idx, T, K, nt, c.n_experts, bitmap, prefix, offsets, feat, L, L, rows, L, h->at<int32_t>(p.perm),
+            h->at<int32_t>(p.inv));
+    }
+    // ---------------------------------------------------------------- expert up (+ activation)
+    {
+        PhaseScope ps(h, PH_UP_TC, s, 1);
+        GemmArgs a = base;
+        a.K = L;
+        a.mt_list = mt_list;
+        a.mt_count = hdr + HDR_MT;
+        a.b_rows_per_expert = h->g * m;
+        a.up_offset = m;
+        a.N0 = m;
+        a.out0 = hbuf;
+        a.ld0 = m;
+        if (c.act == LMOE_ACT_SWIGLU) {
+            a.n_tiles = (m + 127) / 128;
+            launch_gemm<256, EPI_SWIGLU>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
+        } else if (c.act == LMOE_ACT_RELU2) {
+            a.n_tiles = (m + 255) / 256;
+            launch_gemm<256, EPI_RELU2>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
+        } else {
+            a.n_tiles = (m + 255) / 256;
+            launch_gemm<256, EPI_BF16>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
+        }
+    }
+    if (h->small_max > 0) {
+        PhaseScope ps(h, PH_UP_STREAM, s, 1);
+        const int grid = h->num_sms * 3;
+        if (c.act == LMOE_ACT_SWIGLU)
+            expert_stream_kernel<GEMV_SWIGLU><<<grid, GEMV_THREADS, 0, s>>>(
+                rows, L, static_cast<const __nv_bfloat16*>(h->w.w1), 2 * m, m, L, m, hbuf, m, small_list, hdr + HDR_NSMALL);
+        else if (c.act == LMOE_ACT_RELU2)
+            expert_stream_kernel<GEMV_RELU2><<<grid, GEMV_THREADS, 0, s>>>(
+                rows, L, static_cast<const __nv_bfloat16*>(h->w.w1), m, 0, L, m, hbuf, m, small_list, hdr + HDR_NSMALL);
+        else
+            expert_stream_kernel<GEMV_NONE><<<grid, GEMV_THREADS, 0, s>>>(
+                rows, L, static_cast<const __nv_bfloat16*>(h->w.w1), m, 0, L, m, hbuf, m, small_list, hdr + HDR_NSMALL);
+    }
+    // ---------------------------------------------------------------- expert down (output reuses the gathered rows)
+    {
+        PhaseScope ps(h, PH_DOWN_TC, s, 1);
+        GemmArgs a = base;
+        a.K = m;
+        a.mt_list = mt_list;
+        a.mt_count = hdr + HDR_MT;
+        a.b_rows_per_expert = L;
+        a.N0 = L;
+        a.out0 = rows;
+        a.ld0 = L;
+        a.n_tiles = (L + 255) / 256;
+        launch_gemm<256, EPI_BF16>(h->a_h, h->w2, h->w2, a, h->num_sms, s);
+    }
+    if (h->small_max > 0) {
+        PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
+        expert_stream_kernel<GEMV_NONE><<<h->num_sms * 3, GEMV_THREADS, 0, s>>>(
+            hbuf, m, static_cast<const __nv_bfloat16*>(h->w.w2), L, 0, m, L, rows, L, small_list, hdr + HDR_NSMALL);
+    }
+    // ---------------------------------------------------------------- combine in the latent width
+    {
+        PhaseScope ps(h, PH_COMBINE, s, 1);
+        __nv_bfloat16* out = proj ? h->at<__nv_bfloat16>(p.yl) : yb;
+        combine_kernel<<<T, 128, 0, s>>>(rows, L, h->at<int32_t>(p.inv), idx, wts, feat, L,
+                                          static_cast<const __nv_bfloat16*>(h->w.const_vecs), T, K, L, c.n_experts,
+                                          c.n_zero, c.n_copy, proj ? nullptr : xb, d, out, proj ? L : d);
+    }
+    // ---------------------------------------------------------------- W_up + residual
+    if (proj) {
+        PhaseScope ps(h, PH_WUP, s, 1);
+        GemmArgs a = base;
+        a.M = T;
+        a.K = L;
+        a.N0 = d;
+        a.out0 = yb;
+        a.ld0 = d;
+        a.resid = xb;
+        a.ld_resid = d;
+        if (m_tiles * ((d + 255) / 256) >= h->num_sms) {
+            a.n_tiles = (d + 255) / 256;
+            launch_gemm<256, EPI_RESID>(h->a_yl, h->wup256, h->wup256, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+        } else {
+            a.n_tiles = (d + 63) / 64;
+            launch_gemm<64, EPI_RESID>(h->a_yl, h->wup64, h->wup64, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+        }
+    }
+    if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
+    if (h->prof && h->prof_n < h->prof_max) ++h->prof_n;
+
+    if (dbg != nullptr) {
+        bool ok = true;
+        auto cp = [&](void* dst, const void* src, size_t bytes) {
+            if (dst) ok &= cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+        };
+        cp(dbg->topk_idx, idx, static_cast<size_t>(T) * K * 4);
+        cp(dbg->topk_w, wts, static_cast<size_t>(T) * K * 4);
+        cp(dbg->counts, h->at<int>(p.counts), static_cast<size_t>(nt) * 4);
+        cp(dbg->offsets, h->at<int>(p.offsets), static_cast<size_t>(nt + 1) * 4);
+        cp(dbg->perm, h->at<int32_t>(p.perm), static_cast<size_t>(T) * K * 4);
+        if (proj) {
+            cp(dbg->z, z, static_cast<size_t>(T) * L * 2);
+            cp(dbg->yl, h->at<__nv_bfloat16>(p.yl), static_cast<size_t>(T) * L * 2);
+        }
+        if (dbg->logits)
+            ok &= cudaMemcpy2DAsync(dbg->logits, static_cast<size_t>(nt) * 4, logits, static_cast<size_t>(p.ld_logits) * 4,
+                                    static_cast<size_t>(nt) * 4, T, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
+        if (!ok) return LMOE_ERR_CUDA;
+    }
+    return LMOE_OK;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+size_t lmoe_workspace_bytes(const lmoe_config* cfg) {
+    if (cfg == nullptr || !config_ok(*cfg)) return 0;
+    return make_plan(*cfg).total;
+}
+
+int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, size_t workspace_bytes,
+                lmoe_handle** out) {
+    if (out == nullptr || cfg == nullptr || w == nullptr) return LMOE_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!config_ok(*cfg)) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    const lmoe_config& c = *cfg;
+    const Plan p = make_plan(c);
+    if (workspace == nullptr || workspace_bytes < p.total) return LMOE_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return LMOE_ERR_INVALID_ARG;
+    if (w->w_router == nullptr || w->w1 == nullptr || w->w2 == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (c.has_proj && (w->w_down == nullptr || w->w_up == nullptr)) return LMOE_ERR_INVALID_ARG;
+    if (c.n_const > 0 && w->const_vecs == nullptr) return LMOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {w->w_router, w->router_bias, w->w_down, w->w_up, w->w1, w->w2, w->const_vecs};
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return LMOE_ERR_INVALID_ARG;
+
+    lmoe_handle* h = new (std::nothrow) lmoe_handle();
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    h->c = c;
+    h->w = *w;
+    h->ws = static_cast<uint8_t*>(workspace);
+    h->p = p;
+    h->n_tot = n_total(c);
+    h->g = c.act == LMOE_ACT_SWIGLU ? 2 : 1;
+    if (cudaGetDevice(&h->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
+        !set_all_smem_attrs()) {
+        delete h;
+        return LMOE_ERR_CUDA;
+    }
+    const int L = c.latent, d = c.d, m = c.m, nt = h->n_tot;
+    const int fdim = c.latent_router ? L : d;
+    const uint64_t R = static_cast<uint64_t>(c.max_tokens) * c.top_k;
+    bool ok = true;
+    ok &= make_map(&h->wr64, w->w_router, nt, fdim, fdim, 64);
+    ok &= make_map(&h->wr256, w->w_router, nt, fdim, fdim, 256);
+    if (c.has_proj) {
+        ok &= make_map(&h->wdown64, w->w_down, L, d, d, 64);
+        ok &= make_map(&h->wdown256, w->w_down, L, d, d, 256);
+        ok &= make_map(&h->wup64, w->w_up, d, L, L, 64);
+        ok &= make_map(&h->wup256, w->w_up, d, L, L, 256);
+        ok &= make_map(&h->a_yl, h->at<void>(p.yl), c.max_tokens, L, L, 128);
+        ok &= make_map(&h->a_z, h->at<void>(p.z), c.max_tokens, L, L, 128);
+    }
+    ok &= make_map(&h->w1, w->w1, static_cast<uint64_t>(c.n_experts) * h->g * m, L, L, h->g == 2 ? 128 : 256);
+    ok &= make_map(&h->w2, w->w2, static_cast<uint64_t>(c.n_experts) * L, m, m, 256);
+    ok &= make_map(&h->a_rows, h->at<void>(p.rows), R, L, L, 128);
+    ok &= make_map(&h->a_h, h->at<void>(p.hbuf), R, m, m, 128);
+    ok &= cudaMemset(h->at<void>(p.hdr), 0, HDR_WORDS * 4) == cudaSuccess;
+    if (!ok) {
+        delete h;
+        return LMOE_ERR_CUDA;
+    }
+    *out = h;
+    return LMOE_OK;
+}
+
+int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, void* stream, const lmoe_debug* dbg) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
+    if (T == 0) return LMOE_OK;
+    if (x == nullptr || y == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return LMOE_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(T) * h->c.d * 2;
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+    if (xa < ya + bytes && ya < xa + bytes) return LMOE_ERR_INVALID_ARG;
+    return run_forward(h, x, y, T, static_cast<cudaStream_t>(stream), dbg);
+}
+
+int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, void* stream) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
+    if (T == 0) return LMOE_OK;
+    if (x_host == nullptr || y_host == nullptr) return LMOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t bytes = static_cast<size_t>(T) * h->c.d * 2;
+    void* xin = h->at<void>(h->p.xin);
+    void* yout = h->at<void>(h->p.yout);
+    if (cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return LMOE_ERR_CUDA;
+    const int rc = run_forward(h, xin, yout, T, s, nullptr);
+    if (rc != LMOE_OK) return rc;
+    if (cudaMemcpyAsync(y_host, yout, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return LMOE_ERR_CUDA;
+    return LMOE_OK;
+}
+
+int lmoe_last_error(lmoe_handle* h) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    int err = 0;
+    int* dev = h->at<int>(h->p.hdr) + HDR_ERR;
+    if (cudaMemcpy(&err, dev, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
+    if (err != 0 && cudaMemset(dev, 0, 4) != cudaSuccess) return LMOE_ERR_CUDA;
+    if (err & DEVERR_TIMEOUT) return LMOE_ERR_TIMEOUT;
+    if (err & DEVERR_BAD_INDEX) return LMOE_ERR_BAD_INDEX;
+    return LMOE_OK;
+}
+
+void lmoe_destroy(lmoe_handle* h) {
+    if (h == nullptr) return;
+    free_events(h);
+    delete h;
+}
+
+const char* lmoe_status_string(int status) {
+    switch (status) {
+        case LMOE_OK: return "ok";
+        case LMOE_ERR_INVALID_ARG: return "invalid argument";
+        case LMOE_ERR_UNSUPPORTED_SHAPE: return "unsupported layer shape";
+        case LMOE_ERR_TOO_MANY_TOKENS: return "token count outside [0, max_tokens]";
+        case LMOE_ERR_CUDA: return "CUDA call failed";
+        case LMOE_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
+        case LMOE_ERR_BAD_INDEX: return "expert id out of range";
+        case LMOE_ERR_WORKSPACE: return "workspace missing or too small";
+        default: return "unknown status";
+    }
+}
+
+int lmoe_set_profiling(lmoe_handle* h, int enable, int max_forwards) {
+    if (h == nullptr || (enable && max_forwards < 1)) return LMOE_ERR_INVALID_ARG;
+    free_events(h);
+    h->prof = enable != 0;
+    if (!h->prof) return LMOE_OK;
+    const size_t n = static_cast<size_t>(max_forwards) * PH_COUNT;
+    h->ev.assign(2 * n, nullptr);
+    h->launches.assign(n, 0);
+    for (auto& e : h->ev)
+        if (cudaEventCreate(&e) != cudaSuccess) {
+            free_events(h);
+            h->prof = false;
+            return LMOE_ERR_CUDA;
+        }
+    h->prof_max = max_forwards;
+    h->prof_n = 0;
+    return LMOE_OK;
+}
+
+int lmoe_phase_times(lmoe_handle* h, float* ms, int32_t* launches) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    std::vector<float> acc(PH_COUNT, 0.f);
+    std::vector<int32_t> nl(PH_COUNT, 0);
+    for (int f = 0; f < h->prof_n; ++f)
+        for (int ph = 0; ph < PH_COUNT; ++ph) {
+            const size_t i = static_cast<size_t>(f) * PH_COUNT + ph;
+            if (h->launches[i] == 0) continue;
+            float t = 0.f;
+            if (cudaEventElapsedTime(&t, h->ev[2 * i], h->ev[2 * i + 1]) != cudaSuccess) return LMOE_ERR_CUDA;
+            acc[ph] += t;
+            nl[ph] += h->launches[i];
+            h->launches[i] = 0;
+        }
+    h->prof_n = 0;
+    for (int ph = 0; ph < PH_COUNT; ++ph) {
+        if (ms) ms[ph] = acc[ph];
+        if (launches) launches[ph] = nl[ph];
+    }
+    return LMOE_OK;
+}
+
+int lmoe_num_phases(void) { return PH_COUNT; }
+
+const char* lmoe_phase_name(int phase) { return (phase >= 0 && phase < PH_COUNT) ? kPhaseNames[phase] : nullptr; }
+
+int lmoe_routing_stats(lmoe_handle* h, int32_t* out4) {
+    if (h == nullptr || out4 == nullptr) return LMOE_ERR_INVALID_ARG;
+    int hdr[HDR_WORDS];
+    std::vector<int> counts(h->n_tot);
+    if (cudaMemcpy(hdr, h->at<int>(h->p.hdr), sizeof hdr, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(counts.data(), h->at<int>(h->p.counts), counts.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return LMOE_ERR_CUDA;
+    int touched = 0;
+    for (int e = 0; e < h->c.n_experts; ++e) touched += counts[e] > 0;
+    out4[0] = hdr[HDR_ROWS];
+    out4[1] = touched;
+    out4[2] = hdr[HDR_MT];
+    out4[3] = hdr[HDR_NSMALL];
+    return LMOE_OK;
+}
+
+int lmoe_set_small_rows(lmoe_handle* h, int32_t rows) {
+    if (h == nullptr || rows < 0 || rows > SMALL_MAX) return LMOE_ERR_INVALID_ARG;
+    h->small_max = rows;
+    return LMOE_OK;
+}
+
+int lmoe_set_wait_timeout(lmoe_handle* h, uint64_t ns) {
+    if (h == nullptr || ns == 0) return LMOE_ERR_INVALID_ARG;
+    h->timeout_ns = ns;
+    return LMOE_OK;
+}
+
+int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, int32_t K, void* stream, int* err_word) {
+    if (A == nullptr || B == nullptr || C == nullptr || err_word == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (M < 0 || N < 64 || N % 64 != 0 || K < 64 || K % 64 != 0 || K > 65536) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(A) || !aligned16(B) || !aligned16(C)) return LMOE_ERR_INVALID_ARG;
+    if (M == 0) return LMOE_OK;
+    static std::once_flag attr_once;
+    static bool attr_ok = false;
+    std::call_once(attr_once, [] { attr_ok = set_all_smem_attrs(); });
+    if (!attr_ok) return LMOE_ERR_CUDA;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LMOE_ERR_CUDA;
+    const int m_tiles = (M + 127) / 128;
+    const bool big = static_cast<long long>(m_tiles) * ((N + 255) / 256) >= sms;
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, A, M, K, K, 128) || !make_map(&mb, B, N, K, K, big ? 256 : 64)) return LMOE_ERR_CUDA;
+    GemmArgs a{};
+    a.M = M;
+    a.K = K;
+    a.N0 = N;
+    a.out0 = static_cast<__nv_bfloat16*>(C);
+    a.ld0 = N;
+    a.err = err_word;
+    a.timeout_ns = 1000000000ull;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (big) {
+        a.n_tiles = (N + 255) / 256;
+        launch_gemm<256, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);
+    } else {
+        a.n_tiles = (N + 63) / 64;
+        launch_gemm<64, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);
+    }
+    return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+}  // extern "C"

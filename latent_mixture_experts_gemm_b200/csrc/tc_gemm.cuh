@@ -1,0 +1,350 @@
+// tc_gemm.cuh -- persistent tcgen05 GEMM for sm_100a: D[128 x BN] tiles of A[M,K] * B[N,K]^T.
+//
+// Both operands are bf16 and K-major (rows contiguous along K); TMA brings
+// 128 x 64 A tiles and BN x 64 B tiles into shared memory with the 128-byte
+// swizzle; one thread issues tcgen05.mma (M=128, N=BN, K=16) into a tensor
+// memory accumulator; four epilogue warps read the accumulator back with
+// tcgen05.ld and apply the fused epilogue.  Two accumulators (2 x BN TMEM
+// columns) let the epilogue of tile i overlap the main loop of tile i+1.
+//
+// Warp roles (192 threads): warp 0 = TMA producer, warp 1 = TMEM owner and MMA
+// issuer, warps 2..5 = epilogue (warp w reads TMEM lanes 32*(w%4) .. +31).
+//
+// Tile maps:
+//   dense   -- tiles over ceil(M/128) x n_tiles, n fastest (CTAs working at
+//              the same time share the A rows through L2);
+//   grouped -- an M-tile list built on the device (expert, first row, rows);
+//              tile t -> list entry t / n_tiles, column tile t % n_tiles; the
+//              B rows are those of the entry's expert.
+#pragma once
+#include "ptx.cuh"
+
+namespace lmoe {
+
+enum Epi : int {
+    EPI_BF16 = 0,         // out0 = bf16(acc)
+    EPI_RELU2 = 1,        // out0 = bf16(relu(acc)^2)
+    EPI_SWIGLU = 2,       // accumulator columns [0,BN/2) gate, [BN/2,BN) up: out0 = bf16(silu(g) * u)
+    EPI_RESID = 3,        // out0 = bf16(acc + resid)
+    EPI_PROJ_ROUTER = 4,  // column tiles < n_tiles0: bf16 -> out0; the rest: fp32 -> out1 (masked to N1)
+};
+
+struct GemmArgs {
+    int M;                 // dense: rows of A
+    int K;                 // reduction length, multiple of 64
+    int n_tiles;           // column tiles per M-tile
+    int n_tiles0;          // EPI_PROJ_ROUTER: column tiles of segment 0
+    int N0;                // valid output columns of out0 (segment 0)
+    int N1;                // EPI_PROJ_ROUTER: valid columns of out1
+    const int4* mt_list;   // grouped: {expert, first row, rows, 0}; nullptr => dense
+    const int* mt_count;   // grouped: number of list entries (device)
+    int b_rows_per_expert; // grouped: rows of B per expert
+    int up_offset;         // EPI_SWIGLU: row offset of the up half inside an expert
+    __nv_bfloat16* out0;
+    int ld0;
+    float* out1;
+    int ld1;
+    const __nv_bfloat16* resid;
+    int ld_resid;
+    int* err;
+    unsigned long long timeout_ns;
+};
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int BM = 128;
+    static constexpr int BK = 64;
+    static constexpr int A_BYTES = BM * BK * 2;
+    static constexpr int B_BYTES = BN * BK * 2;
+    static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
+    static constexpr int TMEM_COLS = 2 * BN;  // power of two for BN in {64,128,256}
+    static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+struct TileJob {
+    int a_row0, rows;   // A rows (and output rows) of this tile
+    int b_row0, b_row1; // B rows of the (first, second) half
+    int col0;           // first output column
+    int seg;            // EPI_PROJ_ROUTER: 0 latent columns, 1 router columns
+};
+
+template <int BN, int EPI>
+__device__ __forceinline__ void tile_job(const GemmArgs& a, int t, TileJob& j) {
+    const int mt = t / a.n_tiles, nt = t % a.n_tiles;
+    j.seg = 0;
+    if (a.mt_list != nullptr) {
+        const int4 e = a.mt_list[mt];
+        j.a_row0 = e.y;
+        j.rows = e.z;
+        if (EPI == EPI_SWIGLU) {
+            j.col0 = nt * (BN / 2);
+            j.b_row0 = e.x * a.b_rows_per_expert + j.col0;
+            j.b_row1 = j.b_row0 + a.up_offset;
+        } else {
+            j.col0 = nt * BN;
+            j.b_row0 = e.x * a.b_rows_per_expert + j.col0;
+            j.b_row1 = 0;
+        }
+    } else {
+        j.a_row0 = mt * 128;
+        j.rows = min(128, a.M - j.a_row0);
+        if (EPI == EPI_PROJ_ROUTER && nt >= a.n_tiles0) {
+            j.seg = 1;
+            j.col0 = (nt - a.n_tiles0) * BN;
+        } else {
+            j.col0 = (EPI == EPI_SWIGLU) ? nt * (BN / 2) : nt * BN;
+        }
+        j.b_row0 = j.col0;
+        j.b_row1 = j.col0 + a.up_offset;
+    }
+}
+
+template <int BN>
+__device__ __forceinline__ int total_tiles(const GemmArgs& a) {
+    if (a.mt_list != nullptr) return (*a.mt_count) * a.n_tiles;
+    return ((a.M + 127) / 128) * a.n_tiles;
+}
+
+// Bound of the waits that drain in-flight copies and MMAs before the CTA
+// exits: never shorter than 200 ms, whatever the configured wait bound.
+__device__ __forceinline__ uint64_t drain_ns(const GemmArgs& a) {
+    return a.timeout_ns > 200000000ull ? a.timeout_ns : 200000000ull;
+}
+
+__device__ __forceinline__ float act_relu2(float v) {
+    const float r = fmaxf(v, 0.0f);
+    return r * r;
+}
+__device__ __forceinline__ float act_silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
+
+template <int BN, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
+    using C = GemmCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int ntiles = total_tiles<BN>(args);
+    if (static_cast<int>(blockIdx.x) >= ntiles) return;  // no tile for this CTA: skip TMEM and barrier set-up
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 4);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (EPI == EPI_PROJ_ROUTER) tma_prefetch_desc(&tmB2);
+    }
+    if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int nkb = args.K / C::BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer
+            uint32_t kc = 0;
+            uint32_t last_parity[C::STAGES];
+            bool issued[C::STAGES];
+            for (int s = 0; s < C::STAGES; ++s) issued[s] = false, last_parity[s] = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+                TileJob j;
+                tile_job<BN, EPI>(args, t, j);
+                const CUtensorMap* bmap = (EPI == EPI_PROJ_ROUTER && j.seg == 1) ? &tmB2 : &tmB;
+                for (int kb = 0; kb < nkb; ++kb, ++kc) {
+                    const int s = kc % C::STAGES;
+                    const uint32_t ph = (kc / C::STAGES) & 1;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.err, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+                    tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * C::BK, j.a_row0);
+                    if (EPI == EPI_SWIGLU) {
+                        tma_load_2d(sB + s * C::B_BYTES, bmap, &full[s], kb * C::BK, j.b_row0);
+                        tma_load_2d(sB + s * C::B_BYTES + C::B_BYTES / 2, bmap, &full[s], kb * C::BK, j.b_row1);
+                    } else {
+                        tma_load_2d(sB + s * C::B_BYTES, bmap, &full[s], kb * C::BK, j.b_row0);
+                    }
+                    issued[s] = true;
+                    last_parity[s] = ph;
+                }
+            }
+            // Never leave a copy in flight into shared memory: wait for the last
+            // load issued on each stage (immediate when it was consumed).
+            for (int s = 0; s < C::STAGES; ++s)
+                if (issued[s]) {
+                    int no_abort = 0;
+                    mbar_wait_bounded(&full[s], last_parity[s], &no_abort, args.err, drain_ns(args));
+                }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ------------------------------------------------ MMA issuer
+            constexpr uint32_t idesc = umma_idesc_bf16(128, BN);
+            uint32_t kc = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+                const int buf = it & 1;
+                const uint32_t use = (it >> 1) & 1;
+                if (!mbar_wait_bounded(&tempty[buf], use ^ 1, abort_flag, args.err, args.timeout_ns)) break;
+                tc_fence_after();
+                const uint32_t dtmem = tmem_base + buf * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++kc) {
+                    const int s = kc % C::STAGES;
+                    const uint32_t ph = (kc / C::STAGES) & 1;
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, args.err, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = umma_desc_sw128(smem_u32(sA + s * C::A_BYTES));
+                    const uint64_t bd = umma_desc_sw128(smem_u32(sB + s * C::B_BYTES));
+#pragma unroll
+                    for (int kk = 0; kk < C::BK / 16; ++kk)
+                        umma_bf16(dtmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&empty[s]);
+                }
+                if (ok) umma_commit(&tfull[buf]);
+            }
+            // Wait for every MMA this thread issued before TMEM can be released.
+            umma_commit(mma_done);
+            int no_abort = 0;
+            mbar_wait_bounded(mma_done, 0, &no_abort, args.err, drain_ns(args));
+        }
+    } else {
+        // ---------------------------------------------------- epilogue
+        const int quad = warp & 3;
+        const int row_in_tile = quad * 32 + lane;
+        int it = 0;
+        for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+            TileJob j;
+            tile_job<BN, EPI>(args, t, j);
+            const int buf = it & 1;
+            const uint32_t use = (it >> 1) & 1;
+            // One lane waits and the verdict is broadcast, so the whole warp
+            // either reads the accumulator (tcgen05.ld is warp-collective) or leaves.
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(&tfull[buf], use, abort_flag, args.err, args.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quad * 32) << 16);
+            const bool row_ok = row_in_tile < j.rows;
+            const size_t row = static_cast<size_t>(j.a_row0) + row_in_tile;
+            if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < BN / 2; c += 32) {
+                    uint32_t g[32], u[32];
+                    tmem_ld_32x32b_x32(tbase + c, g);
+                    tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
+                    tmem_ld_wait();
+                    const int col = j.col0 + c;
+                    if (row_ok && col < args.N0) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16x2(act_silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                                act_silu_mul(__uint_as_float(g[2 * i + 1]),
+                                                             __uint_as_float(u[2 * i + 1])));
+                        uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < BN; c += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tbase + c, v);
+                    tmem_ld_wait();
+                    const int col = j.col0 + c;
+                    if (!row_ok) continue;
+                    if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
+                        float* dst = args.out1 + row * args.ld1 + col;
+                        if (col + 32 <= args.N1) {
+                            float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (col + i < args.N1) dst[i] = __uint_as_float(v[i]);
+                        }
+                        continue;
+                    }
+                    if (col >= args.N0) continue;
+                    float f[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+                    if (EPI == EPI_RELU2) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
+                    }
+                    if (EPI == EPI_RESID) {
+                        const uint4* rs = reinterpret_cast<const uint4*>(args.resid + row * args.ld_resid + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint4 q = rs[i];
+                            f[8 * i + 0] += bf16lo(q.x);
+                            f[8 * i + 1] += bf16hi(q.x);
+                            f[8 * i + 2] += bf16lo(q.y);
+                            f[8 * i + 3] += bf16hi(q.y);
+                            f[8 * i + 4] += bf16lo(q.z);
+                            f[8 * i + 5] += bf16hi(q.z);
+                            f[8 * i + 6] += bf16lo(q.w);
+                            f[8 * i + 7] += bf16hi(q.w);
+                        }
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(pack_bf16x2(f[8 * i + 0], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
+                                            pack_bf16x2(f[8 * i + 4], f[8 * i + 5]), pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace lmoe

@@ -1,0 +1,243 @@
+"""ctypes binding of ``liblmoe.so`` (the C ABI in ``include/lmoe.h``).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch provides device memory and streams.  If the library is
+missing this module raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "liblmoe.so")
+
+LMOE_OK = 0
+STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_ARG", -2: "LMOE_ERR_UNSUPPORTED_SHAPE", -3: "LMOE_ERR_TOO_MANY_TOKENS",
+          -4: "LMOE_ERR_CUDA", -5: "LMOE_ERR_TIMEOUT", -6: "LMOE_ERR_BAD_INDEX", -7: "LMOE_ERR_WORKSPACE"}
+
+P = ctypes.c_void_p
+I32 = ctypes.c_int32
+
+
+class lmoe_config(ctypes.Structure):
+    _fields_ = [(n, I32) for n in ("d", "latent", "m", "n_experts", "top_k", "max_tokens", "act", "n_zero", "n_copy",
+                                   "n_const", "has_proj", "latent_router")]
+
+
+class lmoe_weights(ctypes.Structure):
+    _fields_ = [("w_router", P), ("router_bias", P), ("w_down", P), ("w_up", P), ("w1", P), ("w2", P),
+                ("const_vecs", P)]
+
+
+class lmoe_debug(ctypes.Structure):
+    _fields_ = [("topk_idx", P), ("topk_w", P), ("counts", P), ("offsets", P), ("perm", P), ("z", P), ("yl", P),
+                ("logits", P)]
+
+
+class LmoeError(RuntimeError):
+    def __init__(self, call: str, status: int):
+        super().__init__(f"{call} failed: {STATUS.get(status, status)} ({_text(status)})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing (run __graft_entry__.build())")
+        L = ctypes.CDLL(LIB_PATH)
+        L.lmoe_workspace_bytes.argtypes = [ctypes.POINTER(lmoe_config)]
+        L.lmoe_workspace_bytes.restype = ctypes.c_size_t
+        L.lmoe_create.argtypes = [ctypes.POINTER(lmoe_config), ctypes.POINTER(lmoe_weights), P, ctypes.c_size_t,
+                                  ctypes.POINTER(P)]
+        L.lmoe_forward.argtypes = [P, P, P, I32, P, ctypes.POINTER(lmoe_debug)]
+        L.lmoe_forward_host.argtypes = [P, P, P, I32, P]
+        L.lmoe_last_error.argtypes = [P]
+        L.lmoe_destroy.argtypes = [P]
+        L.lmoe_destroy.restype = None
+        L.lmoe_status_string.argtypes = [ctypes.c_int]
+        L.lmoe_status_string.restype = ctypes.c_char_p
+        L.lmoe_set_profiling.argtypes = [P, ctypes.c_int, ctypes.c_int]
+        L.lmoe_phase_times.argtypes = [P, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(I32)]
+        L.lmoe_num_phases.argtypes = []
+        L.lmoe_phase_name.argtypes = [ctypes.c_int]
+        L.lmoe_phase_name.restype = ctypes.c_char_p
+        L.lmoe_routing_stats.argtypes = [P, ctypes.POINTER(I32)]
+        L.lmoe_set_small_rows.argtypes = [P, I32]
+        L.lmoe_set_wait_timeout.argtypes = [P, ctypes.c_uint64]
+        L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
+        _lib = L
+    return _lib
+
+
+def _text(status: int) -> str:
+    try:
+        return lib().lmoe_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - only while reporting another error
+        return "?"
+
+
+def _check(call: str, status: int) -> None:
+    if status != LMOE_OK:
+        raise LmoeError(call, status)
+
+
+def _p(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ------------------------------------------------------------------ C-ABI calls, same names
+def lmoe_workspace_bytes(cfg: lmoe_config) -> int:
+    return int(lib().lmoe_workspace_bytes(ctypes.byref(cfg)))
+
+
+def lmoe_create(cfg: lmoe_config, weights: lmoe_weights, workspace: int, nbytes: int) -> int:
+    h = P()
+    _check("lmoe_create", lib().lmoe_create(ctypes.byref(cfg), ctypes.byref(weights), workspace, nbytes,
+                                            ctypes.byref(h)))
+    return h.value
+
+
+def lmoe_forward(h: int, x: int, y: int, T: int, stream: Optional[int], dbg: Optional[lmoe_debug] = None) -> None:
+    _check("lmoe_forward", lib().lmoe_forward(h, x, y, T, stream, ctypes.byref(dbg) if dbg is not None else None))
+
+
+def lmoe_forward_host(h: int, x_host: int, y_host: int, T: int, stream: Optional[int]) -> None:
+    _check("lmoe_forward_host", lib().lmoe_forward_host(h, x_host, y_host, T, stream))
+
+
+def lmoe_last_error(h: int) -> int:
+    return int(lib().lmoe_last_error(h))
+
+
+def lmoe_destroy(h: int) -> None:
+    lib().lmoe_destroy(h)
+
+
+def lmoe_status_string(status: int) -> str:
+    return _text(status)
+
+
+def lmoe_set_profiling(h: int, enable: bool, max_forwards: int = 1) -> None:
+    _check("lmoe_set_profiling", lib().lmoe_set_profiling(h, int(enable), int(max_forwards)))
+
+
+def lmoe_num_phases() -> int:
+    return int(lib().lmoe_num_phases())
+
+
+def lmoe_phase_name(i: int) -> str:
+    return lib().lmoe_phase_name(i).decode()
+
+
+def lmoe_phase_times(h: int) -> Dict[str, tuple]:
+    n = lmoe_num_phases()
+    ms = (ctypes.c_float * n)()
+    nl = (I32 * n)()
+    _check("lmoe_phase_times", lib().lmoe_phase_times(h, ms, nl))
+    return {lmoe_phase_name(i): (float(ms[i]), int(nl[i])) for i in range(n)}
+
+
+def lmoe_routing_stats(h: int) -> Dict[str, int]:
+    out = (I32 * 4)()
+    _check("lmoe_routing_stats", lib().lmoe_routing_stats(h, out))
+    return {"ffn_rows": out[0], "experts_touched": out[1], "tc_mtiles": out[2], "stream_experts": out[3]}
+
+
+def lmoe_set_small_rows(h: int, rows: int) -> None:
+    _check("lmoe_set_small_rows", lib().lmoe_set_small_rows(h, rows))
+
+
+def lmoe_set_wait_timeout(h: int, ns: int) -> None:
+    _check("lmoe_set_wait_timeout", lib().lmoe_set_wait_timeout(h, ns))
+
+
+def lmoe_gemm_bf16(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor, err: torch.Tensor, stream=None) -> None:
+    """C = A @ B^T on the tensor-core kernel (bf16 in/out, fp32 accumulate)."""
+    M, K = A.shape
+    N = B.shape[0]
+    _check("lmoe_gemm_bf16", lib().lmoe_gemm_bf16(A.data_ptr(), B.data_ptr(), C.data_ptr(), M, N, K, _stream(stream),
+                                                  err.data_ptr()))
+
+
+# ------------------------------------------------------------------ convenience owner of a layer
+def make_config(cfg, max_tokens: int) -> lmoe_config:
+    return lmoe_config(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, int(max_tokens), cfg.act, cfg.n_zero,
+                       cfg.n_copy, cfg.n_const, cfg.has_proj, cfg.latent_router)
+
+
+class LatentMoE:
+    """A layer on one GPU: device copies of the weights, a workspace and a handle.
+
+    ``cfg`` is a ``synth.LayerConfig`` (or anything with the same fields),
+    ``layer`` the dict of CPU tensors from ``synth.make_layer``.
+    """
+
+    def __init__(self, cfg, layer: Dict[str, torch.Tensor], max_tokens: int, device: str = "cuda"):
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.max_tokens = int(max_tokens)
+        dev = lambda t: None if t is None else t.to(self.device).contiguous()  # noqa: E731
+        self.w = {k: dev(layer.get(k)) for k in ("w_router", "bias", "w_down", "w_up", "w1", "w2", "const_vecs")}
+        self.c = make_config(cfg, self.max_tokens)
+        nbytes = lmoe_workspace_bytes(self.c)
+        if nbytes == 0:
+            raise LmoeError("lmoe_workspace_bytes", -2)
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.weights = lmoe_weights(_p(self.w["w_router"]), _p(self.w["bias"]), _p(self.w["w_down"]),
+                                    _p(self.w["w_up"]), _p(self.w["w1"]), _p(self.w["w2"]), _p(self.w["const_vecs"]))
+        with torch.cuda.device(self.device):
+            self.h = lmoe_create(self.c, self.weights, self.workspace.data_ptr(), nbytes)
+
+    def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None, debug: bool = False, stream=None):
+        T = int(x.shape[0])
+        if y is None:
+            y = torch.empty_like(x)
+        dbg = None
+        out = {}
+        if debug:
+            K, L, nt = self.cfg.top_k, self.cfg.latent, self.cfg.n_total
+            out = {"idx": torch.empty((T, K), dtype=torch.int32, device=self.device),
+                   "w": torch.empty((T, K), dtype=torch.float32, device=self.device),
+                   "counts": torch.empty(nt, dtype=torch.int32, device=self.device),
+                   "offsets": torch.empty(nt + 1, dtype=torch.int32, device=self.device),
+                   "perm": torch.empty(T * K, dtype=torch.int32, device=self.device),
+                   "logits": torch.empty((T, nt), dtype=torch.float32, device=self.device)}
+            if self.cfg.has_proj:
+                out["z"] = torch.empty((T, L), dtype=torch.bfloat16, device=self.device)
+                out["yl"] = torch.empty((T, L), dtype=torch.bfloat16, device=self.device)
+            dbg = lmoe_debug(_p(out["idx"]), _p(out["w"]), _p(out["counts"]), _p(out["offsets"]), _p(out["perm"]),
+                             _p(out.get("z")), _p(out.get("yl")), _p(out["logits"]))
+        lmoe_forward(self.h, x.data_ptr(), y.data_ptr(), T, _stream(stream), dbg)
+        return (y, out) if debug else y
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, stream=None) -> None:
+        lmoe_forward_host(self.h, x_host.data_ptr(), y_host.data_ptr(), int(x_host.shape[0]), _stream(stream))
+
+    def last_error(self) -> int:
+        return lmoe_last_error(self.h)
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            lmoe_destroy(self.h)
+            self.h = None
+
+    def __del__(self):  # pragma: no cover - interpreter shutdown order varies
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -12,7 +12,11 @@
  *        f = x (the gate stays at the full width d: "LatentMoE: How MoE Made
  *        a Key Paradigm Leap in 2026", section 2 closing note; Kimi K3 /
  *        Nemotron 3 Super article, "LatentMoE 具体怎么做", closing note), or
- *        f = z when the latent-router reading is selected.
+ *        f = bf16(z) when the latent-router reading is selected ("routing
+ *        happens in the latent", the same sections' second bullet).  The
+ *        latent is stored in bf16 before the gate reads it, so the top-K'
+ *        decision (an integer decided by floating point) is taken on the same
+ *        bf16 input on both sides; everything else stays in fp64.
  *   2. top-K' selection: the K' largest logits, ties to the lower expert id,
  *      slots ordered by (logit descending, id ascending).
  *   3. renormalised softmax over the selected logits
@@ -72,6 +76,20 @@ static double widen(uint16_t h)
 }
 
 static int n_total(const oracle_cfg *c) { return c->n_ffn + c->n_zero + c->n_copy + c->n_const; }
+
+/* Round to the nearest bfloat16 (ties to even) through binary32, the way a
+ * value accumulated in fp32 is stored as bf16.  Used for one input only: the
+ * latent the latent-router reading feeds to the gate (see step 1). */
+static double round_bf16(double v)
+{
+    float f = (float)v;
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    u += 0x7FFFu + ((u >> 16) & 1u);
+    u &= 0xFFFF0000u;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
 
 /* out[o] = sum_i W[o*in_dim + i] * v[i] */
 static void matvec(int out_dim, int in_dim, const uint16_t *W, const double *v, double *out)
@@ -196,6 +214,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
     {
         double *xt = (double *)malloc(sizeof(double) * (size_t)d);
         double *z = (double *)malloc(sizeof(double) * (size_t)L);
+        double *zr = (double *)malloc(sizeof(double) * (size_t)L);
         double *lg = (double *)malloc(sizeof(double) * (size_t)Nt);
         double *u = (double *)malloc(sizeof(double) * (size_t)up_rows);
         double *h = (double *)malloc(sizeof(double) * (size_t)m);
@@ -204,7 +223,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
         double *up = (double *)malloc(sizeof(double) * (size_t)d);
         double *w = (double *)malloc(sizeof(double) * (size_t)K);
         int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
-        if (!xt || !z || !lg || !u || !h || !o || !yl || !up || !w || !sel) bad = 1;
+        if (!xt || !z || !zr || !lg || !u || !h || !o || !yl || !up || !w || !sel) bad = 1;
 
 #pragma omp for schedule(dynamic, 1)
         for (int t = 0; t < T; ++t) {
@@ -213,8 +232,13 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             /* step 4: latent projection (identity for the standard MoE) */
             if (c->has_proj) matvec(L, d, w_down, xt, z);
             else memcpy(z, xt, sizeof(double) * (size_t)d);
-            /* step 1: router logits at the full width (or in the latent) */
-            matvec(Nt, fdim, w_router, c->latent_router ? z : xt, lg);
+            /* step 1: router logits at the full width (or on the bf16 latent) */
+            if (c->latent_router) {
+                for (int j = 0; j < L; ++j) zr[j] = round_bf16(z[j]);
+                matvec(Nt, fdim, w_router, zr, lg);
+            } else {
+                matvec(Nt, fdim, w_router, xt, lg);
+            }
             if (bias)
                 for (int e = 0; e < Nt; ++e) lg[e] += (double)bias[e];
             /* steps 2-3 */
@@ -261,7 +285,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             if (yl_out) memcpy(yl_out + (size_t)t * L, yl, sizeof(double) * (size_t)L);
             if (logits_out) memcpy(logits_out + (size_t)t * Nt, lg, sizeof(double) * (size_t)Nt);
         }
-        free(xt); free(z); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
+        free(xt); free(z); free(zr); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
     }
     return bad ? -1 : 0;
 }

@@ -1,0 +1,93 @@
+"""The C-ABI library loads and exports every entry point include/*.h declares; host-side
+argument checks reject bad input before any CUDA call (these run without a GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from latent_mixture_experts_gemm_b200 import lmoe, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(hdr).read(), flags=re.S)
+        names.update(re.findall(r"LMOE_API\s+[\w\s\*]*?\b(lmoe_\w+)\s*\(", text))
+    return sorted(names)
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("lmoe_workspace_bytes", "lmoe_create", "lmoe_forward", "lmoe_forward_host", "lmoe_last_error",
+                     "lmoe_destroy", "lmoe_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = lmoe.lib()
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    for code in lmoe.STATUS:
+        assert lmoe.lmoe_status_string(code) not in ("", "unknown status")
+    assert lmoe.lmoe_status_string(12345) == "unknown status"
+
+
+def test_workspace_bytes_and_shape_checks():
+    ok = lmoe.make_config(synth.WORKLOADS["nemotron_prefill"], 8192)
+    n = lmoe.lmoe_workspace_bytes(ok)
+    assert n > 2 * 8192 * 22 * 1024 * 2   # at least the gathered rows (reused for outputs) and hidden rows
+    small = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
+    assert 0 < lmoe.lmoe_workspace_bytes(small) < n
+    bad = [dict(d=100), dict(latent=0), dict(m=32), dict(top_k=0), dict(top_k=33), dict(n_experts=0),
+           dict(max_tokens=0), dict(act=7), dict(has_proj=0)]
+    for b in bad:
+        c = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
+        for k, v in b.items():
+            setattr(c, k, v)
+        assert lmoe.lmoe_workspace_bytes(c) == 0, b
+    c = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
+    c.n_experts = 1020
+    c.n_zero = 5           # n_total 1025 > 1024
+    assert lmoe.lmoe_workspace_bytes(c) == 0
+
+
+def test_create_rejects_before_touching_the_device():
+    L = lmoe.lib()
+    cfg = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
+    w = lmoe.lmoe_weights()
+    h = ctypes.c_void_p()
+    assert L.lmoe_create(None, ctypes.byref(w), None, 0, ctypes.byref(h)) == -1
+    bad = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
+    bad.d = 65
+    assert L.lmoe_create(ctypes.byref(bad), ctypes.byref(w), None, 0, ctypes.byref(h)) == -2
+    assert L.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), None, 0, ctypes.byref(h)) == -7
+    # a workspace that is large enough but misaligned, then missing weights
+    big = lmoe.lmoe_workspace_bytes(cfg)
+    assert L.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), 0x1001, big, ctypes.byref(h)) == -1
+    assert L.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), 0x10000, big, ctypes.byref(h)) == -1
+    assert h.value is None
+
+
+def test_null_handle_calls_are_rejected():
+    L = lmoe.lib()
+    assert L.lmoe_forward(None, None, None, 1, None, None) == -1
+    assert L.lmoe_forward_host(None, None, None, 1, None) == -1
+    assert L.lmoe_last_error(None) == -1
+    assert L.lmoe_set_profiling(None, 1, 1) == -1
+    L.lmoe_destroy(None)
+    assert lmoe.lmoe_num_phases() == 9
+    assert [lmoe.lmoe_phase_name(i) for i in range(3)] == ["router_proj_gemm", "topk_softmax", "dispatch"]
+
+
+def test_gemm_shape_checks():
+    L = lmoe.lib()
+    assert L.lmoe_gemm_bf16(0x100, 0x100, 0x100, 128, 100, 64, None, 0x100) == -2
+    assert L.lmoe_gemm_bf16(0x100, 0x100, 0x100, 128, 64, 96, None, 0x100) == -2
+    assert L.lmoe_gemm_bf16(0x100, 0x100, 0x100, 128, 64, 64, None, None) == -1

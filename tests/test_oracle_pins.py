@@ -150,7 +150,9 @@ def _dense_bruteforce(cfg, layer):
     W1, W2 = _np(layer["w1"]), _np(layer["w2"])
     T, m = x.shape[0], cfg.m
     z = x @ Wd.T if cfg.has_proj else x.copy()
-    lg = (z if cfg.latent_router else x) @ Wr.T
+    # the latent router reads the latent stored in bf16 (round to nearest even through fp32)
+    z_gate = torch.from_numpy(z).to(torch.float32).to(torch.bfloat16).double().numpy()
+    lg = (z_gate if cfg.latent_router else x) @ Wr.T
     if layer.get("bias") is not None:
         lg = lg + layer["bias"].double().numpy()
     U = np.einsum("eol,tl->teo", W1, z)
