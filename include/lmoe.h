@@ -170,17 +170,23 @@ LMOE_API const char *lmoe_phase_name(int phase);
 
 /*
  * Sizes of the last forward's routing, read back from the device (blocking;
- * synchronise first): out[0] = rows routed to FFN experts, out[1] = FFN
- * experts with at least one row, out[2] = tensor-core M-tiles, out[3] =
- * experts served by the weight-streaming path.  Used to compute the
- * algorithmic work of a forward.
+ * synchronise first).  out8[0] rows routed to FFN experts, [1] FFN experts
+ * with at least one row, [2] tensor-core M-tiles, [3] experts on the
+ * weight-streaming path, [4] rows on that path, [5] experts on the grouped
+ * tensor-core path, [6] rows on that path, [7] the row threshold the forward
+ * used (see lmoe_set_small_rows).  Used to compute the algorithmic work of a
+ * forward.
  */
-LMOE_API int lmoe_routing_stats(lmoe_handle *h, int32_t *out4);
+LMOE_API int lmoe_routing_stats(lmoe_handle *h, int32_t *out8);
 
 /*
- * Routing threshold: FFN experts with at most `rows` routed rows take the
- * weight-streaming path (default 8, the maximum), the others the tensor-core
- * grouped GEMM; 0 sends every expert to the tensor cores.
+ * Expert-path threshold: FFN experts with at most `rows` routed rows (0..32,
+ * default 16) take the weight-streaming GEMM (the expert's weights as the
+ * 128-row tensor-core operand, its rows as a 16- or 32-row operand); the
+ * others take the grouped GEMM in 128-row tiles.  A forward with T <= 32
+ * tokens raises a nonzero threshold to 16 (T <= 16) or 32, so that every
+ * expert streams and the grouped GEMM is not launched.  0 sends every expert
+ * to the grouped GEMM.
  */
 LMOE_API int lmoe_set_small_rows(lmoe_handle *h, int32_t rows);
 

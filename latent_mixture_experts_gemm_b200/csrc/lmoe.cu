@@ -21,6 +21,7 @@
 #include "../../include/lmoe.h"
 #include "moe_kernels.cuh"
 #include "tc_gemm.cuh"
+#include "tc_swap.cuh"
 
 using namespace lmoe;
 
@@ -73,9 +74,14 @@ bool config_ok(const lmoe_config& c) {
     return true;
 }
 
+// Few-token path (T <= kFewTokenRows): the projections stream their weights
+// with split-K on the weight-streaming kernel.
+constexpr int kFewTokenRows = 32;
+constexpr int kFewTokenMaxSplits = 16;
+
 struct Plan {
     size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
-        xin, yout, total;
+        partial, xin, yout, total;
     int ld_logits, nwords, mt_max;
 };
 
@@ -109,6 +115,11 @@ Plan make_plan(const lmoe_config& c) {
     p.rows = take(R * L * 2);  // gathered expert inputs, then (reused) expert outputs
     p.hbuf = take(R * m * 2);
     p.yl = c.has_proj ? take(T * L * 2) : 0;
+    {   // split-K partial sums of the few-token projections: [splits][128-row tiles][32 tokens] fp32
+        auto up128 = [](size_t v) { return (v + 127) / 128 * 128; };
+        const size_t rows = std::max(up128(L) + up128(nt), std::max(up128(d), up128(nt)));
+        p.partial = take(static_cast<size_t>(kFewTokenMaxSplits) * rows * kFewTokenRows * 4);
+    }
     p.xin = take(T * d * 2);
     p.yout = take(T * d * 2);
     p.total = off;
@@ -129,8 +140,22 @@ bool set_smem_attr() {
                                 GemmCfg<BN>::SMEM_BYTES) == cudaSuccess;
 }
 
+template <int NT, int EPI>
+bool set_swap_attr() {
+    return cudaFuncSetAttribute(tc_swap_kernel<NT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SwapCfg<NT, EPI>::SMEM_BYTES) == cudaSuccess;
+}
+
 bool set_all_smem_attrs() {
     bool ok = true;
+    ok &= cudaFuncSetAttribute(dispatch_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (2 * SMALL_BATCH_WORDS * 1024 + 1024) * 4) == cudaSuccess;
+    ok &= set_swap_attr<16, EPI_BF16>();
+    ok &= set_swap_attr<16, EPI_RELU2>();
+    ok &= set_swap_attr<16, EPI_SWIGLU>();
+    ok &= set_swap_attr<32, EPI_BF16>();
+    ok &= set_swap_attr<32, EPI_RELU2>();
+    ok &= set_swap_attr<32, EPI_SWIGLU>();
     ok &= set_smem_attr<64, EPI_BF16>();
     ok &= set_smem_attr<256, EPI_BF16>();
     ok &= set_smem_attr<64, EPI_RESID>();
@@ -140,6 +165,76 @@ bool set_all_smem_attrs() {
     ok &= set_smem_attr<256, EPI_RELU2>();
     ok &= set_smem_attr<256, EPI_SWIGLU>();
     return ok;
+}
+
+template <int NT, int EPI>
+void launch_swap(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& w2, const SwapArgs& args, int grid,
+                 cudaStream_t s) {
+    tc_swap_kernel<NT, EPI><<<grid, 192, SwapCfg<NT, EPI>::SMEM_BYTES, s>>>(w, x, w2, args);
+}
+
+// Weight-streaming launch for the experts of the small list, dispatched on the token tile and epilogue.
+void launch_stream(int nt, int epi, const CUtensorMap& w, const CUtensorMap& x16, const CUtensorMap& x32,
+                   const SwapArgs& a, int grid, cudaStream_t s) {
+    if (nt <= 16) {
+        if (epi == EPI_RELU2) launch_swap<16, EPI_RELU2>(w, x16, w, a, grid, s);
+        else if (epi == EPI_SWIGLU) launch_swap<16, EPI_SWIGLU>(w, x16, w, a, grid, s);
+        else launch_swap<16, EPI_BF16>(w, x16, w, a, grid, s);
+    } else {
+        if (epi == EPI_RELU2) launch_swap<32, EPI_RELU2>(w, x32, w, a, grid, s);
+        else if (epi == EPI_SWIGLU) launch_swap<32, EPI_SWIGLU>(w, x32, w, a, grid, s);
+        else launch_swap<32, EPI_BF16>(w, x32, w, a, grid, s);
+    }
+}
+
+// Few-token projection: split-K weight streaming into fp32 partials, then the
+// in-order reduction with its epilogue.  Returns the number of launches.
+struct FewTokenGemm {
+    const CUtensorMap* w;   // first weight segment (128-row boxes)
+    const CUtensorMap* w2;  // second weight segment (or the same map)
+    const CUtensorMap* x16;
+    const CUtensorMap* x32;
+    int rows0, rows1;       // weight rows of the two segments (rows1 may be 0)
+    int K;
+    __nv_bfloat16* out0;
+    int ld0;
+    float* out1;
+    int ld1;
+    const __nv_bfloat16* resid;
+    int ld_resid;
+};
+
+int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_splits, int num_sms, int* err,
+                     unsigned long long timeout_ns, cudaStream_t s) {
+    const int t0 = (g.rows0 + 127) / 128, t1 = (g.rows1 + 127) / 128;
+    const int nkb = g.K / 64;
+    int splits = (num_sms + t0 + t1 - 1) / (t0 + t1);
+    splits = std::max(1, std::min(splits, std::min(max_splits, nkb)));
+    SwapArgs a{};
+    a.K = g.K;
+    a.n_wtiles = t0 + t1;
+    a.n_wtiles0 = t0;
+    a.k_splits = splits;
+    a.list = nullptr;
+    a.dense_rows = T;
+    a.partial = partial;
+    a.part_rows = (t0 + t1) * 128;
+    a.err = err;
+    a.timeout_ns = timeout_ns;
+    const int units = (t0 + t1) * splits;
+    const int grid = std::min(num_sms, units);
+    const long outs = static_cast<long>(g.rows0 + g.rows1) * T;
+    const unsigned rgrid = static_cast<unsigned>((outs + 255) / 256);
+    if (T <= 16) {
+        launch_swap<16, EPI_BF16>(*g.w, *g.x16, *g.w2, a, grid, s);
+        swap_reduce_kernel<16><<<rgrid, 256, 0, s>>>(partial, a.part_rows, splits, T, g.rows0, g.rows1, t0 * 128,
+                                                      g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
+    } else {
+        launch_swap<32, EPI_BF16>(*g.w, *g.x32, *g.w2, a, grid, s);
+        swap_reduce_kernel<32><<<rgrid, 256, 0, s>>>(partial, a.part_rows, splits, T, g.rows0, g.rows1, t0 * 128,
+                                                      g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
+    }
+    return 2;
 }
 
 template <int BN, int EPI>
@@ -156,11 +251,16 @@ struct lmoe_handle {
     lmoe_weights w{};
     uint8_t* ws = nullptr;
     Plan p{};
-    int n_tot = 0, g = 1, num_sms = 148, small_max = SMALL_MAX, device = 0;
+    int n_tot = 0, g = 1, num_sms = 148, small_max = 16, device = 0;
+    int last_small = 16;  // threshold the last forward used
     unsigned long long timeout_ns = 1000000000ull;
     // weight descriptors: router/projection operands for both column tiles, expert weights, workspace operands
     CUtensorMap wdown64{}, wdown256{}, wr64{}, wr256{}, wup64{}, wup256{}, w1{}, w2{};
     CUtensorMap a_rows{}, a_h{}, a_yl{}, a_z{};
+    // weight-streaming operands: 128-row weight tiles, 16- and 32-row token tiles
+    CUtensorMap w1s{}, w2s{}, rows16{}, rows32{}, h16{}, h32{};
+    // few-token projections: 128-row weight tiles and 16/32-row token tiles of z and yl
+    CUtensorMap wdown128{}, wr128{}, wup128{}, z16{}, z32{}, yl16{}, yl32{};
     // profiling
     bool prof = false;
     int prof_max = 0, prof_n = 0;
@@ -225,47 +325,70 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     base.timeout_ns = h->timeout_ns;
 
     // ---------------------------------------------------------------- router (+ W_down)
-    {
+    if (T <= kFewTokenRows) {
+        // few tokens: split-K weight streaming (weights as the 128-row operand) + in-order reduction
+        CUtensorMap x16, x32;
+        if (!make_map(&x16, x, T, d, d, 16) || !make_map(&x32, x, T, d, d, 32)) return LMOE_ERR_CUDA;
+        float* part = h->at<float>(p.partial);
         const bool fused = proj && !c.latent_router;
-        const int n256 = (fused ? (L + 255) / 256 : 0) + (nt + 255) / 256;
-        const bool big = m_tiles * n256 >= h->num_sms;
-        const int n_gemm = (proj && c.latent_router) ? 2 : 1;
-        PhaseScope ps(h, PH_ROUTER, s, n_gemm);
+        const int n_launch = (proj && c.latent_router) ? 4 : 2;
+        PhaseScope ps(h, PH_ROUTER, s, n_launch);
         if (proj && c.latent_router) {
+            FewTokenGemm g{&h->wdown128, &h->wdown128, &x16, &x32, L, 0, d, z, L, nullptr, 0, nullptr, 0};
+            launch_few_token(g, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
+            FewTokenGemm r{&h->wr128, &h->wr128, &h->z16, &h->z32, 0, nt, L, nullptr, 0, logits, p.ld_logits,
+                           nullptr, 0};
+            launch_few_token(r, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
+        } else if (fused) {
+            FewTokenGemm g{&h->wdown128, &h->wr128, &x16, &x32, L, nt, d, z, L, logits, p.ld_logits, nullptr, 0};
+            launch_few_token(g, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
+        } else {
+            FewTokenGemm r{&h->wr128, &h->wr128, &x16, &x32, 0, nt, d, nullptr, 0, logits, p.ld_logits, nullptr, 0};
+            launch_few_token(r, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
+        }
+    } else {
+        {
+            const bool fused = proj && !c.latent_router;
+            const int n256 = (fused ? (L + 255) / 256 : 0) + (nt + 255) / 256;
+            const bool big = m_tiles * n256 >= h->num_sms;
+            const int n_gemm = (proj && c.latent_router) ? 2 : 1;
+            PhaseScope ps(h, PH_ROUTER, s, n_gemm);
+            if (proj && c.latent_router) {
+                GemmArgs a = base;
+                a.M = T;
+                a.K = d;
+                a.N0 = L;
+                a.out0 = z;
+                a.ld0 = L;
+                if (big) {
+                    a.n_tiles = (L + 255) / 256;
+                    launch_gemm<256, EPI_BF16>(a_x, h->wdown256, h->wdown256, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+                } else {
+                    a.n_tiles = (L + 63) / 64;
+                    launch_gemm<64, EPI_BF16>(a_x, h->wdown64, h->wdown64, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+                }
+            }
             GemmArgs a = base;
             a.M = T;
-            a.K = d;
-            a.N0 = L;
+            a.K = c.latent_router ? L : d;
+            a.N0 = fused ? L : 0;
+            a.N1 = nt;
             a.out0 = z;
             a.ld0 = L;
+            a.out1 = logits;
+            a.ld1 = p.ld_logits;
+            const CUtensorMap& A = (proj && c.latent_router) ? h->a_z : a_x;
             if (big) {
-                a.n_tiles = (L + 255) / 256;
-                launch_gemm<256, EPI_BF16>(a_x, h->wdown256, h->wdown256, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+                a.n_tiles0 = fused ? (L + 255) / 256 : 0;
+                a.n_tiles = a.n_tiles0 + (nt + 255) / 256;
+                launch_gemm<256, EPI_PROJ_ROUTER>(A, fused ? h->wdown256 : h->wr256, h->wr256, a,
+                                                  std::min(h->num_sms, m_tiles * a.n_tiles), s);
             } else {
-                a.n_tiles = (L + 63) / 64;
-                launch_gemm<64, EPI_BF16>(a_x, h->wdown64, h->wdown64, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+                a.n_tiles0 = fused ? (L + 63) / 64 : 0;
+                a.n_tiles = a.n_tiles0 + (nt + 63) / 64;
+                launch_gemm<64, EPI_PROJ_ROUTER>(A, fused ? h->wdown64 : h->wr64, h->wr64, a,
+                                                 std::min(h->num_sms, m_tiles * a.n_tiles), s);
             }
-        }
-        GemmArgs a = base;
-        a.M = T;
-        a.K = c.latent_router ? L : d;
-        a.N0 = fused ? L : 0;
-        a.N1 = nt;
-        a.out0 = z;
-        a.ld0 = L;
-        a.out1 = logits;
-        a.ld1 = p.ld_logits;
-        const CUtensorMap& A = (proj && c.latent_router) ? h->a_z : a_x;
-        if (big) {
-            a.n_tiles0 = fused ? (L + 255) / 256 : 0;
-            a.n_tiles = a.n_tiles0 + (nt + 255) / 256;
-            launch_gemm<256, EPI_PROJ_ROUTER>(A, fused ? h->wdown256 : h->wr256, h->wr256, a,
-                                              std::min(h->num_sms, m_tiles * a.n_tiles), s);
-        } else {
-            a.n_tiles0 = fused ? (L + 63) / 64 : 0;
-            a.n_tiles = a.n_tiles0 + (nt + 63) / 64;
-            launch_gemm<64, EPI_PROJ_ROUTER>(A, fused ? h->wdown64 : h->wr64, h->wr64, a,
-                                             std::min(h->num_sms, m_tiles * a.n_tiles), s);
         }
     }
     // ---------------------------------------------------------------- top-K' + softmax
@@ -282,24 +405,39 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         else topk_softmax_kernel<32><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
     }
     // ---------------------------------------------------------------- counting sort by expert
+    // Experts with at most `small` rows stream their weights; when every expert
+    // must (T <= small) the grouped GEMMs are not launched at all.
+    int small = h->small_max;
+    if (small > 0 && T <= SMALL_MAX) small = T <= 16 ? 16 : SMALL_MAX;
+    const bool need_tc = T > small;
+    h->last_small = small;
     {
-        PhaseScope ps(h, PH_DISPATCH, s, 4);
         const int nwords = (T + 31) / 32;
-        uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
-        uint32_t* prefix = h->at<uint32_t>(p.prefix);
         int* counts = h->at<int>(p.counts);
         int* offsets = h->at<int>(p.offsets);
-        dispatch_bitmap_kernel<<<(nwords + 7) / 8, 256, 8 * nt * 4, s>>>(idx, T, K, nt, bitmap, hdr);
-        dispatch_expert_scan_kernel<<<(nt + 7) / 8, 256, 0, s>>>(bitmap, T, nt, prefix, counts);
-        dispatch_offsets_kernel<<<1, 1024, 0, s>>>(counts, nt, c.n_experts, h->small_max, offsets, mt_list, small_list,
-                                                   hdr);
         const long slots = static_cast<long>(T) * K;
-        dispatch_scatter_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
-            idx, T, K, nt, c.n_experts, bitmap, prefix, offsets, feat, L, L, rows, L, h->at<int32_t>(p.perm),
-            h->at<int32_t>(p.inv));
+        if (nwords <= SMALL_BATCH_WORDS) {
+            PhaseScope ps(h, PH_DISPATCH, s, 2);
+            const size_t sm = (static_cast<size_t>(2 * nwords) * nt + nt) * 4;
+            dispatch_small_kernel<<<1, 1024, sm, s>>>(idx, T, K, nt, c.n_experts, small, counts, offsets, mt_list,
+                                                      small_list, h->at<int32_t>(p.perm), h->at<int32_t>(p.inv), hdr);
+            dispatch_gather_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
+                idx, h->at<int32_t>(p.inv), T, K, c.n_experts, feat, L, L, rows, L);
+        } else {
+            PhaseScope ps(h, PH_DISPATCH, s, 4);
+            uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
+            uint32_t* prefix = h->at<uint32_t>(p.prefix);
+            dispatch_bitmap_kernel<<<(nwords + 7) / 8, 256, 8 * nt * 4, s>>>(idx, T, K, nt, bitmap, hdr);
+            dispatch_expert_scan_kernel<<<(nt + 7) / 8, 256, 0, s>>>(bitmap, T, nt, prefix, counts);
+            dispatch_offsets_kernel<<<1, 1024, 0, s>>>(counts, nt, c.n_experts, small, offsets, mt_list, small_list,
+                                                       hdr);
+            dispatch_scatter_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
+                idx, T, K, nt, c.n_experts, bitmap, prefix, offsets, feat, L, L, rows, L, h->at<int32_t>(p.perm),
+                h->at<int32_t>(p.inv));
+        }
     }
     // ---------------------------------------------------------------- expert up (+ activation)
-    {
+    if (need_tc) {
         PhaseScope ps(h, PH_UP_TC, s, 1);
         GemmArgs a = base;
         a.K = L;
@@ -321,21 +459,26 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
             launch_gemm<256, EPI_BF16>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
         }
     }
-    if (h->small_max > 0) {
+    if (small > 0) {
         PhaseScope ps(h, PH_UP_STREAM, s, 1);
-        const int grid = h->num_sms * 3;
-        if (c.act == LMOE_ACT_SWIGLU)
-            expert_stream_kernel<GEMV_SWIGLU><<<grid, GEMV_THREADS, 0, s>>>(
-                rows, L, static_cast<const __nv_bfloat16*>(h->w.w1), 2 * m, m, L, m, hbuf, m, small_list, hdr + HDR_NSMALL);
-        else if (c.act == LMOE_ACT_RELU2)
-            expert_stream_kernel<GEMV_RELU2><<<grid, GEMV_THREADS, 0, s>>>(
-                rows, L, static_cast<const __nv_bfloat16*>(h->w.w1), m, 0, L, m, hbuf, m, small_list, hdr + HDR_NSMALL);
-        else
-            expert_stream_kernel<GEMV_NONE><<<grid, GEMV_THREADS, 0, s>>>(
-                rows, L, static_cast<const __nv_bfloat16*>(h->w.w1), m, 0, L, m, hbuf, m, small_list, hdr + HDR_NSMALL);
+        SwapArgs a{};
+        a.K = L;
+        a.k_splits = 1;
+        a.n_wtiles = (m + 127) / 128;
+        a.list = small_list;
+        a.count = hdr + HDR_NSMALL;
+        a.w_rows_per_expert = h->g * m;
+        a.up_offset = m;
+        a.n_out = m;
+        a.out = hbuf;
+        a.ld_out = m;
+        a.err = hdr + HDR_ERR;
+        a.timeout_ns = h->timeout_ns;
+        const int epi = c.act == LMOE_ACT_SWIGLU ? EPI_SWIGLU : (c.act == LMOE_ACT_RELU2 ? EPI_RELU2 : EPI_BF16);
+        launch_stream(small, epi, h->w1s, h->rows16, h->rows32, a, h->num_sms, s);
     }
     // ---------------------------------------------------------------- expert down (output reuses the gathered rows)
-    {
+    if (need_tc) {
         PhaseScope ps(h, PH_DOWN_TC, s, 1);
         GemmArgs a = base;
         a.K = m;
@@ -348,10 +491,22 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.n_tiles = (L + 255) / 256;
         launch_gemm<256, EPI_BF16>(h->a_h, h->w2, h->w2, a, h->num_sms, s);
     }
-    if (h->small_max > 0) {
+    if (small > 0) {
         PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
-        expert_stream_kernel<GEMV_NONE><<<h->num_sms * 3, GEMV_THREADS, 0, s>>>(
-            hbuf, m, static_cast<const __nv_bfloat16*>(h->w.w2), L, 0, m, L, rows, L, small_list, hdr + HDR_NSMALL);
+        SwapArgs a{};
+        a.K = m;
+        a.k_splits = 1;
+        a.n_wtiles = (L + 127) / 128;
+        a.list = small_list;
+        a.count = hdr + HDR_NSMALL;
+        a.w_rows_per_expert = L;
+        a.up_offset = 0;
+        a.n_out = L;
+        a.out = rows;
+        a.ld_out = L;
+        a.err = hdr + HDR_ERR;
+        a.timeout_ns = h->timeout_ns;
+        launch_stream(small, EPI_BF16, h->w2s, h->h16, h->h32, a, h->num_sms, s);
     }
     // ---------------------------------------------------------------- combine in the latent width
     {
@@ -362,7 +517,12 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
                                           c.n_zero, c.n_copy, proj ? nullptr : xb, d, out, proj ? L : d);
     }
     // ---------------------------------------------------------------- W_up + residual
-    if (proj) {
+    if (proj && T <= kFewTokenRows) {
+        PhaseScope ps(h, PH_WUP, s, 2);
+        FewTokenGemm g{&h->wup128, &h->wup128, &h->yl16, &h->yl32, d, 0, L, yb, d, nullptr, 0, xb, d};
+        launch_few_token(g, T, h->at<float>(p.partial), kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns,
+                         s);
+    } else if (proj) {
         PhaseScope ps(h, PH_WUP, s, 1);
         GemmArgs a = base;
         a.M = T;
@@ -449,6 +609,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     const int fdim = c.latent_router ? L : d;
     const uint64_t R = static_cast<uint64_t>(c.max_tokens) * c.top_k;
     bool ok = true;
+    ok &= make_map(&h->wr128, w->w_router, nt, fdim, fdim, 128);
     ok &= make_map(&h->wr64, w->w_router, nt, fdim, fdim, 64);
     ok &= make_map(&h->wr256, w->w_router, nt, fdim, fdim, 256);
     if (c.has_proj) {
@@ -458,11 +619,23 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
         ok &= make_map(&h->wup256, w->w_up, d, L, L, 256);
         ok &= make_map(&h->a_yl, h->at<void>(p.yl), c.max_tokens, L, L, 128);
         ok &= make_map(&h->a_z, h->at<void>(p.z), c.max_tokens, L, L, 128);
+        ok &= make_map(&h->wdown128, w->w_down, L, d, d, 128);
+        ok &= make_map(&h->wup128, w->w_up, d, L, L, 128);
+        ok &= make_map(&h->z16, h->at<void>(p.z), c.max_tokens, L, L, 16);
+        ok &= make_map(&h->z32, h->at<void>(p.z), c.max_tokens, L, L, 32);
+        ok &= make_map(&h->yl16, h->at<void>(p.yl), c.max_tokens, L, L, 16);
+        ok &= make_map(&h->yl32, h->at<void>(p.yl), c.max_tokens, L, L, 32);
     }
     ok &= make_map(&h->w1, w->w1, static_cast<uint64_t>(c.n_experts) * h->g * m, L, L, h->g == 2 ? 128 : 256);
     ok &= make_map(&h->w2, w->w2, static_cast<uint64_t>(c.n_experts) * L, m, m, 256);
     ok &= make_map(&h->a_rows, h->at<void>(p.rows), R, L, L, 128);
     ok &= make_map(&h->a_h, h->at<void>(p.hbuf), R, m, m, 128);
+    ok &= make_map(&h->w1s, w->w1, static_cast<uint64_t>(c.n_experts) * h->g * m, L, L, 128);
+    ok &= make_map(&h->w2s, w->w2, static_cast<uint64_t>(c.n_experts) * L, m, m, 128);
+    ok &= make_map(&h->rows16, h->at<void>(p.rows), R, L, L, 16);
+    ok &= make_map(&h->rows32, h->at<void>(p.rows), R, L, L, 32);
+    ok &= make_map(&h->h16, h->at<void>(p.hbuf), R, m, m, 16);
+    ok &= make_map(&h->h32, h->at<void>(p.hbuf), R, m, m, 32);
     ok &= cudaMemset(h->at<void>(p.hdr), 0, HDR_WORDS * 4) == cudaSuccess;
     if (!ok) {
         delete h;
@@ -576,19 +749,33 @@ int lmoe_num_phases(void) { return PH_COUNT; }
 
 const char* lmoe_phase_name(int phase) { return (phase >= 0 && phase < PH_COUNT) ? kPhaseNames[phase] : nullptr; }
 
-int lmoe_routing_stats(lmoe_handle* h, int32_t* out4) {
-    if (h == nullptr || out4 == nullptr) return LMOE_ERR_INVALID_ARG;
+int lmoe_routing_stats(lmoe_handle* h, int32_t* out8) {
+    if (h == nullptr || out8 == nullptr) return LMOE_ERR_INVALID_ARG;
     int hdr[HDR_WORDS];
     std::vector<int> counts(h->n_tot);
     if (cudaMemcpy(hdr, h->at<int>(h->p.hdr), sizeof hdr, cudaMemcpyDeviceToHost) != cudaSuccess ||
         cudaMemcpy(counts.data(), h->at<int>(h->p.counts), counts.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
         return LMOE_ERR_CUDA;
-    int touched = 0;
-    for (int e = 0; e < h->c.n_experts; ++e) touched += counts[e] > 0;
-    out4[0] = hdr[HDR_ROWS];
-    out4[1] = touched;
-    out4[2] = hdr[HDR_MT];
-    out4[3] = hdr[HDR_NSMALL];
+    int touched = 0, st_experts = 0, st_rows = 0, tc_experts = 0, tc_rows = 0;
+    for (int e = 0; e < h->c.n_experts; ++e) {
+        const int n = counts[e];
+        touched += n > 0;
+        if (n > 0 && n <= h->last_small) {
+            ++st_experts;
+            st_rows += n;
+        } else if (n > h->last_small) {
+            ++tc_experts;
+            tc_rows += n;
+        }
+    }
+    out8[0] = hdr[HDR_ROWS];
+    out8[1] = touched;
+    out8[2] = hdr[HDR_MT];
+    out8[3] = hdr[HDR_NSMALL];
+    out8[4] = st_rows;
+    out8[5] = tc_experts;
+    out8[6] = tc_rows;
+    out8[7] = h->last_small;
     return LMOE_OK;
 }
 

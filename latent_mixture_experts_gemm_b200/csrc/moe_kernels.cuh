@@ -1,7 +1,6 @@
 // moe_kernels.cuh -- the non-tensor-core steps of the LatentMoE layer forward:
 // top-K' routing with renormalised softmax, the counting sort of (token, slot)
-// pairs by expert, the decode-regime expert weight streaming, and the
-// fixed-order combine.
+// pairs by expert, and the fixed-order combine.
 #pragma once
 #include <cfloat>
 #include <climits>
@@ -20,63 +19,111 @@ enum : int {
 
 // ============================================================================ routing
 // One warp per token.  Scores are the router logits plus the optional bias;
-// the K' largest are selected in order (value descending, id ascending on
-// ties) by K' rounds of a warp arg-max, and their softmax is renormalised over
-// the selection: w_k = exp(l_k - l_max) / sum_j exp(l_j - l_max).
+// the K' largest are selected (value descending, expert id ascending on ties)
+// and their softmax is renormalised over the selection:
+//   w_k = exp(l_k - l_max) / sum_{j in S} exp(l_j - l_max).
+// Lane j holds experts j, j+32, ... as order-preserving 32-bit keys.
+//   1. The K'-th largest key tau is found bit by bit from the top: keep a bit
+//      when at least K' keys are >= the prefix with it (counts by redux.sync).
+//   2. All keys > tau are selected; among keys == tau the lowest ids fill the
+//      remaining slots (ballots in id order).
+//   3. The K' selected (key, id) pairs are compacted to lanes 0..K'-1 and put in
+//      slot order by a warp bitonic sort on (key descending, id ascending).
+// Every step is exact integer work on the keys: no floating-point comparison
+// other than the fp32 values the keys encode.
+
+// Order-preserving map of an fp32 value to an unsigned key (larger value, larger key).
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t u = __float_as_uint(v);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// (key, id) a precedes b: larger key first, then lower id.
+__device__ __forceinline__ bool slot_before(uint32_t ka, uint32_t ia, uint32_t kb, uint32_t ib) {
+    return ka > kb || (ka == kb && ia < ib);
+}
+
 template <int NPL>
 __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int ld,
                                                            const float* __restrict__ bias, int T, int n_tot, int K,
                                                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
-    const int lane = threadIdx.x & 31;
-    const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    __shared__ uint32_t s_key[8][32], s_id[8][32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= T) return;
     const float* row = logits + static_cast<size_t>(t) * ld;
-    float v[NPL];
-    uint32_t taken = 0;
+    uint32_t key[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < n_tot) {
-            v[i] = row[e] + (bias != nullptr ? bias[e] : 0.0f);
-        } else {
-            v[i] = -FLT_MAX;
-            taken |= 1u << i;
-        }
+        key[i] = e < n_tot ? order_key(row[e] + (bias != nullptr ? bias[e] : 0.0f)) : 0u;  // 0: no expert
     }
-    float sel_v = -FLT_MAX;
-    int sel_e = 0;
+    // 1. tau = the K'-th largest key
+    uint32_t tau = 0;
 #pragma unroll 1
-    for (int k = 0; k < K; ++k) {
-        float bv = -FLT_MAX;
-        int be = INT_MAX;
+    for (int b = 31; b >= 0; --b) {
+        const uint32_t cand = tau | (1u << b);
+        uint32_t c = 0;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i)
-            if (!((taken >> i) & 1u) && (be == INT_MAX || v[i] > bv)) {
-                bv = v[i];
-                be = lane + 32 * i;
-            }
+        for (int i = 0; i < NPL; ++i) c += key[i] >= cand ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(K)) tau = cand;
+    }
+    // 2. selection: keys above tau, then the lowest ids among keys equal to tau
+    uint32_t gt = 0;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-            const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-            if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
-                bv = ov;
-                be = oe;
-            }
+    for (int i = 0; i < NPL; ++i) gt += key[i] > tau ? 1u : 0u;
+    int need = K - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    const uint32_t below = (1u << lane) - 1u;
+    uint32_t sel = 0;  // bit i: key[i] selected
+    int before = 0;    // tied ids already taken in lower rows i
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const uint32_t tie = __ballot_sync(0xffffffffu, key[i] == tau);
+        const int order = before + __popc(tie & below);
+        if (key[i] > tau || (key[i] == tau && order < need)) sel |= 1u << i;
+        before += __popc(tie);
+    }
+    // 3. compact to lanes 0..K'-1 in id order, then bitonic sort into slot order
+    int base = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const uint32_t m = __ballot_sync(0xffffffffu, (sel >> i) & 1u);
+        if ((sel >> i) & 1u) {
+            const int c = base + __popc(m & below);
+            s_key[warp][c] = key[i];
+            s_id[warp][c] = static_cast<uint32_t>(lane + 32 * i);
         }
-        if ((be & 31) == lane) taken |= 1u << (be >> 5);
-        if (lane == k) {
-            sel_v = bv;
-            sel_e = be;
+        base += __popc(m);
+    }
+    __syncwarp();
+    uint32_t mk = lane < K ? s_key[warp][lane] : 0u;
+    uint32_t mi = lane < K ? s_id[warp][lane] : 0xffffffffu;
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            const uint32_t ok = __shfl_xor_sync(0xffffffffu, mk, stride);
+            const uint32_t oi = __shfl_xor_sync(0xffffffffu, mi, stride);
+            const bool lower = (lane & stride) == 0;          // this lane keeps the earlier slot of the pair
+            const bool ascending = (lane & size) == 0;        // direction of this bitonic block (slot order)
+            const bool mine_first = slot_before(mk, mi, ok, oi);
+            if (lower == ascending ? !mine_first : mine_first) {
+                mk = ok;
+                mi = oi;
+            }
         }
     }
+    const float sel_v = key_value(mk);
     const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
     const float ex = lane < K ? expf(sel_v - vmax) : 0.0f;
     float sum = ex;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     if (lane < K) {
-        idx_out[static_cast<size_t>(t) * K + lane] = sel_e;
+        idx_out[static_cast<size_t>(t) * K + lane] = static_cast<int32_t>(mi);
         w_out[static_cast<size_t>(t) * K + lane] = ex / sum;
     }
 }
@@ -202,6 +249,94 @@ __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __res
     }
 }
 
+// Small batches (T <= 256): bitmap, per-expert prefix, offsets, tile lists and
+// the placement (perm / inv) in one block of 1024 threads, the bitmap in shared
+// memory.  The same positions as the multi-kernel path:
+//   pos = offsets[e] + prefix[w][e] + popcount(bits[w][e] below bit t % 32).
+constexpr int SMALL_BATCH_WORDS = 8;
+
+__global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
+                                                              int n_ffn, int small_max, int* __restrict__ counts,
+                                                              int* __restrict__ offsets, int4* __restrict__ mt_list,
+                                                              int4* __restrict__ small_list, int32_t* __restrict__ perm,
+                                                              int32_t* __restrict__ inv, int* __restrict__ hdr) {
+    extern __shared__ uint32_t sm[];  // bits[nwords][n_tot], prefix[nwords][n_tot], base[n_tot]
+    __shared__ int scratch[33];
+    const int nwords = (T + 31) >> 5;
+    uint32_t* bits = sm;
+    uint32_t* prefix = sm + nwords * n_tot;
+    int* base = reinterpret_cast<int*>(prefix + nwords * n_tot);
+    for (int i = threadIdx.x; i < nwords * n_tot; i += blockDim.x) bits[i] = 0;
+    __syncthreads();
+    const int slots = T * K;
+    for (int i = threadIdx.x; i < slots; i += blockDim.x) {
+        const int e = idx[i];
+        const int t = i / K;
+        if (e < 0 || e >= n_tot) {
+            atomicOr(&hdr[HDR_ERR], DEVERR_BAD_INDEX);
+            continue;
+        }
+        atomicOr(&bits[(t >> 5) * n_tot + e], 1u << (t & 31));
+    }
+    __syncthreads();
+    const int e = threadIdx.x;
+    int c = 0;
+    if (e < n_tot)
+        for (int w = 0; w < nwords; ++w) {
+            prefix[w * n_tot + e] = c;
+            c += __popc(bits[w * n_tot + e]);
+        }
+    int total;
+    const int off = block_exclusive_scan(c, scratch, &total);
+    if (e < n_tot) {
+        counts[e] = c;
+        offsets[e] = off;
+        base[e] = off;
+    }
+    if (e == 0) offsets[n_tot] = total;
+    const bool ffn = e < n_ffn;
+    const int ntile = (ffn && c > small_max) ? (c + 127) / 128 : 0;
+    const int small = (ffn && c > 0 && c <= small_max) ? 1 : 0;
+    int mt_total, small_total, rows_total;
+    const int mt_pos = block_exclusive_scan(ntile, scratch, &mt_total);
+    const int sm_pos = block_exclusive_scan(small, scratch, &small_total);
+    block_exclusive_scan(ffn ? c : 0, scratch, &rows_total);
+    for (int i = 0; i < ntile; ++i) mt_list[mt_pos + i] = make_int4(e, off + 128 * i, min(128, c - 128 * i), 0);
+    if (small) small_list[sm_pos] = make_int4(e, off, c, 0);
+    if (e == 0) {
+        hdr[HDR_ROWS] = rows_total;
+        hdr[HDR_MT] = mt_total;
+        hdr[HDR_NSMALL] = small_total;
+    }
+    __syncthreads();  // base[] visible to every thread
+    for (int i = threadIdx.x; i < slots; i += blockDim.x) {
+        const int ex = idx[i];
+        if (ex < 0 || ex >= n_tot) continue;
+        const int t = i / K, w = t >> 5;
+        const int cell = w * n_tot + ex;
+        const int pos = base[ex] + static_cast<int>(prefix[cell]) + __popc(bits[cell] & ((1u << (t & 31)) - 1u));
+        perm[pos] = i;
+        inv[i] = pos;
+    }
+}
+
+// One warp per slot: copy the token's feature row to its sorted row (FFN experts only).
+__global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ inv,
+                                                              int T, int K, int n_ffn,
+                                                              const __nv_bfloat16* __restrict__ feat, int ld_feat,
+                                                              int fdim, __nv_bfloat16* __restrict__ rows_out,
+                                                              int ld_rows) {
+    const int lane = threadIdx.x & 31;
+    const long i = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (i >= static_cast<long>(T) * K) return;
+    const int e = idx[i];
+    if (e < 0 || e >= n_ffn) return;
+    const int t = static_cast<int>(i / K);
+    const uint4* src = reinterpret_cast<const uint4*>(feat + static_cast<size_t>(t) * ld_feat);
+    uint4* dst = reinterpret_cast<uint4*>(rows_out + static_cast<size_t>(inv[i]) * ld_rows);
+    for (int c = lane; c < fdim / 8; c += 32) dst[c] = src[c];
+}
+
 // One warp per slot: place it (perm / inv) and, for FFN experts, copy the
 // token's feature row (latent z, or x for the standard MoE) to its sorted row.
 __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
@@ -232,136 +367,44 @@ __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int32_t* __
     }
 }
 
-// ============================================================================ decode experts
-// Experts that received only a few rows (decode) are bound by reading their
-// weights once.  Each work item is (list entry, block of 64 output columns);
-// a warp covers 8 columns with 4 lanes per column, streaming the weight rows
-// with 16-byte loads; the expert's rows (<= SMALL_MAX) sit in shared memory as
-// fp32, K in chunks of KCHUNK.  Accumulation is fp32 in a fixed order.
-constexpr int SMALL_MAX = 8;
-constexpr int GEMV_KCHUNK = 1024;
-constexpr int GEMV_THREADS = 256;
-constexpr int GEMV_COLS = 64;
-enum : int { GEMV_NONE = 0, GEMV_RELU2 = 1, GEMV_SWIGLU = 2 };
-
-template <int ACT>
-__global__ void __launch_bounds__(GEMV_THREADS) expert_stream_kernel(
-    const __nv_bfloat16* __restrict__ A, int ld_a, const __nv_bfloat16* __restrict__ W, int w_rows_per_expert,
-    int up_offset, int K, int n_out, __nv_bfloat16* __restrict__ out, int ld_out, const int4* __restrict__ list,
-    const int* __restrict__ list_count) {
-    __shared__ __align__(16) float sA[SMALL_MAX * GEMV_KCHUNK];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = lane & 3;
-    const int nblk = n_out / GEMV_COLS;
-    const int total = (*list_count) * nblk;
-    for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        const int j = item / nblk, nb = item % nblk;
-        const int4 L = list[j];
-        const int e = L.x, row0 = L.y, rows = L.z;
-        const int col = nb * GEMV_COLS + warp * 8 + (lane >> 2);
-        const __nv_bfloat16* wrow = W + (static_cast<size_t>(e) * w_rows_per_expert + col) * K;
-        const __nv_bfloat16* wrow2 = wrow + static_cast<size_t>(up_offset) * K;
-        float acc[SMALL_MAX], acc2[SMALL_MAX];
-#pragma unroll
-        for (int r = 0; r < SMALL_MAX; ++r) acc[r] = 0.f, acc2[r] = 0.f;
-        for (int k0 = 0; k0 < K; k0 += GEMV_KCHUNK) {
-            const int klen = min(GEMV_KCHUNK, K - k0);
-            __syncthreads();
-            for (int x = threadIdx.x; x < rows * (klen / 8); x += GEMV_THREADS) {
-                const int r = x / (klen / 8), c8 = x % (klen / 8);
-                const uint4 v = *reinterpret_cast<const uint4*>(A + static_cast<size_t>(row0 + r) * ld_a + k0 + c8 * 8);
-                float4* d = reinterpret_cast<float4*>(sA + r * GEMV_KCHUNK + c8 * 8);
-                d[0] = make_float4(bf16lo(v.x), bf16hi(v.x), bf16lo(v.y), bf16hi(v.y));
-                d[1] = make_float4(bf16lo(v.z), bf16hi(v.z), bf16lo(v.w), bf16hi(v.w));
-            }
-            __syncthreads();
-#pragma unroll 4
-            for (int c = q; c < klen / 8; c += 4) {
-                const uint4 wv = ld_stream_v4(wrow + k0 + c * 8);
-                const float w0 = bf16lo(wv.x), w1 = bf16hi(wv.x), w2 = bf16lo(wv.y), w3 = bf16hi(wv.y);
-                const float w4 = bf16lo(wv.z), w5 = bf16hi(wv.z), w6 = bf16lo(wv.w), w7 = bf16hi(wv.w);
-                float u0 = 0, u1 = 0, u2 = 0, u3 = 0, u4 = 0, u5 = 0, u6 = 0, u7 = 0;
-                if (ACT == GEMV_SWIGLU) {
-                    const uint4 uv = ld_stream_v4(wrow2 + k0 + c * 8);
-                    u0 = bf16lo(uv.x), u1 = bf16hi(uv.x), u2 = bf16lo(uv.y), u3 = bf16hi(uv.y);
-                    u4 = bf16lo(uv.z), u5 = bf16hi(uv.z), u6 = bf16lo(uv.w), u7 = bf16hi(uv.w);
-                }
-#pragma unroll
-                for (int r = 0; r < SMALL_MAX; ++r) {
-                    if (r < rows) {
-                        const float4 a0 = *reinterpret_cast<const float4*>(sA + r * GEMV_KCHUNK + c * 8);
-                        const float4 a1 = *reinterpret_cast<const float4*>(sA + r * GEMV_KCHUNK + c * 8 + 4);
-                        float s = acc[r];
-                        s = fmaf(w0, a0.x, s); s = fmaf(w1, a0.y, s); s = fmaf(w2, a0.z, s); s = fmaf(w3, a0.w, s);
-                        s = fmaf(w4, a1.x, s); s = fmaf(w5, a1.y, s); s = fmaf(w6, a1.z, s); s = fmaf(w7, a1.w, s);
-                        acc[r] = s;
-                        if (ACT == GEMV_SWIGLU) {
-                            float s2 = acc2[r];
-                            s2 = fmaf(u0, a0.x, s2); s2 = fmaf(u1, a0.y, s2); s2 = fmaf(u2, a0.z, s2); s2 = fmaf(u3, a0.w, s2);
-                            s2 = fmaf(u4, a1.x, s2); s2 = fmaf(u5, a1.y, s2); s2 = fmaf(u6, a1.z, s2); s2 = fmaf(u7, a1.w, s2);
-                            acc2[r] = s2;
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < SMALL_MAX; ++r) {
-            acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
-            acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 2);
-            if (ACT == GEMV_SWIGLU) {
-                acc2[r] += __shfl_xor_sync(0xffffffffu, acc2[r], 1);
-                acc2[r] += __shfl_xor_sync(0xffffffffu, acc2[r], 2);
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < SMALL_MAX; ++r) {
-            if (r < rows && (r & 3) == q) {
-                float v = acc[r];
-                if (ACT == GEMV_RELU2) {
-                    v = fmaxf(v, 0.f);
-                    v = v * v;
-                } else if (ACT == GEMV_SWIGLU) {
-                    v = v / (1.0f + expf(-v)) * acc2[r];
-                }
-                out[static_cast<size_t>(row0 + r) * ld_out + col] = __float2bfloat16_rn(v);
-            }
-        }
-    }
-}
+// Experts with at most this many rows take the weight-streaming (swap-AB) GEMM.
+constexpr int SMALL_MAX = 32;
 
 // ============================================================================ combine
 // yl_t = sum_k w_tk * o_k in slot order (fp32), o_k the expert's output row, 0
 // (zero expert), the token's own feature row (copy expert) or the constant
 // vector; plus the residual when the layer has no up-projection.  One block per
-// token, 8 columns (16 bytes) per thread per step; no atomics.
+// token, 8 columns (16 bytes) per thread per step; no atomics.  The slot table
+// (source row, weight) is resolved once per token in shared memory so that the
+// K' row loads of a step are independent and issue back to back; a zero expert
+// contributes with weight 0 (adding +-0 leaves the fp32 sum unchanged).
 __global__ void __launch_bounds__(128) combine_kernel(
     const __nv_bfloat16* __restrict__ O, int ld_o, const int32_t* __restrict__ inv, const int32_t* __restrict__ idx,
     const float* __restrict__ w, const __nv_bfloat16* __restrict__ feat, int ld_feat,
     const __nv_bfloat16* __restrict__ const_vecs, int T, int K, int L, int n_ffn, int n_zero, int n_copy,
     const __nv_bfloat16* __restrict__ resid, int ld_resid, __nv_bfloat16* __restrict__ out, int ld_out) {
-    __shared__ int s_e[32], s_pos[32];
+    __shared__ const __nv_bfloat16* s_src[32];
     __shared__ float s_w[32];
     const int t = blockIdx.x;
     if (threadIdx.x < K) {
         const size_t i = static_cast<size_t>(t) * K + threadIdx.x;
-        s_e[threadIdx.x] = idx[i];
-        s_pos[threadIdx.x] = inv[i];
-        s_w[threadIdx.x] = w[i];
+        const int e = idx[i];
+        const __nv_bfloat16* src = feat + static_cast<size_t>(t) * ld_feat;  // copy expert (and zero: weight 0)
+        float wk = w[i];
+        if (e < n_ffn) src = O + static_cast<size_t>(inv[i]) * ld_o;
+        else if (e < n_ffn + n_zero) wk = 0.0f;
+        else if (e >= n_ffn + n_zero + n_copy) src = const_vecs + static_cast<size_t>(e - n_ffn - n_zero - n_copy) * L;
+        s_src[threadIdx.x] = src;
+        s_w[threadIdx.x] = wk;
     }
     __syncthreads();
     for (int c8 = threadIdx.x; c8 < L / 8; c8 += blockDim.x) {
         float acc[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+#pragma unroll 8
         for (int k = 0; k < K; ++k) {
-            const int e = s_e[k];
-            const __nv_bfloat16* src;
-            if (e < n_ffn) src = O + static_cast<size_t>(s_pos[k]) * ld_o;
-            else if (e < n_ffn + n_zero) continue;
-            else if (e < n_ffn + n_zero + n_copy) src = feat + static_cast<size_t>(t) * ld_feat;
-            else src = const_vecs + static_cast<size_t>(e - n_ffn - n_zero - n_copy) * L;
-            const uint4 v = *reinterpret_cast<const uint4*>(src + c8 * 8);
+            const uint4 v = *reinterpret_cast<const uint4*>(s_src[k] + c8 * 8);
             const float wk = s_w[k];
             acc[0] = fmaf(wk, bf16lo(v.x), acc[0]);
             acc[1] = fmaf(wk, bf16hi(v.x), acc[1]);

@@ -153,9 +153,10 @@ def lmoe_phase_times(h: int) -> Dict[str, tuple]:
 
 
 def lmoe_routing_stats(h: int) -> Dict[str, int]:
-    out = (I32 * 4)()
+    out = (I32 * 8)()
     _check("lmoe_routing_stats", lib().lmoe_routing_stats(h, out))
-    return {"ffn_rows": out[0], "experts_touched": out[1], "tc_mtiles": out[2], "stream_experts": out[3]}
+    return {"ffn_rows": out[0], "experts_touched": out[1], "tc_mtiles": out[2], "stream_experts": out[3],
+            "stream_rows": out[4], "tc_experts": out[5], "tc_rows": out[6], "small_rows_threshold": out[7]}
 
 
 def lmoe_set_small_rows(h: int, rows: int) -> None:

@@ -29,6 +29,8 @@ CASES = {
     "medium_identity_act": MEDIUM.with_(act="identity", seed=25),
     "medium_topk_all": MEDIUM.with_(n_ffn=8, top_k=8, seed=26),
     "medium_top1": MEDIUM.with_(top_k=1, seed=27),
+    "medium_16_tokens": MEDIUM.with_(tokens=16, seed=28),
+    "medium_17_tokens_swiglu": MEDIUM.with_(tokens=17, act="swiglu", n_copy=1, seed=29),
     "nemotron_decode": synth.WORKLOADS["nemotron_decode"],
     "std_decode": synth.WORKLOADS["std_decode"],
 }
@@ -60,7 +62,11 @@ def _run_and_check(cfg, layer, small_rows=None, sample=None):
         rows = np.arange(T) if sample is None else sample
         xs = layer["x"][rows]
         ref = oracle.forward(cfg, layer, x=xs, want=("y", "idx", "w", "logits", "z", "yl"))
-        differ = P.check_routing(gidx[rows], gw[rows], ref, cfg.top_k)
+        # With the latent router the gate reads the bf16 latent: where the GPU's fp32-accumulated z and the
+        # oracle's fp64 z round to neighbouring bf16 values, a logit moves by ~W_r * ulp(z) ~ 1e-4..1e-3,
+        # and the renormalised weights by as much; elsewhere the weights are fp32 softmaxes of fp32 logits.
+        w_atol = 1e-3 if cfg.latent_router else 2e-5
+        differ = P.check_routing(gidx[rows], gw[rows], ref, cfg.top_k, w_atol=w_atol)
         # logits (the GPU debug copy excludes the bias)
         lg_ref = ref["logits"] - (0 if layer["bias"] is None else layer["bias"].double().numpy())
         P.assert_close(P.to_np(dbg["logits"])[rows], lg_ref, "logits", max_vs_rms=2e-3, mean_rel=1e-3)
