@@ -203,6 +203,42 @@ LMOE_API int lmoe_set_wait_timeout(lmoe_handle *h, uint64_t ns);
 LMOE_API int lmoe_gemm_bf16(const void *A, const void *B, void *C, int32_t M, int32_t N, int32_t K, void *stream,
                    int *err_word);
 
+/*
+ * Expert counting sort without any caller-provided scratch.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory.  Examples are a plugin whose host framework
+ * owns the whole device-memory budget and gives it no allocation hook, and a
+ * latency-critical loop where the implicit device synchronisation of cudaMalloc
+ * is unacceptable.  Such callers cannot provide the workspace that lmoe_create
+ * needs.  This call does the same stable sort of the (token, slot) pairs by
+ * expert as lmoe_forward's dispatch step.  It uses the same kernels, with its
+ * scratch in a fixed device array of the library: a 2 MiB + 256 B bitmap /
+ * prefix / header area that every device which loads the library holds until
+ * the process exits.  It allocates nothing (no cudaMalloc, no cudaFree, no
+ * allocating library call).
+ *
+ *   idx      device int32 [T, top_k]: expert ids in [0, n_total) (out-of-range
+ *            ids are skipped and their slots left unset)
+ *   counts   device int32 [n_total]: rows per expert
+ *   offsets  device int32 [n_total + 1]: exclusive scan of counts
+ *   perm     device int32 [T * top_k]: the slot index t*top_k+k at each sorted
+ *            position
+ *   inv      device int32 [T * top_k]: the sorted position of each slot
+ *
+ * Limits: 0 <= T <= 8192 (else LMOE_ERR_TOO_MANY_TOKENS); 1 <= top_k <= 32,
+ * top_k <= n_total <= 1024 (else LMOE_ERR_UNSUPPORTED_SHAPE).  A rejected call
+ * enqueues no work.
+ * The first call on a device looks up the device address of the scratch array
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  Every call on a device shares the one scratch array, so
+ * calls whose work overlaps on the GPU (different streams, no ordering between
+ * them) race and corrupt each other's results; order them on one stream.
+ * Asynchronous on `stream`.
+ */
+LMOE_API int lmoe_dispatch_noalloc(const int32_t *idx, int32_t T, int32_t top_k, int32_t n_total, int32_t *counts,
+                                   int32_t *offsets, int32_t *perm, int32_t *inv, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -8,7 +8,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB = os.path.join(HERE, "liblmoe.so")
-SOURCES = [os.path.join(HERE, "csrc", "lmoe.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "lmoe.cu"), os.path.join(HERE, "csrc", "noalloc.cu")]
 DEPS = glob.glob(os.path.join(HERE, "csrc", "*")) + [os.path.join(HERE, "..", "include", "lmoe.h")]
 NVCC_FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-gencode", "arch=compute_100a,code=sm_100a",
               "-Xcompiler", "-fPIC", "-shared", "-Xcompiler", "-fvisibility=hidden"]

@@ -8,6 +8,9 @@
 
 namespace lmoe {
 
+// The non-template kernels below have internal linkage (static) so that more
+// than one translation unit of the library can include this header.
+
 // Workspace header words (int32), written on the device.
 enum : int {
     HDR_ERR = 0,        // device error bits
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 // at most once).  Every step is integer arithmetic: bit-exact and deterministic.
 
 // One warp per 32-token word; 8 words per block.
-__global__ void __launch_bounds__(256) dispatch_bitmap_kernel(const int32_t* __restrict__ idx, int T, int K,
+static __global__ void __launch_bounds__(256) dispatch_bitmap_kernel(const int32_t* __restrict__ idx, int T, int K,
                                                               int n_tot, uint32_t* __restrict__ bitmap,
                                                               int* __restrict__ hdr) {
     extern __shared__ uint32_t sbits[];  // [8][n_tot]
@@ -164,7 +167,7 @@ __global__ void __launch_bounds__(256) dispatch_bitmap_kernel(const int32_t* __r
 }
 
 // One warp per expert: exclusive prefix of per-word counts and the total.
-__global__ void __launch_bounds__(256) dispatch_expert_scan_kernel(const uint32_t* __restrict__ bitmap, int T,
+static __global__ void __launch_bounds__(256) dispatch_expert_scan_kernel(const uint32_t* __restrict__ bitmap, int T,
                                                                    int n_tot, uint32_t* __restrict__ prefix,
                                                                    int* __restrict__ counts) {
     const int lane = threadIdx.x & 31;
@@ -219,7 +222,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 // Single block of 1024 threads: offsets (exclusive scan of counts), the
 // tensor-core M-tile list (experts with more than `small_max` rows, split in
 // 128-row tiles) and the weight-streaming list (experts with 1..small_max rows).
-__global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __restrict__ counts, int n_tot, int n_ffn,
+static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __restrict__ counts, int n_tot, int n_ffn,
                                                                 int small_max, int* __restrict__ offsets,
                                                                 int4* __restrict__ mt_list, int4* __restrict__ small_list,
                                                                 int* __restrict__ hdr) {
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __res
 //   pos = offsets[e] + prefix[w][e] + popcount(bits[w][e] below bit t % 32).
 constexpr int SMALL_BATCH_WORDS = 8;
 
-__global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
+static __global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
                                                               int n_ffn, int small_max, int* __restrict__ counts,
                                                               int* __restrict__ offsets, int4* __restrict__ mt_list,
                                                               int4* __restrict__ small_list, int32_t* __restrict__ perm,
@@ -321,7 +324,7 @@ __global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __r
 }
 
 // One warp per slot: copy the token's feature row to its sorted row (FFN experts only).
-__global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ inv,
+static __global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ inv,
                                                               int T, int K, int n_ffn,
                                                               const __nv_bfloat16* __restrict__ feat, int ld_feat,
                                                               int fdim, __nv_bfloat16* __restrict__ rows_out,
@@ -339,7 +342,7 @@ __global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __r
 
 // One warp per slot: place it (perm / inv) and, for FFN experts, copy the
 // token's feature row (latent z, or x for the standard MoE) to its sorted row.
-__global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
+static __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
                                                                int n_ffn, const uint32_t* __restrict__ bitmap,
                                                                const uint32_t* __restrict__ prefix,
                                                                const int* __restrict__ offsets,
@@ -378,7 +381,7 @@ constexpr int SMALL_MAX = 32;
 // (source row, weight) is resolved once per token in shared memory so that the
 // K' row loads of a step are independent and issue back to back; a zero expert
 // contributes with weight 0 (adding +-0 leaves the fp32 sum unchanged).
-__global__ void __launch_bounds__(128) combine_kernel(
+static __global__ void __launch_bounds__(128) combine_kernel(
     const __nv_bfloat16* __restrict__ O, int ld_o, const int32_t* __restrict__ inv, const int32_t* __restrict__ idx,
     const float* __restrict__ w, const __nv_bfloat16* __restrict__ feat, int ld_feat,
     const __nv_bfloat16* __restrict__ const_vecs, int T, int K, int L, int n_ffn, int n_zero, int n_copy,

@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_set_small_rows.argtypes = [P, I32]
         L.lmoe_set_wait_timeout.argtypes = [P, ctypes.c_uint64]
         L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
+        L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
         _lib = L
     return _lib
 
@@ -173,6 +174,15 @@ def lmoe_gemm_bf16(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor, err: torch
     N = B.shape[0]
     _check("lmoe_gemm_bf16", lib().lmoe_gemm_bf16(A.data_ptr(), B.data_ptr(), C.data_ptr(), M, N, K, _stream(stream),
                                                   err.data_ptr()))
+
+
+def lmoe_dispatch_noalloc(idx: torch.Tensor, n_total: int, counts: torch.Tensor, offsets: torch.Tensor,
+                          perm: torch.Tensor, inv: torch.Tensor, stream=None) -> None:
+    """Expert counting sort of ``idx`` [T, top_k] (int32, device) into caller buffers, with no device
+    allocation: the library's fixed scratch array serves as workspace (see ``include/lmoe.h``)."""
+    T, K = idx.shape
+    _check("lmoe_dispatch_noalloc", lib().lmoe_dispatch_noalloc(
+        _p(idx), T, K, n_total, _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)))
 
 
 # ------------------------------------------------------------------ convenience owner of a layer
