@@ -140,6 +140,26 @@ bool set_smem_attr() {
                                 GemmCfg<BN>::SMEM_BYTES) == cudaSuccess;
 }
 
+// Kernel launch with programmatic dependent launch: the kernel may be placed
+// while its predecessor in the stream drains; every kernel of the layer waits
+// for its predecessor first thing (pdl_begin), so results are unchanged.
+bool g_use_pdl = true;
+
+template <typename... P, typename... A>
+void launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_use_pdl ? 1 : 0;
+    cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
+
 template <int NT, int EPI>
 bool set_swap_attr() {
     return cudaFuncSetAttribute(tc_swap_kernel<NT, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -170,7 +190,7 @@ bool set_all_smem_attrs() {
 template <int NT, int EPI>
 void launch_swap(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& w2, const SwapArgs& args, int grid,
                  cudaStream_t s) {
-    tc_swap_kernel<NT, EPI><<<grid, 192, SwapCfg<NT, EPI>::SMEM_BYTES, s>>>(w, x, w2, args);
+    launch(tc_swap_kernel<NT, EPI>, grid, 192, SwapCfg<NT, EPI>::SMEM_BYTES, s, w, x, w2, args);
 }
 
 // Weight-streaming launch for the experts of the small list, dispatched on the token tile and epilogue.
@@ -221,18 +241,17 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
     a.part_rows = (t0 + t1) * 128;
     a.err = err;
     a.timeout_ns = timeout_ns;
-    const int units = (t0 + t1) * splits;
-    const int grid = std::min(num_sms, units);
+    const int grid = std::min(num_sms, (t0 + t1) * splits);
     const long outs = static_cast<long>(g.rows0 + g.rows1) * T;
     const unsigned rgrid = static_cast<unsigned>((outs + 255) / 256);
     if (T <= 16) {
         launch_swap<16, EPI_BF16>(*g.w, *g.x16, *g.w2, a, grid, s);
-        swap_reduce_kernel<16><<<rgrid, 256, 0, s>>>(partial, a.part_rows, splits, T, g.rows0, g.rows1, t0 * 128,
-                                                      g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
+        launch(swap_reduce_kernel<16>, rgrid, 256, 0, s, static_cast<const float*>(partial), a.part_rows, splits, T,
+               g.rows0, g.rows1, t0 * 128, g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
     } else {
         launch_swap<32, EPI_BF16>(*g.w, *g.x32, *g.w2, a, grid, s);
-        swap_reduce_kernel<32><<<rgrid, 256, 0, s>>>(partial, a.part_rows, splits, T, g.rows0, g.rows1, t0 * 128,
-                                                      g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
+        launch(swap_reduce_kernel<32>, rgrid, 256, 0, s, static_cast<const float*>(partial), a.part_rows, splits, T,
+               g.rows0, g.rows1, t0 * 128, g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
     }
     return 2;
 }
@@ -240,7 +259,7 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
 template <int BN, int EPI>
 void launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args, int grid,
                  cudaStream_t s) {
-    tc_gemm_kernel<BN, EPI><<<grid, 192, GemmCfg<BN>::SMEM_BYTES, s>>>(a, b, b2, args);
+    launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, args);
 }
 
 }  // namespace
@@ -391,50 +410,50 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
             }
         }
     }
-    // ---------------------------------------------------------------- top-K' + softmax
-    {
-        PhaseScope ps(h, PH_TOPK, s, 1);
-        const int npl = (nt + 31) / 32;
-        const dim3 grid((T + 7) / 8), block(256);
-        const float* bias = h->w.router_bias;
-        if (npl <= 1) topk_softmax_kernel<1><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
-        else if (npl <= 2) topk_softmax_kernel<2><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
-        else if (npl <= 4) topk_softmax_kernel<4><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
-        else if (npl <= 8) topk_softmax_kernel<8><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
-        else if (npl <= 16) topk_softmax_kernel<16><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
-        else topk_softmax_kernel<32><<<grid, block, 0, s>>>(logits, p.ld_logits, bias, T, nt, K, idx, wts);
-    }
-    // ---------------------------------------------------------------- counting sort by expert
     // Experts with at most `small` rows stream their weights; when every expert
     // must (T <= small) the grouped GEMMs are not launched at all.
     int small = h->small_max;
     if (small > 0 && T <= SMALL_MAX) small = T <= 16 ? 16 : SMALL_MAX;
     const bool need_tc = T > small;
     h->last_small = small;
+    const int nwords = (T + 31) / 32;
+    int* counts = h->at<int>(p.counts);
+    int* offsets = h->at<int>(p.offsets);
+    int32_t* perm = h->at<int32_t>(p.perm);
+    int32_t* inv = h->at<int32_t>(p.inv);
+    const long slots = static_cast<long>(T) * K;
+    const int npl = (nt + 31) / 32;
+    const float* bias = h->w.router_bias;
+    // ---------------------------------------------------------------- top-K' + softmax
     {
-        const int nwords = (T + 31) / 32;
-        int* counts = h->at<int>(p.counts);
-        int* offsets = h->at<int>(p.offsets);
-        const long slots = static_cast<long>(T) * K;
-        if (nwords <= SMALL_BATCH_WORDS) {
-            PhaseScope ps(h, PH_DISPATCH, s, 2);
-            const size_t sm = (static_cast<size_t>(2 * nwords) * nt + nt) * 4;
-            dispatch_small_kernel<<<1, 1024, sm, s>>>(idx, T, K, nt, c.n_experts, small, counts, offsets, mt_list,
-                                                      small_list, h->at<int32_t>(p.perm), h->at<int32_t>(p.inv), hdr);
-            dispatch_gather_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
-                idx, h->at<int32_t>(p.inv), T, K, c.n_experts, feat, L, L, rows, L);
-        } else {
-            PhaseScope ps(h, PH_DISPATCH, s, 4);
-            uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
-            uint32_t* prefix = h->at<uint32_t>(p.prefix);
-            dispatch_bitmap_kernel<<<(nwords + 7) / 8, 256, 8 * nt * 4, s>>>(idx, T, K, nt, bitmap, hdr);
-            dispatch_expert_scan_kernel<<<(nt + 7) / 8, 256, 0, s>>>(bitmap, T, nt, prefix, counts);
-            dispatch_offsets_kernel<<<1, 1024, 0, s>>>(counts, nt, c.n_experts, small, offsets, mt_list, small_list,
-                                                       hdr);
-            dispatch_scatter_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
-                idx, T, K, nt, c.n_experts, bitmap, prefix, offsets, feat, L, L, rows, L, h->at<int32_t>(p.perm),
-                h->at<int32_t>(p.inv));
-        }
+        PhaseScope ps(h, PH_TOPK, s, 1);
+        const dim3 grid((T + 7) / 8), block(256);
+#define LMOE_TOPK(N) launch(topk_softmax_kernel<N>, grid, block, 0, s, logits, p.ld_logits, bias, T, nt, K, idx, wts)
+        if (npl <= 1) LMOE_TOPK(1);
+        else if (npl <= 2) LMOE_TOPK(2);
+        else if (npl <= 4) LMOE_TOPK(4);
+        else if (npl <= 8) LMOE_TOPK(8);
+        else if (npl <= 16) LMOE_TOPK(16);
+        else LMOE_TOPK(32);
+#undef LMOE_TOPK
+    }
+    // ---------------------------------------------------------------- counting sort by expert (+ row gather)
+    if (nwords <= SMALL_BATCH_WORDS) {
+        PhaseScope ps(h, PH_DISPATCH, s, 2);
+        const size_t sm = (static_cast<size_t>(2 * nwords) * nt + nt) * 4;
+        launch(dispatch_small_kernel, 1, 1024, sm, s, idx, T, K, nt, c.n_experts, small, counts, offsets, mt_list,
+               small_list, perm, inv, hdr);
+        launch(dispatch_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
+               feat, L, L, rows, L);
+    } else {
+        PhaseScope ps(h, PH_DISPATCH, s, 4);
+        uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
+        uint32_t* prefix = h->at<uint32_t>(p.prefix);
+        launch(dispatch_bitmap_kernel, (nwords + 7) / 8, 256, 8 * nt * 4, s, idx, T, K, nt, bitmap, hdr);
+        launch(dispatch_expert_scan_kernel, (nt + 7) / 8, 256, 0, s, bitmap, T, nt, prefix, counts);
+        launch(dispatch_offsets_kernel, 1, 1024, 0, s, counts, nt, c.n_experts, small, offsets, mt_list, small_list, hdr);
+        launch(dispatch_scatter_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, T, K, nt, c.n_experts,
+               bitmap, prefix, offsets, feat, L, L, rows, L, perm, inv);
     }
     // ---------------------------------------------------------------- expert up (+ activation)
     if (need_tc) {
@@ -512,9 +531,10 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     {
         PhaseScope ps(h, PH_COMBINE, s, 1);
         __nv_bfloat16* out = proj ? h->at<__nv_bfloat16>(p.yl) : yb;
-        combine_kernel<<<T, 128, 0, s>>>(rows, L, h->at<int32_t>(p.inv), idx, wts, feat, L,
-                                          static_cast<const __nv_bfloat16*>(h->w.const_vecs), T, K, L, c.n_experts,
-                                          c.n_zero, c.n_copy, proj ? nullptr : xb, d, out, proj ? L : d);
+        launch(combine_kernel, T, 128, 0, s, static_cast<const __nv_bfloat16*>(rows), L,
+               static_cast<const int32_t*>(inv), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
+               feat, L, static_cast<const __nv_bfloat16*>(h->w.const_vecs), T, K, L, c.n_experts, c.n_zero, c.n_copy,
+               proj ? static_cast<const __nv_bfloat16*>(nullptr) : xb, d, out, proj ? L : d);
     }
     // ---------------------------------------------------------------- W_up + residual
     if (proj && T <= kFewTokenRows) {

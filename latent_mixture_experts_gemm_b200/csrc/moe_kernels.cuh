@@ -49,15 +49,13 @@ __device__ __forceinline__ bool slot_before(uint32_t ka, uint32_t ia, uint32_t k
     return ka > kb || (ka == kb && ia < ib);
 }
 
+// Top-K' and renormalised softmax of one token, by one warp.  s_key / s_id:
+// 32 words each of this warp's shared memory.
 template <int NPL>
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int ld,
-                                                           const float* __restrict__ bias, int T, int n_tot, int K,
-                                                           int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
-    __shared__ uint32_t s_key[8][32], s_id[8][32];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
-    if (t >= T) return;
-    const float* row = logits + static_cast<size_t>(t) * ld;
+__device__ __forceinline__ void topk_one_token(const float* __restrict__ row, const float* __restrict__ bias,
+                                               int n_tot, int K, uint32_t* s_key, uint32_t* s_id,
+                                               int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+    const int lane = threadIdx.x & 31;
     uint32_t key[NPL];
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
@@ -78,7 +76,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
     uint32_t gt = 0;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) gt += key[i] > tau ? 1u : 0u;
-    int need = K - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    const int need = K - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
     const uint32_t below = (1u << lane) - 1u;
     uint32_t sel = 0;  // bit i: key[i] selected
     int before = 0;    // tied ids already taken in lower rows i
@@ -96,22 +94,22 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
         const uint32_t m = __ballot_sync(0xffffffffu, (sel >> i) & 1u);
         if ((sel >> i) & 1u) {
             const int c = base + __popc(m & below);
-            s_key[warp][c] = key[i];
-            s_id[warp][c] = static_cast<uint32_t>(lane + 32 * i);
+            s_key[c] = key[i];
+            s_id[c] = static_cast<uint32_t>(lane + 32 * i);
         }
         base += __popc(m);
     }
     __syncwarp();
-    uint32_t mk = lane < K ? s_key[warp][lane] : 0u;
-    uint32_t mi = lane < K ? s_id[warp][lane] : 0xffffffffu;
+    uint32_t mk = lane < K ? s_key[lane] : 0u;
+    uint32_t mi = lane < K ? s_id[lane] : 0xffffffffu;
 #pragma unroll
     for (int size = 2; size <= 32; size <<= 1) {
 #pragma unroll
         for (int stride = size >> 1; stride > 0; stride >>= 1) {
             const uint32_t ok = __shfl_xor_sync(0xffffffffu, mk, stride);
             const uint32_t oi = __shfl_xor_sync(0xffffffffu, mi, stride);
-            const bool lower = (lane & stride) == 0;          // this lane keeps the earlier slot of the pair
-            const bool ascending = (lane & size) == 0;        // direction of this bitonic block (slot order)
+            const bool lower = (lane & stride) == 0;    // this lane keeps the earlier slot of the pair
+            const bool ascending = (lane & size) == 0;  // direction of this bitonic block (slot order)
             const bool mine_first = slot_before(mk, mi, ok, oi);
             if (lower == ascending ? !mine_first : mine_first) {
                 mk = ok;
@@ -126,9 +124,22 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     if (lane < K) {
-        idx_out[static_cast<size_t>(t) * K + lane] = static_cast<int32_t>(mi);
-        w_out[static_cast<size_t>(t) * K + lane] = ex / sum;
+        idx_out[lane] = static_cast<int32_t>(mi);
+        w_out[lane] = ex / sum;
     }
+}
+
+template <int NPL>
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int ld,
+                                                           const float* __restrict__ bias, int T, int n_tot, int K,
+                                                           int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+    pdl_begin();
+    __shared__ uint32_t s_key[8][32], s_id[8][32];
+    const int warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t >= T) return;
+    topk_one_token<NPL>(logits + static_cast<size_t>(t) * ld, bias, n_tot, K, s_key[warp], s_id[warp],
+                        idx_out + static_cast<size_t>(t) * K, w_out + static_cast<size_t>(t) * K);
 }
 
 // ============================================================================ dispatch
@@ -143,6 +154,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 static __global__ void __launch_bounds__(256) dispatch_bitmap_kernel(const int32_t* __restrict__ idx, int T, int K,
                                                               int n_tot, uint32_t* __restrict__ bitmap,
                                                               int* __restrict__ hdr) {
+    pdl_begin();
     extern __shared__ uint32_t sbits[];  // [8][n_tot]
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int word = blockIdx.x * 8 + warp;
@@ -170,6 +182,7 @@ static __global__ void __launch_bounds__(256) dispatch_bitmap_kernel(const int32
 static __global__ void __launch_bounds__(256) dispatch_expert_scan_kernel(const uint32_t* __restrict__ bitmap, int T,
                                                                    int n_tot, uint32_t* __restrict__ prefix,
                                                                    int* __restrict__ counts) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (e >= n_tot) return;
@@ -226,6 +239,7 @@ static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int
                                                                 int small_max, int* __restrict__ offsets,
                                                                 int4* __restrict__ mt_list, int4* __restrict__ small_list,
                                                                 int* __restrict__ hdr) {
+    pdl_begin();
     __shared__ int scratch[33];
     const int e = threadIdx.x;
     const int c = e < n_tot ? counts[e] : 0;
@@ -258,13 +272,14 @@ static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int
 //   pos = offsets[e] + prefix[w][e] + popcount(bits[w][e] below bit t % 32).
 constexpr int SMALL_BATCH_WORDS = 8;
 
-static __global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
-                                                              int n_ffn, int small_max, int* __restrict__ counts,
-                                                              int* __restrict__ offsets, int4* __restrict__ mt_list,
-                                                              int4* __restrict__ small_list, int32_t* __restrict__ perm,
-                                                              int32_t* __restrict__ inv, int* __restrict__ hdr) {
-    extern __shared__ uint32_t sm[];  // bits[nwords][n_tot], prefix[nwords][n_tot], base[n_tot]
-    __shared__ int scratch[33];
+// Body of the small-batch dispatch for a block of 1024 threads.  `sm` holds
+// (2 * nwords + 1) * n_tot words of dynamic shared memory; `scratch` 33 ints.
+__device__ __forceinline__ void dispatch_small_body(const int32_t* __restrict__ idx, int T, int K, int n_tot,
+                                                    int n_ffn, int small_max, int* __restrict__ counts,
+                                                    int* __restrict__ offsets, int4* __restrict__ mt_list,
+                                                    int4* __restrict__ small_list, int32_t* __restrict__ perm,
+                                                    int32_t* __restrict__ inv, int* __restrict__ hdr, uint32_t* sm,
+                                                    int* scratch) {
     const int nwords = (T + 31) >> 5;
     uint32_t* bits = sm;
     uint32_t* prefix = sm + nwords * n_tot;
@@ -323,12 +338,25 @@ static __global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32
     }
 }
 
+static __global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
+                                                              int n_ffn, int small_max, int* __restrict__ counts,
+                                                              int* __restrict__ offsets, int4* __restrict__ mt_list,
+                                                              int4* __restrict__ small_list, int32_t* __restrict__ perm,
+                                                              int32_t* __restrict__ inv, int* __restrict__ hdr) {
+    pdl_begin();
+    extern __shared__ uint32_t sm[];
+    __shared__ int scratch[33];
+    dispatch_small_body(idx, T, K, n_tot, n_ffn, small_max, counts, offsets, mt_list, small_list, perm, inv, hdr, sm,
+                        scratch);
+}
+
 // One warp per slot: copy the token's feature row to its sorted row (FFN experts only).
 static __global__ void __launch_bounds__(256) dispatch_gather_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ inv,
                                                               int T, int K, int n_ffn,
                                                               const __nv_bfloat16* __restrict__ feat, int ld_feat,
                                                               int fdim, __nv_bfloat16* __restrict__ rows_out,
                                                               int ld_rows) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const long i = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (i >= static_cast<long>(T) * K) return;
@@ -350,6 +378,7 @@ static __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int3
                                                                int fdim, __nv_bfloat16* __restrict__ rows_out,
                                                                int ld_rows, int32_t* __restrict__ perm,
                                                                int32_t* __restrict__ inv) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const long i = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (i >= static_cast<long>(T) * K) return;
@@ -386,6 +415,7 @@ static __global__ void __launch_bounds__(128) combine_kernel(
     const float* __restrict__ w, const __nv_bfloat16* __restrict__ feat, int ld_feat,
     const __nv_bfloat16* __restrict__ const_vecs, int T, int K, int L, int n_ffn, int n_zero, int n_copy,
     const __nv_bfloat16* __restrict__ resid, int ld_resid, __nv_bfloat16* __restrict__ out, int ld_out) {
+    pdl_begin();
     __shared__ const __nv_bfloat16* s_src[32];
     __shared__ float s_w[32];
     const int t = blockIdx.x;

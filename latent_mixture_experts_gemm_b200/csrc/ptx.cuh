@@ -17,6 +17,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Programmatic dependent launch.  Every kernel of the layer starts with
+// pdl_begin(): it lets the next kernel in the stream be launched now (its CTAs
+// are placed as SMs free up and run up to their own wait), then waits until the
+// previous kernel has completed and its memory is visible.  Every CTA waits
+// before it can exit, so completion stays ordered along the stream.  Without
+// the launch attribute both instructions are no-ops.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

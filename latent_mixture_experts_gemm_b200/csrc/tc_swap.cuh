@@ -108,6 +108,7 @@ template <int NT, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const __grid_constant__ CUtensorMap tmW2, const SwapArgs args) {
+    pdl_begin();
     using C = SwapCfg<NT, EPI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -293,6 +294,7 @@ __global__ void __launch_bounds__(256) swap_reduce_kernel(const float* __restric
                                                           __nv_bfloat16* __restrict__ out0, int ld0,
                                                           float* __restrict__ out1, int ld1,
                                                           const __nv_bfloat16* __restrict__ resid, int ld_resid) {
+    pdl_begin();
     const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int cols = n0 + n1;
     if (i >= static_cast<long>(cols) * T) return;
