@@ -531,7 +531,8 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     {
         PhaseScope ps(h, PH_COMBINE, s, 1);
         __nv_bfloat16* out = proj ? h->at<__nv_bfloat16>(p.yl) : yb;
-        launch(combine_kernel, T, 128, 0, s, static_cast<const __nv_bfloat16*>(rows), L,
+        auto kern = T <= 256 ? combine_kernel<32> : combine_kernel<8>;
+        launch(kern, T, 128, 0, s, static_cast<const __nv_bfloat16*>(rows), L,
                static_cast<const int32_t*>(inv), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
                feat, L, static_cast<const __nv_bfloat16*>(h->w.const_vecs), T, K, L, c.n_experts, c.n_zero, c.n_copy,
                proj ? static_cast<const __nv_bfloat16*>(nullptr) : xb, d, out, proj ? L : d);

@@ -49,73 +49,134 @@ __device__ __forceinline__ bool slot_before(uint32_t ka, uint32_t ia, uint32_t k
     return ka > kb || (ka == kb && ia < ib);
 }
 
+// One compare-exchange step of a warp bitonic network on (key, id) pairs in
+// slot order (larger key first, then lower id); `e` is the element's index in
+// the sequence, `size` the bitonic block length, `stride` the partner distance.
+__device__ __forceinline__ void bitonic_step(uint32_t& k, uint32_t& i, int e, int size, int stride, int lane) {
+    const uint32_t ok = __shfl_xor_sync(0xffffffffu, k, stride);
+    const uint32_t oi = __shfl_xor_sync(0xffffffffu, i, stride);
+    const bool lower = (lane & stride) == 0;  // this element keeps the earlier slot of the pair
+    const bool ascending = (e & size) == 0;   // direction of this bitonic block (slot order)
+    const bool mine_first = slot_before(k, i, ok, oi);
+    if (lower == ascending ? !mine_first : mine_first) {
+        k = ok;
+        i = oi;
+    }
+}
+
 // Top-K' and renormalised softmax of one token, by one warp.  s_key / s_id:
-// 32 words each of this warp's shared memory.
+// 64 words each of this warp's shared memory.
+//
+// Fast path: the K'-th largest of the 32 lane maxima is a lower bound of the
+// K'-th largest key (it is the K'-th largest of a subset), so every selected
+// key is among the keys at or above it.  When at most 64 keys qualify, they are
+// sorted outright (64-element warp bitonic sort) and the first K' are taken.
+// Otherwise the exact radix selection below runs.
 template <int NPL>
 __device__ __forceinline__ void topk_one_token(const float* __restrict__ row, const float* __restrict__ bias,
                                                int n_tot, int K, uint32_t* s_key, uint32_t* s_id,
                                                int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     const int lane = threadIdx.x & 31;
+    const uint32_t below = (1u << lane) - 1u;
     uint32_t key[NPL];
+    uint32_t lmax = 0;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
         key[i] = e < n_tot ? order_key(row[e] + (bias != nullptr ? bias[e] : 0.0f)) : 0u;  // 0: no expert
+        lmax = max(lmax, key[i]);
     }
-    // 1. tau = the K'-th largest key
-    uint32_t tau = 0;
-#pragma unroll 1
-    for (int b = 31; b >= 0; --b) {
-        const uint32_t cand = tau | (1u << b);
-        uint32_t c = 0;
+    // K'-th largest lane maximum (descending bitonic sort of the 32 maxima by key)
+    uint32_t sk = lmax, si = static_cast<uint32_t>(lane);
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) c += key[i] >= cand ? 1u : 0u;
-        if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(K)) tau = cand;
-    }
-    // 2. selection: keys above tau, then the lowest ids among keys equal to tau
-    uint32_t gt = 0;
+    for (int size = 2; size <= 32; size <<= 1)
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) gt += key[i] > tau ? 1u : 0u;
-    const int need = K - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
-    const uint32_t below = (1u << lane) - 1u;
-    uint32_t sel = 0;  // bit i: key[i] selected
-    int before = 0;    // tied ids already taken in lower rows i
+        for (int stride = size >> 1; stride > 0; stride >>= 1) bitonic_step(sk, si, lane, size, stride, lane);
+    const uint32_t lb = max(__shfl_sync(0xffffffffu, sk, K - 1), 1u);
+    uint32_t cand = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        const uint32_t tie = __ballot_sync(0xffffffffu, key[i] == tau);
-        const int order = before + __popc(tie & below);
-        if (key[i] > tau || (key[i] == tau && order < need)) sel |= 1u << i;
-        before += __popc(tie);
-    }
-    // 3. compact to lanes 0..K'-1 in id order, then bitonic sort into slot order
-    int base = 0;
+    for (int i = 0; i < NPL; ++i)
+        if (key[i] >= lb) cand |= 1u << i;
+    const int n_cand = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popc(cand))));
+
+    uint32_t mk, mi;
+    if (n_cand <= 64) {
+        // compact the candidates to 64 slots in id order, then sort them into slot order
+        int base = 0;
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-        const uint32_t m = __ballot_sync(0xffffffffu, (sel >> i) & 1u);
-        if ((sel >> i) & 1u) {
-            const int c = base + __popc(m & below);
-            s_key[c] = key[i];
-            s_id[c] = static_cast<uint32_t>(lane + 32 * i);
+        for (int i = 0; i < NPL; ++i) {
+            const uint32_t m = __ballot_sync(0xffffffffu, (cand >> i) & 1u);
+            if ((cand >> i) & 1u) {
+                const int c = base + __popc(m & below);
+                s_key[c] = key[i];
+                s_id[c] = static_cast<uint32_t>(lane + 32 * i);
+            }
+            base += __popc(m);
         }
-        base += __popc(m);
-    }
-    __syncwarp();
-    uint32_t mk = lane < K ? s_key[lane] : 0u;
-    uint32_t mi = lane < K ? s_id[lane] : 0xffffffffu;
+        __syncwarp();
+        uint32_t k0 = lane < n_cand ? s_key[lane] : 0u, i0 = lane < n_cand ? s_id[lane] : 0xffffffffu;
+        uint32_t k1 = lane + 32 < n_cand ? s_key[lane + 32] : 0u, i1 = lane + 32 < n_cand ? s_id[lane + 32] : 0xffffffffu;
+        __syncwarp();
 #pragma unroll
-    for (int size = 2; size <= 32; size <<= 1) {
+        for (int size = 2; size <= 64; size <<= 1) {
 #pragma unroll
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            const uint32_t ok = __shfl_xor_sync(0xffffffffu, mk, stride);
-            const uint32_t oi = __shfl_xor_sync(0xffffffffu, mi, stride);
-            const bool lower = (lane & stride) == 0;    // this lane keeps the earlier slot of the pair
-            const bool ascending = (lane & size) == 0;  // direction of this bitonic block (slot order)
-            const bool mine_first = slot_before(mk, mi, ok, oi);
-            if (lower == ascending ? !mine_first : mine_first) {
-                mk = ok;
-                mi = oi;
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                if (stride == 32) {  // partner in the same lane: element lane vs lane + 32 (ascending block)
+                    if (!slot_before(k0, i0, k1, i1)) {
+                        const uint32_t tk = k0, ti = i0;
+                        k0 = k1, i0 = i1, k1 = tk, i1 = ti;
+                    }
+                } else {
+                    bitonic_step(k0, i0, lane, size, stride, lane);
+                    bitonic_step(k1, i1, lane + 32, size, stride, lane);
+                }
             }
         }
+        mk = lane < K ? k0 : 0u;
+        mi = lane < K ? i0 : 0xffffffffu;
+    } else {
+        // exact radix selection: tau = the K'-th largest key, bit by bit from the top
+        uint32_t tau = 0;
+#pragma unroll 1
+        for (int b = 31; b >= 0; --b) {
+            const uint32_t c2 = tau | (1u << b);
+            uint32_t c = 0;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) c += key[i] >= c2 ? 1u : 0u;
+            if (__reduce_add_sync(0xffffffffu, c) >= static_cast<uint32_t>(K)) tau = c2;
+        }
+        // keys above tau, then the lowest ids among keys equal to tau
+        uint32_t gt = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) gt += key[i] > tau ? 1u : 0u;
+        const int need = K - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+        uint32_t sel = 0;
+        int before = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const uint32_t tie = __ballot_sync(0xffffffffu, key[i] == tau);
+            const int order = before + __popc(tie & below);
+            if (key[i] > tau || (key[i] == tau && order < need)) sel |= 1u << i;
+            before += __popc(tie);
+        }
+        int base = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            const uint32_t m = __ballot_sync(0xffffffffu, (sel >> i) & 1u);
+            if ((sel >> i) & 1u) {
+                const int c = base + __popc(m & below);
+                s_key[c] = key[i];
+                s_id[c] = static_cast<uint32_t>(lane + 32 * i);
+            }
+            base += __popc(m);
+        }
+        __syncwarp();
+        mk = lane < K ? s_key[lane] : 0u;
+        mi = lane < K ? s_id[lane] : 0xffffffffu;
+#pragma unroll
+        for (int size = 2; size <= 32; size <<= 1)
+#pragma unroll
+            for (int stride = size >> 1; stride > 0; stride >>= 1) bitonic_step(mk, mi, lane, size, stride, lane);
     }
     const float sel_v = key_value(mk);
     const float vmax = __shfl_sync(0xffffffffu, sel_v, 0);
@@ -134,7 +195,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
                                                            const float* __restrict__ bias, int T, int n_tot, int K,
                                                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     pdl_begin();
-    __shared__ uint32_t s_key[8][32], s_id[8][32];
+    __shared__ uint32_t s_key[8][64], s_id[8][64];
     const int warp = threadIdx.x >> 5;
     const int t = blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= T) return;
@@ -410,7 +471,8 @@ constexpr int SMALL_MAX = 32;
 // (source row, weight) is resolved once per token in shared memory so that the
 // K' row loads of a step are independent and issue back to back; a zero expert
 // contributes with weight 0 (adding +-0 leaves the fp32 sum unchanged).
-static __global__ void __launch_bounds__(128) combine_kernel(
+template <int UNROLL>
+__global__ void __launch_bounds__(128) combine_kernel(
     const __nv_bfloat16* __restrict__ O, int ld_o, const int32_t* __restrict__ inv, const int32_t* __restrict__ idx,
     const float* __restrict__ w, const __nv_bfloat16* __restrict__ feat, int ld_feat,
     const __nv_bfloat16* __restrict__ const_vecs, int T, int K, int L, int n_ffn, int n_zero, int n_copy,
@@ -435,10 +497,19 @@ static __global__ void __launch_bounds__(128) combine_kernel(
         float acc[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-#pragma unroll 8
-        for (int k = 0; k < K; ++k) {
-            const uint4 v = *reinterpret_cast<const uint4*>(s_src[k] + c8 * 8);
-            const float wk = s_w[k];
+        // UNROLL slot rows are loaded before their FMAs (all K' <= 32 of them for small
+        // batches, where latency rules; fewer, for more resident blocks, for large
+        // batches, where bandwidth does); the sum always runs in slot order
+        for (int k0 = 0; k0 < K; k0 += UNROLL) {
+        uint4 rowv[UNROLL];
+#pragma unroll
+        for (int k = 0; k < UNROLL; ++k)
+            if (k0 + k < K) rowv[k] = *reinterpret_cast<const uint4*>(s_src[k0 + k] + c8 * 8);
+#pragma unroll
+        for (int k = 0; k < UNROLL; ++k) {
+            if (k0 + k >= K) break;
+            const uint4 v = rowv[k];
+            const float wk = s_w[k0 + k];
             acc[0] = fmaf(wk, bf16lo(v.x), acc[0]);
             acc[1] = fmaf(wk, bf16hi(v.x), acc[1]);
             acc[2] = fmaf(wk, bf16lo(v.y), acc[2]);
@@ -447,6 +518,7 @@ static __global__ void __launch_bounds__(128) combine_kernel(
             acc[5] = fmaf(wk, bf16hi(v.z), acc[5]);
             acc[6] = fmaf(wk, bf16lo(v.w), acc[6]);
             acc[7] = fmaf(wk, bf16hi(v.w), acc[7]);
+        }
         }
         if (resid != nullptr) {
             const uint4 r = *reinterpret_cast<const uint4*>(resid + static_cast<size_t>(t) * ld_resid + c8 * 8);

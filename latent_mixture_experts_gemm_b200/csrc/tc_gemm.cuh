@@ -117,6 +117,20 @@ __device__ __forceinline__ float act_relu2(float v) {
 }
 __device__ __forceinline__ float act_silu_mul(float g, float u) { return g / (1.0f + expf(-g)) * u; }
 
+// Residual of 64 output columns starting at pair column `pc` of the tile (zeros where not needed).
+template <int BN>
+__device__ __forceinline__ void epi_load_resid(const GemmArgs& a, const TileJob& j, int pc, bool row_ok, size_t row,
+                                               uint4 (&rs)[8]) {
+    const int col = j.col0 + pc;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const bool ok = row_ok && col + 32 * h < a.N0;
+        const uint4* src = reinterpret_cast<const uint4*>(a.resid + row * a.ld_resid + col + 32 * h);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) rs[4 * h + i] = ok ? src[i] : make_uint4(0, 0, 0, 0);
+    }
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -249,6 +263,12 @@ __global__ void __launch_bounds__(192, 1)
             tile_job<BN, EPI>(args, t, j);
             const int buf = it & 1;
             const uint32_t use = (it >> 1) & 1;
+            const bool row_ok = row_in_tile < j.rows;
+            const size_t row = static_cast<size_t>(j.a_row0) + row_in_tile;
+            // The residual of the first 64 columns is requested before the accumulator
+            // is ready; each later 64-column pair is requested one pair ahead.
+            uint4 rs[8];
+            if (EPI == EPI_RESID) epi_load_resid<BN>(args, j, 0, row_ok, row, rs);
             // One lane waits and the verdict is broadcast, so the whole warp
             // either reads the accumulator (tcgen05.ld is warp-collective) or leaves.
             int ok = 1;
@@ -257,8 +277,6 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quad * 32) << 16);
-            const bool row_ok = row_in_tile < j.rows;
-            const size_t row = static_cast<size_t>(j.a_row0) + row_in_tile;
             if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
                 for (int c = 0; c < BN / 2; c += 32) {
@@ -281,56 +299,67 @@ __global__ void __launch_bounds__(192, 1)
                     }
                 }
             } else {
+                // 64 accumulator columns per tcgen05 wait
 #pragma unroll 1
-                for (int c = 0; c < BN; c += 32) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tbase + c, v);
-                    tmem_ld_wait();
-                    const int col = j.col0 + c;
-                    if (!row_ok) continue;
-                    if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
-                        float* dst = args.out1 + row * args.ld1 + col;
-                        if (col + 32 <= args.N1) {
-                            float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                    __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (col + i < args.N1) dst[i] = __uint_as_float(v[i]);
-                        }
-                        continue;
-                    }
-                    if (col >= args.N0) continue;
-                    float f[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-                    if (EPI == EPI_RELU2) {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
-                    }
+                for (int pc = 0; pc < BN; pc += 64) {
+                    uint32_t v2[2][32];
+                    tmem_ld_32x32b_x32(tbase + pc, v2[0]);
+                    tmem_ld_32x32b_x32(tbase + pc + 32, v2[1]);
+                    uint4 rs_now[8];
                     if (EPI == EPI_RESID) {
-                        const uint4* rs = reinterpret_cast<const uint4*>(args.resid + row * args.ld_resid + col);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint4 q = rs[i];
-                            f[8 * i + 0] += bf16lo(q.x);
-                            f[8 * i + 1] += bf16hi(q.x);
-                            f[8 * i + 2] += bf16lo(q.y);
-                            f[8 * i + 3] += bf16hi(q.y);
-                            f[8 * i + 4] += bf16lo(q.z);
-                            f[8 * i + 5] += bf16hi(q.z);
-                            f[8 * i + 6] += bf16lo(q.w);
-                            f[8 * i + 7] += bf16hi(q.w);
-                        }
+                        for (int i = 0; i < 8; ++i) rs_now[i] = rs[i];
+                        if (pc + 64 < BN) epi_load_resid<BN>(args, j, pc + 64, row_ok, row, rs);
                     }
-                    uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
+                    tmem_ld_wait();
+                    if (!row_ok) continue;
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(pack_bf16x2(f[8 * i + 0], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
-                                            pack_bf16x2(f[8 * i + 4], f[8 * i + 5]), pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t(&v)[32] = v2[h];
+                        const int col = j.col0 + pc + 32 * h;
+                        if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
+                            float* dst = args.out1 + row * args.ld1 + col;
+                            if (col + 32 <= args.N1) {
+                                float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                            } else {
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    if (col + i < args.N1) dst[i] = __uint_as_float(v[i]);
+                            }
+                            continue;
+                        }
+                        if (col >= args.N0) continue;
+                        float f[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+                        if (EPI == EPI_RELU2) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
+                        }
+                        if (EPI == EPI_RESID) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const uint4 q = rs_now[4 * h + i];
+                                f[8 * i + 0] += bf16lo(q.x);
+                                f[8 * i + 1] += bf16hi(q.x);
+                                f[8 * i + 2] += bf16lo(q.y);
+                                f[8 * i + 3] += bf16hi(q.y);
+                                f[8 * i + 4] += bf16lo(q.z);
+                                f[8 * i + 5] += bf16hi(q.z);
+                                f[8 * i + 6] += bf16lo(q.w);
+                                f[8 * i + 7] += bf16hi(q.w);
+                            }
+                        }
+                        uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pack_bf16x2(f[8 * i + 0], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
+                                                pack_bf16x2(f[8 * i + 4], f[8 * i + 5]), pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
+                    }
                 }
             }
             tc_fence_before();

@@ -300,8 +300,14 @@ __global__ void __launch_bounds__(256) swap_reduce_kernel(const float* __restric
     if (i >= static_cast<long>(cols) * T) return;
     const int n = static_cast<int>(i % cols), t = static_cast<int>(i / cols);
     const int prow = n < n0 ? n : p1 + (n - n0);
+    // all split loads issue together; the sum is still taken in split order
+    float pv[16];
+#pragma unroll
+    for (int s = 0; s < 16; ++s) pv[s] = s < splits ? partial[(static_cast<size_t>(s) * part_rows + prow) * NT + t] : 0.f;
     float v = 0.f;
-    for (int s = 0; s < splits; ++s) v += partial[(static_cast<size_t>(s) * part_rows + prow) * NT + t];
+#pragma unroll
+    for (int s = 0; s < 16; ++s)
+        if (s < splits) v += pv[s];
     if (n < n0) {
         if (resid != nullptr) v += __bfloat162float(resid[static_cast<size_t>(t) * ld_resid + n]);
         out0[static_cast<size_t>(t) * ld0 + n] = __float2bfloat16_rn(v);

@@ -30,6 +30,7 @@ CASES = {
     "medium_topk_all": MEDIUM.with_(n_ffn=8, top_k=8, seed=26),
     "medium_top1": MEDIUM.with_(top_k=1, seed=27),
     "medium_16_tokens": MEDIUM.with_(tokens=16, seed=28),
+    "medium_1024_experts_top32": MEDIUM.with_(n_ffn=1020, n_zero=2, n_copy=1, n_const=1, top_k=32, seed=30),
     "medium_17_tokens_swiglu": MEDIUM.with_(tokens=17, act="swiglu", n_copy=1, seed=29),
     "nemotron_decode": synth.WORKLOADS["nemotron_decode"],
     "std_decode": synth.WORKLOADS["std_decode"],
@@ -144,3 +145,23 @@ def test_smaller_batches_on_one_handle():
             mod.forward(torch.zeros((cfg.tokens + 1, cfg.d), dtype=torch.bfloat16, device="cuda"))
     finally:
         mod.close()
+
+
+def test_all_equal_logits_pick_the_lowest_ids():
+    """A zero router makes every logit equal: the top-K' are the K' lowest expert ids, weights 1/K'."""
+    for cfg in (MEDIUM.with_(seed=32), MEDIUM.with_(n_ffn=200, top_k=16, tokens=40, seed=33)):
+        layer = synth.make_layer(cfg)
+        layer["w_router"] = torch.zeros_like(layer["w_router"])
+        mod = lmoe.LatentMoE(cfg, layer, max_tokens=cfg.tokens)
+        try:
+            y, dbg = mod.forward(layer["x"].cuda(), debug=True)
+            torch.cuda.synchronize()
+            assert mod.last_error() == 0
+            idx = dbg["idx"].cpu().numpy()
+            assert np.array_equal(idx, np.broadcast_to(np.arange(cfg.top_k), idx.shape))
+            np.testing.assert_allclose(dbg["w"].cpu().numpy(), 1.0 / cfg.top_k, rtol=1e-6)
+            ref = oracle.forward(cfg, layer)
+            assert np.array_equal(ref["idx"], idx)
+            P.assert_close(P.to_np(y), ref["y"], "y")
+        finally:
+            mod.close()
