@@ -114,6 +114,24 @@ def _smi_id(device: int) -> str:
         return str(device)
 
 
+# ----------------------------------------------------------------------------- ranks
+def dist_barrier(world: int) -> None:
+    """Barrier over all ranks (no-op for one process)."""
+    if world > 1:
+        import torch.distributed as tdist
+        tdist.barrier()
+
+
+def dist_max(v: float, world: int, device: torch.device) -> float:
+    """Maximum of a per-rank value over all ranks (the job's time is the slowest rank's)."""
+    if world <= 1:
+        return v
+    import torch.distributed as tdist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- algorithmic work
 def layer_work(cfg, stats, T):
     """F (FLOPs) and B (bytes) of one forward from its actual routing."""
@@ -182,20 +200,9 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
             acc[k] = acc.get(k, 0) + v / len(xd)
     stats = acc
 
-    dist = world > 1
-    if dist:
-        import torch.distributed as tdist
-
-    def barrier():
-        if dist:
-            tdist.barrier()
-
-    def max_over_ranks(v: float) -> float:
-        if not dist:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=f"cuda:{device}")
-        tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
-        return float(t.item())
+    dev = torch.device(f"cuda:{device}")
+    barrier = lambda: dist_barrier(world)  # noqa: E731
+    max_over_ranks = lambda v: dist_max(v, world, dev)  # noqa: E731
 
     for i in range(warmup):
         mod.forward(xd[i % N_INPUT_BATCHES], yd)
