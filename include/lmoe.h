@@ -194,6 +194,15 @@ LMOE_API int lmoe_set_small_rows(lmoe_handle *h, int32_t rows);
 LMOE_API int lmoe_set_wait_timeout(lmoe_handle *h, uint64_t ns);
 
 /*
+ * Failure-path self-test: launch one thread that waits, with the bounded wait
+ * every kernel of the layer uses, on a barrier nothing ever arrives on.  After
+ * `timeout_ns` (1 .. 2e9) it gives up and records a timeout in the handle's
+ * device error word, so lmoe_last_error (after synchronising `stream`) returns
+ * LMOE_ERR_TIMEOUT; the CUDA context stays usable.  Asynchronous.
+ */
+LMOE_API int lmoe_selftest_wait(lmoe_handle *h, uint64_t timeout_ns, void *stream);
+
+/*
  * Plain GEMM on the layer's tensor-core kernel: C[M,N] = A[M,K] * B[N,K]^T,
  * bf16 in (device, row-major, K-major both), fp32 accumulate, bf16 out.
  * K a multiple of 64 (<= 65536), N a multiple of 64, M >= 0.  `err_word` is a

@@ -812,6 +812,12 @@ int lmoe_set_wait_timeout(lmoe_handle* h, uint64_t ns) {
     return LMOE_OK;
 }
 
+int lmoe_selftest_wait(lmoe_handle* h, uint64_t timeout_ns, void* stream) {
+    if (h == nullptr || timeout_ns == 0 || timeout_ns > 2000000000ull) return LMOE_ERR_INVALID_ARG;
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->at<int>(h->p.hdr) + HDR_ERR, timeout_ns);
+    return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
 int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, int32_t K, void* stream, int* err_word) {
     if (A == nullptr || B == nullptr || C == nullptr || err_word == nullptr) return LMOE_ERR_INVALID_ARG;
     if (M < 0 || N < 64 || N % 64 != 0 || K < 64 || K % 64 != 0 || K > 65536) return LMOE_ERR_UNSUPPORTED_SHAPE;

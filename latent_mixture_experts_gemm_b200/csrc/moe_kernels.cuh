@@ -463,6 +463,22 @@ static __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int3
 // Experts with at most this many rows take the weight-streaming (swap-AB) GEMM.
 constexpr int SMALL_MAX = 32;
 
+// ============================================================================ wait self-test
+// One thread waits, with the same bounded wait every kernel of the layer uses,
+// on an mbarrier that nothing ever arrives on: after `timeout_ns` it must give
+// up, set the timeout bit in `err` and return (no trap, no hang).
+static __global__ void wait_selftest_kernel(int* err, unsigned long long timeout_ns) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, err, timeout_ns);
+}
+
 // ============================================================================ combine
 // yl_t = sum_k w_tk * o_k in slot order (fp32), o_k the expert's output row, 0
 // (zero expert), the token's own feature row (copy expert) or the constant

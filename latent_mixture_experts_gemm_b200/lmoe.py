@@ -75,6 +75,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_set_wait_timeout.argtypes = [P, ctypes.c_uint64]
         L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
         L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
+        L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
         _lib = L
     return _lib
 
@@ -166,6 +167,10 @@ def lmoe_set_small_rows(h: int, rows: int) -> None:
 
 def lmoe_set_wait_timeout(h: int, ns: int) -> None:
     _check("lmoe_set_wait_timeout", lib().lmoe_set_wait_timeout(h, ns))
+
+
+def lmoe_selftest_wait(h: int, timeout_ns: int, stream=None) -> None:
+    _check("lmoe_selftest_wait", lib().lmoe_selftest_wait(h, timeout_ns, _stream(stream)))
 
 
 def lmoe_gemm_bf16(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor, err: torch.Tensor, stream=None) -> None:

@@ -165,3 +165,26 @@ def test_all_equal_logits_pick_the_lowest_ids():
             P.assert_close(P.to_np(y), ref["y"], "y")
         finally:
             mod.close()
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    """A wait on a barrier nothing arrives on ends after its bound with LMOE_ERR_TIMEOUT; the handle and the
+    context stay usable (the next forward is exact again and reports no error)."""
+    cfg = synth.WORKLOADS["tiny"]
+    layer = synth.make_layer(cfg)
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=cfg.tokens)
+    try:
+        x = layer["x"].cuda()
+        y0 = mod.forward(x)
+        torch.cuda.synchronize()
+        assert mod.last_error() == 0
+        lmoe.lmoe_selftest_wait(mod.h, 20_000_000)   # 20 ms
+        torch.cuda.synchronize()
+        assert mod.last_error() == -5                 # LMOE_ERR_TIMEOUT
+        assert mod.last_error() == 0                  # reading clears it
+        y1 = mod.forward(x)
+        torch.cuda.synchronize()
+        assert mod.last_error() == 0
+        assert torch.equal(y0, y1)
+    finally:
+        mod.close()
