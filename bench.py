@@ -134,7 +134,7 @@ def dist_max(v: float, world: int, device: torch.device) -> float:
 
 # ----------------------------------------------------------------------------- algorithmic work
 def layer_work(cfg, stats, T):
-    """F (FLOPs) and B (bytes) of one forward from its actual routing."""
+    """F (FLOPs) and B (bytes) of one forward from its actual routing (plus the shared expert, if any)."""
     g = 2 if cfg.gated else 1
     R, E = stats["ffn_rows"], stats["experts_touched"]
     d, L, m, nt = cfg.d, cfg.latent, cfg.m, cfg.n_total
@@ -144,6 +144,10 @@ def layer_work(cfg, stats, T):
     else:
         F = 2 * T * d * nt + 2 * (g + 1) * d * m * R
         B = 2 * ((g + 1) * d * m * E + d * nt) + 4 * T * d
+    ms = getattr(cfg, "shared_m", 0)
+    if ms:
+        F += 2 * T * (g + 1) * d * ms
+        B += 2 * (g + 1) * d * ms
     return float(F), float(B)
 
 
@@ -169,6 +173,9 @@ def phase_units(cfg, stats, T, phase):
         return 2.0 * T * d * n_out, 2.0 * (n_out * d + T * d) + T * (L * 2 if cfg.has_proj else 0) + 4.0 * T * nt
     if phase == "up_proj_gemm":
         return 2.0 * T * L * d, 2.0 * (d * L + T * L + 2 * T * d)
+    if phase == "shared_expert":
+        ms = getattr(cfg, "shared_m", 0)
+        return 2.0 * T * (g + 1) * d * ms, 2.0 * ((g + 1) * d * ms + T * (d + ms) + T * (ms + 2 * d))
     if phase == "combine":
         return 2.0 * T * cfg.top_k * L, 2.0 * (rows_tc + rows_st) * L + 2.0 * T * L
     return 0.0, 0.0
@@ -365,6 +372,7 @@ def run_reference(args, cfg, rank, world):
 def workload_config(cfg):
     return {"workload": cfg.name, "tokens": cfg.tokens, "d": cfg.d, "latent": cfg.latent, "m": cfg.m,
             "experts": cfg.n_ffn, "bypass_experts": [cfg.n_zero, cfg.n_copy, cfg.n_const], "top_k": cfg.top_k,
+            "shared_expert_width": cfg.shared_m,
             "act": ["relu2", "swiglu", "identity"][cfg.act], "projection": bool(cfg.has_proj),
             "l2": "inputs larger than L2 (the touched expert weights, read every step, exceed the 126 MB L2)",
             "parallelism": "replicas (tokens shard with no exchange)"}

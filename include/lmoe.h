@@ -18,6 +18,10 @@
  *   6. y_t = x_t + W_up yl_t, latent -> d ("How LatentMoE Works", step 3).
  * With has_proj = 0 (latent == d) there is no W_down / W_up: the standard MoE
  * of Figure 3a, y_t = x_t + yl_t.
+ * With shared_m > 0 a shared expert at the full width d (it stays at d like the
+ * gate: "LatentMoE: How MoE Made a Key Paradigm Leap in 2026", section 2,
+ * closing note) adds Ws2 act(Ws1 x_t), act as for the routed experts; it runs
+ * on a stream of the handle's own, concurrently with the routed path.
  *
  * Conventions for every entry point:
  *   - all matrices are row-major; bf16 tensors are passed as `void *` (IEEE
@@ -65,7 +69,8 @@ extern "C" {
  * Layer shape.  Constraints (else LMOE_ERR_UNSUPPORTED_SHAPE): d, latent and m
  * multiples of 64 and at most 16384; 1 <= top_k <= min(32, n_total);
  * n_total = n_experts + n_zero + n_copy + n_const <= 1024; n_experts >= 1;
- * max_tokens >= 1; has_proj == 0 requires latent == d.
+ * max_tokens >= 1; has_proj == 0 requires latent == d; shared_m is 0 or a
+ * multiple of 64 up to 16384.
  */
 typedef struct lmoe_config {
     int32_t d;             /* model width */
@@ -80,6 +85,7 @@ typedef struct lmoe_config {
     int32_t n_const;       /* MoE++ constant experts (last ids) */
     int32_t has_proj;      /* 1: LatentMoE with W_down / W_up; 0: standard MoE */
     int32_t latent_router; /* 1: the gate reads z (latent) instead of x (d) */
+    int32_t shared_m;      /* hidden width of the shared expert at d; 0: no shared expert */
 } lmoe_config;
 
 /* Device pointers to the layer's weights (bf16 unless stated).  n_total as above. */
@@ -91,6 +97,8 @@ typedef struct lmoe_weights {
     const void *w1;           /* [n_experts, g*m, latent], g = 2 for SwiGLU else 1 */
     const void *w2;           /* [n_experts, latent, m] */
     const void *const_vecs;   /* [n_const, latent]; may be NULL when n_const == 0 */
+    const void *w_shared1;    /* [g*shared_m, d] (gate rows first when gated); NULL when shared_m == 0 */
+    const void *w_shared2;    /* [d, shared_m]; NULL when shared_m == 0 */
 } lmoe_weights;
 
 /*

@@ -71,6 +71,7 @@ bool config_ok(const lmoe_config& c) {
     if (c.has_proj != 0 && c.has_proj != 1) return false;
     if (c.latent_router != 0 && c.latent_router != 1) return false;
     if (!c.has_proj && c.latent != c.d) return false;
+    if (c.shared_m != 0 && !dim_ok(c.shared_m)) return false;
     return true;
 }
 
@@ -81,7 +82,7 @@ constexpr int kFewTokenMaxSplits = 16;
 
 struct Plan {
     size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
-        partial, xin, yout, total;
+        partial, hs, s2, partial2, xin, yout, total;
     int ld_logits, nwords, mt_max;
 };
 
@@ -120,6 +121,13 @@ Plan make_plan(const lmoe_config& c) {
         const size_t rows = std::max(up128(L) + up128(nt), std::max(up128(d), up128(nt)));
         p.partial = take(static_cast<size_t>(kFewTokenMaxSplits) * rows * kFewTokenRows * 4);
     }
+    if (c.shared_m > 0) {  // shared expert: hidden rows, x + its output, its own split-K partials
+        const size_t g = c.act == LMOE_ACT_SWIGLU ? 2 : 1;
+        const size_t srows = std::max((g * c.shared_m + 127) / 128 * 128, (d + 127) / 128 * 128);
+        p.hs = take(T * static_cast<size_t>(c.shared_m) * 2);
+        p.s2 = take(T * d * 2);
+        p.partial2 = take(static_cast<size_t>(kFewTokenMaxSplits) * srows * kFewTokenRows * 4);
+    }
     p.xin = take(T * d * 2);
     p.yout = take(T * d * 2);
     p.total = off;
@@ -129,10 +137,10 @@ Plan make_plan(const lmoe_config& c) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 enum Phase : int { PH_ROUTER = 0, PH_TOPK, PH_DISPATCH, PH_UP_TC, PH_UP_STREAM, PH_DOWN_TC, PH_DOWN_STREAM, PH_COMBINE,
-                   PH_WUP, PH_COUNT };
+                   PH_WUP, PH_SHARED, PH_COUNT };
 const char* kPhaseNames[PH_COUNT] = {"router_proj_gemm", "topk_softmax", "dispatch", "expert_up_gemm",
                                      "expert_up_stream", "expert_down_gemm", "expert_down_stream", "combine",
-                                     "up_proj_gemm"};
+                                     "up_proj_gemm", "shared_expert"};
 
 template <int BN, int EPI>
 bool set_smem_attr() {
@@ -182,6 +190,8 @@ bool set_all_smem_attrs() {
     ok &= set_smem_attr<256, EPI_RESID>();
     ok &= set_smem_attr<64, EPI_PROJ_ROUTER>();
     ok &= set_smem_attr<256, EPI_PROJ_ROUTER>();
+    ok &= set_smem_attr<64, EPI_RELU2>();
+    ok &= set_smem_attr<64, EPI_SWIGLU>();
     ok &= set_smem_attr<256, EPI_RELU2>();
     ok &= set_smem_attr<256, EPI_SWIGLU>();
     return ok;
@@ -222,7 +232,24 @@ struct FewTokenGemm {
     int ld1;
     const __nv_bfloat16* resid;
     int ld_resid;
+    int act = EPI_BF16;     // activation of segment 0 (EPI_RELU2 / EPI_SWIGLU: gate rows first, then up rows)
+    int out_cols0 = -1;     // output columns of segment 0 (default rows0; rows0 / 2 when gated)
 };
+
+template <int NT>
+void launch_few_token_reduce(const FewTokenGemm& g, int T, const float* partial, int part_rows, int splits, int t0,
+                             cudaStream_t s) {
+    const int n0 = g.out_cols0 >= 0 ? g.out_cols0 : g.rows0;
+    const long outs = static_cast<long>(n0 + g.rows1) * T;
+    const unsigned rgrid = static_cast<unsigned>((outs + 255) / 256);
+#define LMOE_REDUCE(A)                                                                                           \
+    launch(swap_reduce_kernel<NT, A>, rgrid, 256, 0, s, partial, part_rows, splits, T, n0, g.rows1, t0 * 128, n0, \
+           g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid)
+    if (g.act == EPI_RELU2) LMOE_REDUCE(EPI_RELU2);
+    else if (g.act == EPI_SWIGLU) LMOE_REDUCE(EPI_SWIGLU);
+    else LMOE_REDUCE(EPI_BF16);
+#undef LMOE_REDUCE
+}
 
 int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_splits, int num_sms, int* err,
                      unsigned long long timeout_ns, cudaStream_t s) {
@@ -242,16 +269,12 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
     a.err = err;
     a.timeout_ns = timeout_ns;
     const int grid = std::min(num_sms, (t0 + t1) * splits);
-    const long outs = static_cast<long>(g.rows0 + g.rows1) * T;
-    const unsigned rgrid = static_cast<unsigned>((outs + 255) / 256);
     if (T <= 16) {
         launch_swap<16, EPI_BF16>(*g.w, *g.x16, *g.w2, a, grid, s);
-        launch(swap_reduce_kernel<16>, rgrid, 256, 0, s, static_cast<const float*>(partial), a.part_rows, splits, T,
-               g.rows0, g.rows1, t0 * 128, g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
+        launch_few_token_reduce<16>(g, T, partial, a.part_rows, splits, t0, s);
     } else {
         launch_swap<32, EPI_BF16>(*g.w, *g.x32, *g.w2, a, grid, s);
-        launch(swap_reduce_kernel<32>, rgrid, 256, 0, s, static_cast<const float*>(partial), a.part_rows, splits, T,
-               g.rows0, g.rows1, t0 * 128, g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid);
+        launch_few_token_reduce<32>(g, T, partial, a.part_rows, splits, t0, s);
     }
     return 2;
 }
@@ -280,6 +303,11 @@ struct lmoe_handle {
     CUtensorMap w1s{}, w2s{}, rows16{}, rows32{}, h16{}, h32{};
     // few-token projections: 128-row weight tiles and 16/32-row token tiles of z and yl
     CUtensorMap wdown128{}, wr128{}, wup128{}, z16{}, z32{}, yl16{}, yl32{};
+    // shared expert: weights for 64/256-column tiles (gated: half-tile boxes), 128-row weight tiles,
+    // its hidden rows as the A operand (128-row tiles) and as 16/32-row token tiles
+    CUtensorMap ws1_64{}, ws1_256{}, ws2_64{}, ws2_256{}, ws1_128{}, ws2_128{}, a_hs{}, hs16{}, hs32{};
+    cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
+    cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     // profiling
     bool prof = false;
     int prof_max = 0, prof_n = 0;
@@ -342,6 +370,75 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     GemmArgs base{};
     base.err = hdr + HDR_ERR;
     base.timeout_ns = h->timeout_ns;
+
+    // ---------------------------------------------------------------- shared expert (side stream)
+    // s2 = x + Ws2 act(Ws1 x) runs concurrently with the routed path; the up-projection
+    // (or, for the standard MoE, the combine) waits for it and adds s2 instead of x.
+    const __nv_bfloat16* resid = xb;
+    if (c.shared_m > 0) {
+        const int ms = c.shared_m, srows = h->g * ms;
+        __nv_bfloat16* hs = h->at<__nv_bfloat16>(p.hs);
+        __nv_bfloat16* s2 = h->at<__nv_bfloat16>(p.s2);
+        const int epi = c.act == LMOE_ACT_SWIGLU ? EPI_SWIGLU : (c.act == LMOE_ACT_RELU2 ? EPI_RELU2 : EPI_BF16);
+        if (cudaEventRecord(h->ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(h->side, h->ev_fork, 0) != cudaSuccess)
+            return LMOE_ERR_CUDA;
+        {
+            PhaseScope ps(h, PH_SHARED, h->side, T <= kFewTokenRows ? 4 : 2);
+            if (T <= kFewTokenRows) {
+                CUtensorMap x16, x32;
+                if (!make_map(&x16, x, T, d, d, 16) || !make_map(&x32, x, T, d, d, 32)) return LMOE_ERR_CUDA;
+                float* part2 = h->at<float>(p.partial2);
+                FewTokenGemm up{&h->ws1_128, &h->ws1_128, &x16, &x32, srows, 0, d, hs, ms, nullptr, 0, nullptr, 0};
+                up.act = epi;
+                up.out_cols0 = ms;
+                launch_few_token(up, T, part2, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, h->side);
+                FewTokenGemm dn{&h->ws2_128, &h->ws2_128, &h->hs16, &h->hs32, d, 0, ms, s2, d, nullptr, 0, xb, d};
+                launch_few_token(dn, T, part2, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, h->side);
+            } else {
+                GemmArgs a = base;
+                a.M = T;
+                a.K = d;
+                a.N0 = ms;
+                a.out0 = hs;
+                a.ld0 = ms;
+                a.up_offset = ms;
+                const bool big_up = m_tiles * ((ms + (epi == EPI_SWIGLU ? 127 : 255)) / (epi == EPI_SWIGLU ? 128 : 256)) >=
+                                    h->num_sms;
+                if (big_up) {
+                    a.n_tiles = epi == EPI_SWIGLU ? (ms + 127) / 128 : (ms + 255) / 256;
+                    const int grid = std::min(h->num_sms, m_tiles * a.n_tiles);
+                    if (epi == EPI_SWIGLU) launch_gemm<256, EPI_SWIGLU>(a_x, h->ws1_256, h->ws1_256, a, grid, h->side);
+                    else if (epi == EPI_RELU2) launch_gemm<256, EPI_RELU2>(a_x, h->ws1_256, h->ws1_256, a, grid, h->side);
+                    else launch_gemm<256, EPI_BF16>(a_x, h->ws1_256, h->ws1_256, a, grid, h->side);
+                } else {
+                    a.n_tiles = epi == EPI_SWIGLU ? (ms + 31) / 32 : (ms + 63) / 64;
+                    const int grid = std::min(h->num_sms, m_tiles * a.n_tiles);
+                    if (epi == EPI_SWIGLU) launch_gemm<64, EPI_SWIGLU>(a_x, h->ws1_64, h->ws1_64, a, grid, h->side);
+                    else if (epi == EPI_RELU2) launch_gemm<64, EPI_RELU2>(a_x, h->ws1_64, h->ws1_64, a, grid, h->side);
+                    else launch_gemm<64, EPI_BF16>(a_x, h->ws1_64, h->ws1_64, a, grid, h->side);
+                }
+                GemmArgs b = base;
+                b.M = T;
+                b.K = ms;
+                b.N0 = d;
+                b.out0 = s2;
+                b.ld0 = d;
+                b.resid = xb;
+                b.ld_resid = d;
+                if (m_tiles * ((d + 255) / 256) >= h->num_sms) {
+                    b.n_tiles = (d + 255) / 256;
+                    launch_gemm<256, EPI_RESID>(h->a_hs, h->ws2_256, h->ws2_256, b, std::min(h->num_sms, m_tiles * b.n_tiles),
+                                                h->side);
+                } else {
+                    b.n_tiles = (d + 63) / 64;
+                    launch_gemm<64, EPI_RESID>(h->a_hs, h->ws2_64, h->ws2_64, b, std::min(h->num_sms, m_tiles * b.n_tiles),
+                                               h->side);
+                }
+            }
+        }
+        if (cudaEventRecord(h->ev_join, h->side) != cudaSuccess) return LMOE_ERR_CUDA;
+        resid = s2;
+    }
 
     // ---------------------------------------------------------------- router (+ W_down)
     if (T <= kFewTokenRows) {
@@ -531,16 +628,18 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     {
         PhaseScope ps(h, PH_COMBINE, s, 1);
         __nv_bfloat16* out = proj ? h->at<__nv_bfloat16>(p.yl) : yb;
+        if (!proj && c.shared_m > 0 && cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess) return LMOE_ERR_CUDA;
         auto kern = T <= 256 ? combine_kernel<32> : combine_kernel<8>;
         launch(kern, T, 128, 0, s, static_cast<const __nv_bfloat16*>(rows), L,
                static_cast<const int32_t*>(inv), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
                feat, L, static_cast<const __nv_bfloat16*>(h->w.const_vecs), T, K, L, c.n_experts, c.n_zero, c.n_copy,
-               proj ? static_cast<const __nv_bfloat16*>(nullptr) : xb, d, out, proj ? L : d);
+               proj ? static_cast<const __nv_bfloat16*>(nullptr) : resid, d, out, proj ? L : d);
     }
     // ---------------------------------------------------------------- W_up + residual
+    if (proj && c.shared_m > 0 && cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess) return LMOE_ERR_CUDA;
     if (proj && T <= kFewTokenRows) {
         PhaseScope ps(h, PH_WUP, s, 2);
-        FewTokenGemm g{&h->wup128, &h->wup128, &h->yl16, &h->yl32, d, 0, L, yb, d, nullptr, 0, xb, d};
+        FewTokenGemm g{&h->wup128, &h->wup128, &h->yl16, &h->yl32, d, 0, L, yb, d, nullptr, 0, resid, d};
         launch_few_token(g, T, h->at<float>(p.partial), kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns,
                          s);
     } else if (proj) {
@@ -551,7 +650,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.N0 = d;
         a.out0 = yb;
         a.ld0 = d;
-        a.resid = xb;
+        a.resid = resid;
         a.ld_resid = d;
         if (m_tiles * ((d + 255) / 256) >= h->num_sms) {
             a.n_tiles = (d + 255) / 256;
@@ -608,7 +707,9 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     if (w->w_router == nullptr || w->w1 == nullptr || w->w2 == nullptr) return LMOE_ERR_INVALID_ARG;
     if (c.has_proj && (w->w_down == nullptr || w->w_up == nullptr)) return LMOE_ERR_INVALID_ARG;
     if (c.n_const > 0 && w->const_vecs == nullptr) return LMOE_ERR_INVALID_ARG;
-    const void* ptrs[] = {w->w_router, w->router_bias, w->w_down, w->w_up, w->w1, w->w2, w->const_vecs};
+    if (c.shared_m > 0 && (w->w_shared1 == nullptr || w->w_shared2 == nullptr)) return LMOE_ERR_INVALID_ARG;
+    const void* ptrs[] = {w->w_router, w->router_bias, w->w_down, w->w_up, w->w1, w->w2, w->const_vecs,
+                          w->w_shared1, w->w_shared2};
     for (const void* q : ptrs)
         if (!aligned16(q)) return LMOE_ERR_INVALID_ARG;
 
@@ -657,9 +758,24 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     ok &= make_map(&h->rows32, h->at<void>(p.rows), R, L, L, 32);
     ok &= make_map(&h->h16, h->at<void>(p.hbuf), R, m, m, 16);
     ok &= make_map(&h->h32, h->at<void>(p.hbuf), R, m, m, 32);
+    if (c.shared_m > 0) {
+        const int ms = c.shared_m, srows = h->g * ms;
+        ok &= make_map(&h->ws1_64, w->w_shared1, srows, d, d, h->g == 2 ? 32 : 64);
+        ok &= make_map(&h->ws1_256, w->w_shared1, srows, d, d, h->g == 2 ? 128 : 256);
+        ok &= make_map(&h->ws1_128, w->w_shared1, srows, d, d, 128);
+        ok &= make_map(&h->ws2_64, w->w_shared2, d, ms, ms, 64);
+        ok &= make_map(&h->ws2_256, w->w_shared2, d, ms, ms, 256);
+        ok &= make_map(&h->ws2_128, w->w_shared2, d, ms, ms, 128);
+        ok &= make_map(&h->a_hs, h->at<void>(p.hs), c.max_tokens, ms, ms, 128);
+        ok &= make_map(&h->hs16, h->at<void>(p.hs), c.max_tokens, ms, ms, 16);
+        ok &= make_map(&h->hs32, h->at<void>(p.hs), c.max_tokens, ms, ms, 32);
+        ok &= cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking) == cudaSuccess;
+        ok &= cudaEventCreateWithFlags(&h->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+        ok &= cudaEventCreateWithFlags(&h->ev_join, cudaEventDisableTiming) == cudaSuccess;
+    }
     ok &= cudaMemset(h->at<void>(p.hdr), 0, HDR_WORDS * 4) == cudaSuccess;
     if (!ok) {
-        delete h;
+        lmoe_destroy(h);
         return LMOE_ERR_CUDA;
     }
     *out = h;
@@ -708,6 +824,9 @@ int lmoe_last_error(lmoe_handle* h) {
 void lmoe_destroy(lmoe_handle* h) {
     if (h == nullptr) return;
     free_events(h);
+    if (h->ev_fork) cudaEventDestroy(h->ev_fork);
+    if (h->ev_join) cudaEventDestroy(h->ev_join);
+    if (h->side) cudaStreamDestroy(h->side);
     delete h;
 }
 

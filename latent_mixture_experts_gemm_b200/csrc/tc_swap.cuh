@@ -286,11 +286,13 @@ __global__ void __launch_bounds__(192, 1)
 
 // Sum of the K splits in split order, then the epilogue, for the dense
 // few-token projections.  One thread per (output column n, token t), n fastest.
-//   n < n0:             out0[t][n] = bf16(sum (+ resid[t][n] when resid is set)), partial row n
+//   n < n0:             out0[t][n] = bf16(act(sum) (+ resid[t][n] when resid is set)), partial row n
 //   n0 <= n < n0 + n1:  out1[t][n - n0] = sum (fp32 router logits), partial row p1 + (n - n0)
-template <int NT>
+// ACT: EPI_BF16 (none), EPI_RELU2, or EPI_SWIGLU (gate = partial row n, up =
+// partial row up_row0 + n).
+template <int NT, int ACT>
 __global__ void __launch_bounds__(256) swap_reduce_kernel(const float* __restrict__ partial, int part_rows, int splits,
-                                                          int T, int n0, int n1, int p1,
+                                                          int T, int n0, int n1, int p1, int up_row0,
                                                           __nv_bfloat16* __restrict__ out0, int ld0,
                                                           float* __restrict__ out1, int ld1,
                                                           const __nv_bfloat16* __restrict__ resid, int ld_resid) {
@@ -308,6 +310,12 @@ __global__ void __launch_bounds__(256) swap_reduce_kernel(const float* __restric
 #pragma unroll
     for (int s = 0; s < 16; ++s)
         if (s < splits) v += pv[s];
+    if (ACT == EPI_RELU2 && n < n0) v = act_relu2(v);
+    if (ACT == EPI_SWIGLU && n < n0) {
+        float u = 0.f;
+        for (int s = 0; s < splits; ++s) u += partial[(static_cast<size_t>(s) * part_rows + up_row0 + n) * NT + t];
+        v = act_silu_mul(v, u);
+    }
     if (n < n0) {
         if (resid != nullptr) v += __bfloat162float(resid[static_cast<size_t>(t) * ld_resid + n]);
         out0[static_cast<size_t>(t) * ld0 + n] = __float2bfloat16_rn(v);

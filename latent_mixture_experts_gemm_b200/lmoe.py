@@ -25,12 +25,12 @@ I32 = ctypes.c_int32
 
 class lmoe_config(ctypes.Structure):
     _fields_ = [(n, I32) for n in ("d", "latent", "m", "n_experts", "top_k", "max_tokens", "act", "n_zero", "n_copy",
-                                   "n_const", "has_proj", "latent_router")]
+                                   "n_const", "has_proj", "latent_router", "shared_m")]
 
 
 class lmoe_weights(ctypes.Structure):
     _fields_ = [("w_router", P), ("router_bias", P), ("w_down", P), ("w_up", P), ("w1", P), ("w2", P),
-                ("const_vecs", P)]
+                ("const_vecs", P), ("w_shared1", P), ("w_shared2", P)]
 
 
 class lmoe_debug(ctypes.Structure):
@@ -193,7 +193,7 @@ def lmoe_dispatch_noalloc(idx: torch.Tensor, n_total: int, counts: torch.Tensor,
 # ------------------------------------------------------------------ convenience owner of a layer
 def make_config(cfg, max_tokens: int) -> lmoe_config:
     return lmoe_config(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, int(max_tokens), cfg.act, cfg.n_zero,
-                       cfg.n_copy, cfg.n_const, cfg.has_proj, cfg.latent_router)
+                       cfg.n_copy, cfg.n_const, cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0))
 
 
 class LatentMoE:
@@ -208,14 +208,16 @@ class LatentMoE:
         self.device = torch.device(device)
         self.max_tokens = int(max_tokens)
         dev = lambda t: None if t is None else t.to(self.device).contiguous()  # noqa: E731
-        self.w = {k: dev(layer.get(k)) for k in ("w_router", "bias", "w_down", "w_up", "w1", "w2", "const_vecs")}
+        self.w = {k: dev(layer.get(k)) for k in ("w_router", "bias", "w_down", "w_up", "w1", "w2", "const_vecs",
+                                                  "w_shared1", "w_shared2")}
         self.c = make_config(cfg, self.max_tokens)
         nbytes = lmoe_workspace_bytes(self.c)
         if nbytes == 0:
             raise LmoeError("lmoe_workspace_bytes", -2)
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.weights = lmoe_weights(_p(self.w["w_router"]), _p(self.w["bias"]), _p(self.w["w_down"]),
-                                    _p(self.w["w_up"]), _p(self.w["w1"]), _p(self.w["w2"]), _p(self.w["const_vecs"]))
+                                    _p(self.w["w_up"]), _p(self.w["w1"]), _p(self.w["w2"]), _p(self.w["const_vecs"]),
+                                    _p(self.w["w_shared1"]), _p(self.w["w_shared2"]))
         with torch.cuda.device(self.device):
             self.h = lmoe_create(self.c, self.weights, self.workspace.data_ptr(), nbytes)
 

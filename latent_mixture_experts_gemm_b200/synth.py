@@ -7,7 +7,8 @@ from here, so both sides of every parity check see the same bf16 tensors.
 Recipe (one ``torch.Generator('cpu')`` per workload, seeded with its seed):
 
 * draw order: x, router weight, W_down, W_up, W1 (expert by expert), W2
-  (expert by expert), constant-expert vectors, then the Zipf rank permutation;
+  (expert by expert), constant-expert vectors, the Zipf rank permutation, then
+  the shared expert's two matrices (when the layer has one);
 * every weight is ``randn * 1/sqrt(fan_in)`` in fp32, rounded to bf16 (round to
   nearest even); fan_in is the input width of the matrix (d for the router and
   W_down, latent for W_up and W1, m for W2); x and the constant vectors are
@@ -51,6 +52,7 @@ class LayerConfig:
     n_const: int = 0
     has_proj: int = 1
     latent_router: int = 0
+    shared_m: int = 0
     tokens: int = 0
     seed: int = 0
     zipf: float = 0.0
@@ -98,6 +100,11 @@ WORKLOADS: Dict[str, LayerConfig] = {
                        act="relu2", has_proj=0, seed=3),
     "kimi_skew": _cfg(name="kimi_skew", tokens=4096, d=7168, latent=1792, m=1024, n_ffn=896, n_zero=4,
                       n_copy=4, n_const=4, top_k=16, act="swiglu", zipf=1.1, seed=4),
+    # the Nemotron-like layer with a shared expert at the full width (hidden width 2m: the pages give none)
+    "nemotron_decode_shared": _cfg(name="nemotron_decode_shared", tokens=32, d=4096, latent=1024, m=1024,
+                                   n_ffn=512, top_k=22, act="relu2", shared_m=2048, seed=5),
+    "nemotron_prefill_shared": _cfg(name="nemotron_prefill_shared", tokens=8192, d=4096, latent=1024, m=1024,
+                                    n_ffn=512, top_k=22, act="relu2", shared_m=2048, seed=6),
 }
 
 
@@ -112,9 +119,11 @@ def make_layer(cfg: LayerConfig, tokens: Optional[int] = None, seed: Optional[in
     """Draw x and every weight of ``cfg`` on the CPU (bf16, plus an fp32 bias).
 
     Returns a dict with keys ``x, w_router, bias, w_down, w_up, w1, w2,
-    const_vecs``; absent tensors (no projection, no bias, no constant experts)
-    are ``None``.  W1 is ``[N', g*m, latent]`` with the gate rows first when
-    gated; W2 is ``[N', latent, m]``.
+    const_vecs, w_shared1, w_shared2``; absent tensors (no projection, no bias,
+    no constant experts, no shared expert) are ``None``.  W1 is
+    ``[N', g*m, latent]`` with the gate rows first when gated; W2 is
+    ``[N', latent, m]``.  The shared expert's W1 is ``[g*shared_m, d]`` (gate
+    rows first when gated), its W2 ``[d, shared_m]``.
     """
     T = cfg.tokens if tokens is None else tokens
     s = cfg.seed if seed is None else seed
@@ -143,6 +152,12 @@ def make_layer(cfg: LayerConfig, tokens: Optional[int] = None, seed: Optional[in
         out["bias"] = (-cfg.zipf * torch.log(ranks)).to(torch.float32)
     else:
         out["bias"] = None
+    if cfg.shared_m:
+        rows = 2 * cfg.shared_m if cfg.gated else cfg.shared_m
+        out["w_shared1"] = _draw(g, (rows, d), 1.0 / math.sqrt(d))
+        out["w_shared2"] = _draw(g, (d, cfg.shared_m), 1.0 / math.sqrt(cfg.shared_m))
+    else:
+        out["w_shared1"] = out["w_shared2"] = None
     return out
 
 

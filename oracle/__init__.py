@@ -25,7 +25,8 @@ _lib = None
 
 class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
-        "d", "latent", "m", "n_ffn", "top_k", "act", "n_zero", "n_copy", "n_const", "has_proj", "latent_router")]
+        "d", "latent", "m", "n_ffn", "top_k", "act", "n_zero", "n_copy", "n_const", "has_proj", "latent_router",
+        "shared_m")]
 
 
 def lib():
@@ -34,7 +35,7 @@ def lib():
         path = _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
-        L.oracle_forward.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int] + [P] * 15
+        L.oracle_forward.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int] + [P] * 17
         L.oracle_forward.restype = ctypes.c_int
         L.oracle_route.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P]
         L.oracle_route.restype = ctypes.c_int
@@ -56,7 +57,7 @@ def set_num_threads(n: int) -> None:
 
 def _cfg(cfg) -> _Cfg:
     return _Cfg(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, cfg.act, cfg.n_zero, cfg.n_copy, cfg.n_const,
-                cfg.has_proj, cfg.latent_router)
+                cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0))
 
 
 def _bits(t: Optional[torch.Tensor]):
@@ -90,9 +91,11 @@ def forward(cfg, layer: Dict[str, torch.Tensor], x: Optional[torch.Tensor] = Non
     w1 = _bits(layer["w1"])
     w2 = _bits(layer["w2"])
     cv = _bits(layer.get("const_vecs"))
+    ws1 = _bits(layer.get("w_shared1"))
+    ws2 = _bits(layer.get("w_shared2"))
     bias = layer.get("bias")
     bias_np = None if bias is None else bias.detach().cpu().to(torch.float32).contiguous().numpy()
-    keep += [xb, wr, wd, wu, w1, w2, cv, bias_np]
+    keep += [xb, wr, wd, wu, w1, w2, cv, ws1, ws2, bias_np]
     idx_in = None if idx is None else np.ascontiguousarray(idx, dtype=np.int32)
     out = {"y": np.empty((T, cfg.d), np.float64), "idx": np.empty((T, K), np.int32), "w": np.empty((T, K), np.float64)}
     if "z" in want:
@@ -103,7 +106,8 @@ def forward(cfg, layer: Dict[str, torch.Tensor], x: Optional[torch.Tensor] = Non
         out["logits"] = np.empty((T, Nt), np.float64)
     c = _cfg(cfg)
     rc = lib().oracle_forward(ctypes.byref(c), T, _ptr(xb), _ptr(wr), _ptr(bias_np), _ptr(wd), _ptr(wu), _ptr(w1),
-                              _ptr(w2), _ptr(cv), _ptr(idx_in), _ptr(out["y"]), _ptr(out["idx"]), _ptr(out["w"]),
+                              _ptr(w2), _ptr(cv), _ptr(ws1), _ptr(ws2), _ptr(idx_in), _ptr(out["y"]), _ptr(out["idx"]),
+                              _ptr(out["w"]),
                               _ptr(out.get("z")), _ptr(out.get("yl")), _ptr(out.get("logits")))
     if rc != 0:
         raise ValueError("oracle_forward rejected its arguments")

@@ -35,6 +35,10 @@
  *   7. y = x + W_up yl      (project back to d, "How LatentMoE Works"
  *      step 3; the residual add is the plain reading of a layer output),
  *      or y = x + yl without a projection.
+ *   8. with a shared expert (hidden width ms > 0), which stays at the full
+ *      width d ("LatentMoE: How MoE Made a Key Paradigm Leap in 2026",
+ *      section 2 closing note): y += Ws2 act(Ws1 x), act as for the routed
+ *      experts, added to the routed output, outside the routing.
  *
  * Everything is computed in double precision on the bf16 inputs widened
  * exactly; nothing is rounded in between.  OpenMP runs tokens in parallel;
@@ -63,6 +67,7 @@ typedef struct {
     int32_t n_zero, n_copy, n_const;
     int32_t has_proj;      /* 1: W_down / W_up present */
     int32_t latent_router; /* 1: gate reads z instead of x */
+    int32_t shared_m;      /* hidden width of the shared expert at d (0: none) */
 } oracle_cfg;
 
 enum { ORACLE_ACT_RELU2 = 0, ORACLE_ACT_SWIGLU = 1, ORACLE_ACT_IDENTITY = 2 };
@@ -189,7 +194,8 @@ static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t 
  *   x [T,d] bf16; w_router [n_tot, fdim] bf16 (fdim = d, or latent with the
  *   latent router); bias [n_tot] fp32 or NULL; w_down [latent,d]; w_up
  *   [d,latent]; w1 [n_ffn, g*m, latent]; w2 [n_ffn, latent, m]; const_vecs
- *   [n_const, latent]   (all bf16 bit patterns).
+ *   [n_const, latent]; w_shared1 [g*shared_m, d], w_shared2 [d, shared_m]
+ *   (NULL without a shared expert)   (all bf16 bit patterns).
  *   idx_in: if non-NULL, [T,K'] routes to use instead of the router's own
  *   choice (the weights are still the renormalised softmax of the router's
  *   logits at those ids, in the given slot order).
@@ -200,12 +206,16 @@ static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t 
  */
 int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t *w_router, const float *bias,
                    const uint16_t *w_down, const uint16_t *w_up, const uint16_t *w1, const uint16_t *w2,
-                   const uint16_t *const_vecs, const int32_t *idx_in, double *y, int32_t *idx_out, double *w_out,
-                   double *z_out, double *yl_out, double *logits_out)
+                   const uint16_t *const_vecs, const uint16_t *w_shared1, const uint16_t *w_shared2,
+                   const int32_t *idx_in, double *y, int32_t *idx_out, double *w_out, double *z_out, double *yl_out,
+                   double *logits_out)
 {
     const int d = c->d, L = c->latent, m = c->m, K = c->top_k, Nt = n_total(c);
     if (T < 0 || K < 1 || K > Nt || d < 1 || L < 1 || m < 1) return -1;
     if (!c->has_proj && L != d) return -1;
+    if (c->shared_m < 0 || (c->shared_m > 0 && (!w_shared1 || !w_shared2))) return -1;
+    const int ms = c->shared_m;
+    const int s_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * ms : ms;
     const int fdim = c->latent_router ? L : d;
     const int up_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * m : m;
     int bad = 0;
@@ -223,7 +233,10 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
         double *up = (double *)malloc(sizeof(double) * (size_t)d);
         double *w = (double *)malloc(sizeof(double) * (size_t)K);
         int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)K);
-        if (!xt || !z || !zr || !lg || !u || !h || !o || !yl || !up || !w || !sel) bad = 1;
+        double *su = (double *)malloc(sizeof(double) * (size_t)(s_rows > 0 ? s_rows : 1));
+        double *sh = (double *)malloc(sizeof(double) * (size_t)(ms > 0 ? ms : 1));
+        double *so = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!xt || !z || !zr || !lg || !u || !h || !o || !yl || !up || !w || !sel || !su || !sh || !so) bad = 1;
 
 #pragma omp for schedule(dynamic, 1)
         for (int t = 0; t < T; ++t) {
@@ -276,6 +289,23 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             if (c->has_proj) matvec(d, L, w_up, yl, up);
             else memcpy(up, yl, sizeof(double) * (size_t)d);
             for (int i = 0; i < d; ++i) y[(size_t)t * d + i] = xt[i] + up[i];
+            /* step 8: the shared expert at the full width, on x */
+            if (ms > 0) {
+                matvec(s_rows, d, w_shared1, xt, su);
+                for (int j = 0; j < ms; ++j) {
+                    if (c->act == ORACLE_ACT_RELU2) {
+                        double r = su[j] > 0.0 ? su[j] : 0.0;
+                        sh[j] = r * r;
+                    } else if (c->act == ORACLE_ACT_SWIGLU) {
+                        double a = su[j];
+                        sh[j] = a / (1.0 + exp(-a)) * su[ms + j];
+                    } else {
+                        sh[j] = su[j];
+                    }
+                }
+                matvec(d, ms, w_shared2, sh, so);
+                for (int i = 0; i < d; ++i) y[(size_t)t * d + i] += so[i];
+            }
 
             if (idx_out)
                 for (int k = 0; k < K; ++k) idx_out[(size_t)t * K + k] = sel[k];
@@ -285,6 +315,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             if (yl_out) memcpy(yl_out + (size_t)t * L, yl, sizeof(double) * (size_t)L);
             if (logits_out) memcpy(logits_out + (size_t)t * Nt, lg, sizeof(double) * (size_t)Nt);
         }
+        free(su); free(sh); free(so);
         free(xt); free(z); free(zr); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
     }
     return bad ? -1 : 0;

@@ -53,7 +53,8 @@ def _bf(a: np.ndarray) -> np.ndarray:
 
 
 def emulate_bf16(cfg, layer, x: torch.Tensor, idx: np.ndarray, w: np.ndarray) -> np.ndarray:
-    """y with the GPU path's bf16 storage points (z, H, O, yl, y) on the given routes."""
+    """y with the GPU path's bf16 storage points (z, H, O, yl, the shared expert's hidden rows and
+    x + its output, y) on the given routes."""
     f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
     X = f(x)
     W1, W2 = layer["w1"], layer["w2"]
@@ -81,9 +82,20 @@ def emulate_bf16(cfg, layer, x: torch.Tensor, idx: np.ndarray, w: np.ndarray) ->
                 o = f(layer["const_vecs"])[e - cfg.n_ffn - cfg.n_zero - cfg.n_copy]
             acc += float(np.float32(w[t, k])) * o
         yl[t] = acc
+    base = X
+    if getattr(cfg, "shared_m", 0):
+        us = X @ f(layer["w_shared1"]).T
+        ms = cfg.shared_m
+        if cfg.act == 0:
+            hs = np.maximum(us, 0) ** 2
+        elif cfg.act == 1:
+            hs = us[:, :ms] / (1 + np.exp(-us[:, :ms])) * us[:, ms:]
+        else:
+            hs = us
+        base = _bf(X + _bf(hs) @ f(layer["w_shared2"]).T)   # x + shared expert, stored in bf16
     if cfg.has_proj:
-        return _bf(X + _bf(yl) @ f(layer["w_up"]).T)
-    return _bf(X + yl)
+        return _bf(base + _bf(yl) @ f(layer["w_up"]).T)
+    return _bf(base + yl)
 
 
 def assert_layer_close(got, ref, emulated, what="y") -> dict:

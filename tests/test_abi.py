@@ -46,7 +46,7 @@ def test_workspace_bytes_and_shape_checks():
     small = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
     assert 0 < lmoe.lmoe_workspace_bytes(small) < n
     bad = [dict(d=100), dict(latent=0), dict(m=32), dict(top_k=0), dict(top_k=33), dict(n_experts=0),
-           dict(max_tokens=0), dict(act=7), dict(has_proj=0)]
+           dict(max_tokens=0), dict(act=7), dict(has_proj=0), dict(shared_m=100), dict(shared_m=-64)]
     for b in bad:
         c = lmoe.make_config(synth.WORKLOADS["tiny"], 64)
         for k, v in b.items():
@@ -82,7 +82,7 @@ def test_null_handle_calls_are_rejected():
     assert L.lmoe_last_error(None) == -1
     assert L.lmoe_set_profiling(None, 1, 1) == -1
     L.lmoe_destroy(None)
-    assert lmoe.lmoe_num_phases() == 9
+    assert lmoe.lmoe_num_phases() == 10
     assert [lmoe.lmoe_phase_name(i) for i in range(3)] == ["router_proj_gemm", "topk_softmax", "dispatch"]
 
 

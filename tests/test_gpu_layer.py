@@ -32,6 +32,11 @@ CASES = {
     "medium_16_tokens": MEDIUM.with_(tokens=16, seed=28),
     "medium_1024_experts_top32": MEDIUM.with_(n_ffn=1020, n_zero=2, n_copy=1, n_const=1, top_k=32, seed=30),
     "medium_17_tokens_swiglu": MEDIUM.with_(tokens=17, act="swiglu", n_copy=1, seed=29),
+    "medium_shared_expert": MEDIUM.with_(shared_m=256, seed=34),
+    "medium_17_tokens_swiglu_shared": MEDIUM.with_(tokens=17, act="swiglu", shared_m=128, n_zero=1, seed=35),
+    "medium_standard_moe_shared": MEDIUM.with_(latent=512, has_proj=0, shared_m=192, seed=36),
+    "tiny_decode_shared_swiglu": synth.WORKLOADS["tiny"].with_(tokens=9, act="swiglu", shared_m=64, seed=37),
+    "tiny_decode_latent_router": synth.WORKLOADS["tiny"].with_(tokens=12, latent_router=1, seed=38),
     "nemotron_decode": synth.WORKLOADS["nemotron_decode"],
     "std_decode": synth.WORKLOADS["std_decode"],
 }

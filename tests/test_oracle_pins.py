@@ -176,6 +176,16 @@ def _dense_bruteforce(cfg, layer):
         w = P[t] * mask / (P[t] * mask).sum()
         yl[t] = (w[:, None] * O[t]).sum(0)
     up = yl @ Wu.T if cfg.has_proj else yl
+    if getattr(cfg, "shared_m", 0):
+        Us = x @ _np(layer["w_shared1"]).T
+        ms = cfg.shared_m
+        if cfg.act == synth.ACT_RELU2:
+            Hs = np.maximum(Us, 0) ** 2
+        elif cfg.act == synth.ACT_SWIGLU:
+            Hs = scipy.special.expit(Us[:, :ms]) * Us[:, :ms] * Us[:, ms:]
+        else:
+            Hs = Us
+        up = up + Hs @ _np(layer["w_shared2"]).T
     return x + up
 
 
@@ -201,6 +211,29 @@ def test_several_bypass_experts_of_each_kind_match_dense_bruteforce():
     out = oracle.forward(cfg, layer)
     assert np.any(out["idx"] >= cfg.n_ffn + cfg.n_zero + cfg.n_copy + 1)   # a second constant expert is used
     np.testing.assert_allclose(out["y"], _dense_bruteforce(cfg, layer), rtol=1e-11, atol=1e-11)
+
+
+@pytest.mark.parametrize("act", ["relu2", "swiglu"])
+def test_shared_expert_matches_dense_bruteforce(act):
+    cfg = SMALL.with_(act=act, shared_m=12, zipf=0.7)
+    layer = synth.make_layer(cfg)
+    assert layer["w_shared1"].shape == ((24 if act == "swiglu" else 12), cfg.d)
+    out = oracle.forward(cfg, layer)
+    np.testing.assert_allclose(out["y"], _dense_bruteforce(cfg, layer), rtol=1e-11, atol=1e-11)
+
+
+def test_shared_expert_alone_is_a_plain_ffn_on_x():
+    """Routing forced to the zero expert leaves y = x + Ws2 relu(Ws1 x)^2, and scaling Ws2 scales y - x."""
+    cfg = SMALL.with_(top_k=1, shared_m=10)
+    layer = synth.make_layer(cfg)
+    bias = torch.full((cfg.n_total,), -100.0)
+    bias[cfg.n_ffn] = 100.0                       # the zero expert
+    x = _np(layer["x"])
+    ffn = np.maximum(x @ _np(layer["w_shared1"]).T, 0) ** 2 @ _np(layer["w_shared2"]).T
+    a = oracle.forward(cfg, dict(layer, bias=bias))
+    np.testing.assert_allclose(a["y"], x + ffn, rtol=1e-12, atol=1e-12)
+    b = oracle.forward(cfg, dict(layer, bias=bias, w_shared2=layer["w_shared2"] * 2))
+    np.testing.assert_allclose(b["y"] - x, 2 * (a["y"] - x), rtol=1e-12, atol=1e-13)
 
 
 def test_latent_router_matches_dense_bruteforce():
