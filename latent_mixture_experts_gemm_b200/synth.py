@@ -53,6 +53,7 @@ class LayerConfig:
     has_proj: int = 1
     latent_router: int = 0
     shared_m: int = 0
+    expert_fmt: int = 0
     tokens: int = 0
     seed: int = 0
     zipf: float = 0.0
@@ -105,6 +106,11 @@ WORKLOADS: Dict[str, LayerConfig] = {
                                    n_ffn=512, top_k=22, act="relu2", shared_m=2048, seed=5),
     "nemotron_prefill_shared": _cfg(name="nemotron_prefill_shared", tokens=8192, d=4096, latent=1024, m=1024,
                                     n_ffn=512, top_k=22, act="relu2", shared_m=2048, seed=6),
+    # the Nemotron-like decode batch with block-scaled expert weights (MXFP8: E4M3 elements; MXFP4: E2M1)
+    "nemotron_decode_mxfp8": _cfg(name="nemotron_decode_mxfp8", tokens=32, d=4096, latent=1024, m=1024, n_ffn=512,
+                                  top_k=22, act="relu2", expert_fmt=1, seed=7),
+    "nemotron_decode_mxfp4": _cfg(name="nemotron_decode_mxfp4", tokens=32, d=4096, latent=1024, m=1024, n_ffn=512,
+                                  top_k=22, act="relu2", expert_fmt=2, seed=8),
 }
 
 

@@ -26,7 +26,7 @@ _lib = None
 class _Cfg(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "d", "latent", "m", "n_ffn", "top_k", "act", "n_zero", "n_copy", "n_const", "has_proj", "latent_router",
-        "shared_m")]
+        "shared_m", "expert_fmt")]
 
 
 def lib():
@@ -41,6 +41,10 @@ def lib():
         L.oracle_route.restype = ctypes.c_int
         L.oracle_dispatch.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P, P, P, P]
         L.oracle_dispatch.restype = ctypes.c_int
+        L.oracle_mx_quantize.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P, P]
+        L.oracle_mx_quantize.restype = ctypes.c_int
+        L.oracle_mx_dequantize.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
+        L.oracle_mx_dequantize.restype = ctypes.c_int
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = L
@@ -57,7 +61,7 @@ def set_num_threads(n: int) -> None:
 
 def _cfg(cfg) -> _Cfg:
     return _Cfg(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, cfg.act, cfg.n_zero, cfg.n_copy, cfg.n_const,
-                cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0))
+                cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0), getattr(cfg, "expert_fmt", 0))
 
 
 def _bits(t: Optional[torch.Tensor]):
@@ -139,3 +143,35 @@ def dispatch(idx: np.ndarray, n_total: int):
     if rc != 0:
         raise ValueError("oracle_dispatch: expert id out of range")
     return counts, offsets, perm, inv
+
+
+#: MX block formats of the expert weights (``expert_fmt``)
+FMT_BF16, FMT_MXFP8, FMT_MXFP4 = 0, 1, 2
+
+
+def mx_quantize(w: torch.Tensor, fmt: int):
+    """MX encoding of a bf16 matrix [rows, K] (K a multiple of 32).
+
+    Returns ``(codes, scales)``: uint8 [rows, K] element codes, one per byte
+    (E4M3 for MXFP8; E2M1 in the low nibble for MXFP4), and uint8
+    [rows, K/32] E8M0 scale bytes (value 2^(byte - 127)).
+    """
+    w2 = w.reshape(-1, w.shape[-1])
+    rows, K = int(w2.shape[0]), int(w2.shape[1])
+    wb = _bits(w2)
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, max(K // 32, 1)), np.uint8)
+    if lib().oracle_mx_quantize(wb.ctypes.data, rows, K, int(fmt), codes.ctypes.data, scales.ctypes.data) != 0:
+        raise ValueError("oracle_mx_quantize rejected its arguments")
+    return codes, scales
+
+
+def mx_dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray:
+    """The fp64 values an MX encoding from :func:`mx_quantize` stands for."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = c.shape
+    out = np.empty((rows, K), np.float64)
+    if lib().oracle_mx_dequantize(c.ctypes.data, s.ctypes.data, rows, K, int(fmt), out.ctypes.data) != 0:
+        raise ValueError("oracle_mx_dequantize rejected its arguments")
+    return out

@@ -39,9 +39,16 @@
  *      width d ("LatentMoE: How MoE Made a Key Paradigm Leap in 2026",
  *      section 2 closing note): y += Ws2 act(Ws1 x), act as for the routed
  *      experts, added to the routed output, outside the routing.
+ *   9. with block-scaled expert weights (expert_fmt = MXFP8 or MXFP4), W1_e
+ *      and W2_e are first encoded in that MX format (see the MX section
+ *      below) and used at their encoded values; the inputs of both expert
+ *      matrices (z, and the activation h) are stored in bf16 and then
+ *      encoded in MXFP8 before the multiply.  The router, the projections
+ *      and the shared expert stay in bf16.
  *
  * Everything is computed in double precision on the bf16 inputs widened
- * exactly; nothing is rounded in between.  OpenMP runs tokens in parallel;
+ * exactly; nothing is rounded in between except the MX encodings of step 9
+ * (and the bf16 storage they start from).  OpenMP runs tokens in parallel;
  * each token's arithmetic is a straight sequential loop.
  *
  * The counting sort (dispatch) that groups (token, slot) pairs by expert is
@@ -68,9 +75,11 @@ typedef struct {
     int32_t has_proj;      /* 1: W_down / W_up present */
     int32_t latent_router; /* 1: gate reads z instead of x */
     int32_t shared_m;      /* hidden width of the shared expert at d (0: none) */
+    int32_t expert_fmt;    /* 0 bf16 expert weights, 1 MXFP8, 2 MXFP4 */
 } oracle_cfg;
 
 enum { ORACLE_ACT_RELU2 = 0, ORACLE_ACT_SWIGLU = 1, ORACLE_ACT_IDENTITY = 2 };
+enum { ORACLE_FMT_BF16 = 0, ORACLE_FMT_MXFP8 = 1, ORACLE_FMT_MXFP4 = 2 };
 
 static double widen(uint16_t h)
 {
@@ -83,8 +92,10 @@ static double widen(uint16_t h)
 static int n_total(const oracle_cfg *c) { return c->n_ffn + c->n_zero + c->n_copy + c->n_const; }
 
 /* Round to the nearest bfloat16 (ties to even) through binary32, the way a
- * value accumulated in fp32 is stored as bf16.  Used for one input only: the
- * latent the latent-router reading feeds to the gate (see step 1). */
+ * value accumulated in fp32 is stored as bf16.  Used only where the layer
+ * stores a value before an integer decision is taken on it: the latent the
+ * latent-router reading feeds to the gate (step 1), and the expert inputs
+ * that are MX-encoded (step 9). */
 static double round_bf16(double v)
 {
     float f = (float)v;
@@ -94,6 +105,159 @@ static double round_bf16(double v)
     u &= 0xFFFF0000u;
     memcpy(&f, &u, sizeof f);
     return (double)f;
+}
+
+/* ------------------------------------------------------------------ MX block formats
+ *
+ * The pages name the formats only: Kimi K3 serves MXFP4 weights after
+ * quantisation-aware training (the comparison table of "Two Teams, Two
+ * Practices"), and Nemotron 3 Super trains in NVFP4 (the training note of
+ * the outlook section).  Their definition is the Open Compute Project's
+ * Microscaling (MX) specification, v1.0:
+ *   - a block is 32 consecutive values along the reduction (K) axis;
+ *   - the block shares one scale X = 2^s, stored as an E8M0 byte s + 127,
+ *     with s = floor(log2(max_i |V_i|)) - emax, emax being the exponent of
+ *     the element format's largest normal (8 for E4M3, 2 for E2M1); s is
+ *     clamped to [-127, 127];
+ *   - each element is V_i / X rounded to the nearest value of the element
+ *     format (ties to the even mantissa) and saturated to its largest
+ *     magnitude (448 for E4M3, 6 for E2M1);
+ *   - an all-zero block gets s = -127 and zero elements.
+ * E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; normals
+ * (1 + m/8) 2^(e-7), subnormals m/8 2^-6; the code 0x7F / 0xFF is NaN and is
+ * never produced.  E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit;
+ * the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+ * Codes are kept one per byte here (E2M1 in the low nibble, sign in bit 3).
+ */
+static int fmt_mbits(int e2m1) { return e2m1 ? 1 : 3; }
+static int fmt_emin(int e2m1) { return e2m1 ? 0 : -6; }   /* exponent of the smallest normal */
+static int fmt_emax(int e2m1) { return e2m1 ? 2 : 8; }    /* exponent of the largest normal */
+static double fmt_max(int e2m1) { return e2m1 ? 6.0 : 448.0; }
+
+/* Nearest element-format magnitude to a >= 0 (ties to even), saturated. */
+static double round_elem(double a, int e2m1)
+{
+    const double maxv = fmt_max(e2m1);
+    if (a >= maxv) return maxv;
+    if (a == 0.0) return 0.0;
+    int e;
+    frexp(a, &e);
+    e -= 1; /* a = f 2^e with f in [1, 2) */
+    if (e < fmt_emin(e2m1)) e = fmt_emin(e2m1);
+    const double quantum = ldexp(1.0, e - fmt_mbits(e2m1));
+    const double r = rint(a / quantum) * quantum; /* the default rounding mode: to nearest, ties to even */
+    return r > maxv ? maxv : r;
+}
+
+/* Code of an element-format magnitude r (exactly representable) and a sign. */
+static uint8_t elem_code(double r, int neg, int e2m1)
+{
+    const int mb = fmt_mbits(e2m1), emin = fmt_emin(e2m1), bias = e2m1 ? 1 : 7;
+    unsigned code;
+    if (r < ldexp(1.0, emin)) {
+        code = (unsigned)(r / ldexp(1.0, emin - mb)); /* subnormal: m quanta of 2^(emin - mbits) */
+    } else {
+        int e;
+        frexp(r, &e);
+        e -= 1;
+        const unsigned mant = (unsigned)(r / ldexp(1.0, e - mb)) - (1u << mb);
+        code = ((unsigned)(e + bias) << mb) | mant;
+    }
+    if (neg) code |= e2m1 ? 0x8u : 0x80u;
+    return (uint8_t)code;
+}
+
+/* Value of an element code. */
+static double elem_value(uint8_t code, int e2m1)
+{
+    const int mb = fmt_mbits(e2m1), bias = e2m1 ? 1 : 7;
+    const unsigned sign = e2m1 ? (code >> 3) & 1u : (code >> 7) & 1u;
+    const unsigned ebits = e2m1 ? (code >> 1) & 3u : (code >> 3) & 15u;
+    const unsigned mant = code & ((1u << mb) - 1u);
+    double v;
+    if (ebits == 0) v = ldexp((double)mant, 1 - bias - mb);
+    else v = ldexp((double)((1u << mb) + mant), (int)ebits - bias - mb);
+    return sign ? -v : v;
+}
+
+/* Encode one block of 32 values. */
+static void mx_block(const double *v, int e2m1, uint8_t *codes, uint8_t *scale)
+{
+    double amax = 0.0;
+    for (int i = 0; i < 32; ++i) amax = fabs(v[i]) > amax ? fabs(v[i]) : amax;
+    int s = -127;
+    if (amax > 0.0) {
+        int e;
+        frexp(amax, &e);
+        s = (e - 1) - fmt_emax(e2m1);
+        if (s < -127) s = -127;
+        if (s > 127) s = 127;
+    }
+    *scale = (uint8_t)(s + 127);
+    for (int i = 0; i < 32; ++i) {
+        const double q = ldexp(v[i], -s); /* exact: a power-of-two scaling */
+        codes[i] = elem_code(round_elem(fabs(q), e2m1), signbit(q) != 0, e2m1);
+    }
+}
+
+/* MX encoding of a bf16 matrix [rows, K] (K a multiple of 32): codes
+ * [rows, K] one per byte, scales [rows, K/32] as E8M0 bytes.  fmt is
+ * ORACLE_FMT_MXFP8 (E4M3 elements) or ORACLE_FMT_MXFP4 (E2M1 elements).
+ * Returns 0, or -1 on bad arguments. */
+int oracle_mx_quantize(const uint16_t *w, int rows, int K, int fmt, uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || K < 32 || K % 32 != 0 || (fmt != ORACLE_FMT_MXFP8 && fmt != ORACLE_FMT_MXFP4)) return -1;
+    const int e2m1 = fmt == ORACLE_FMT_MXFP4;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        double v[32];
+        for (int b = 0; b < K / 32; ++b) {
+            for (int i = 0; i < 32; ++i) v[i] = widen(w[(size_t)r * K + b * 32 + i]);
+            mx_block(v, e2m1, codes + (size_t)r * K + b * 32, scales + (size_t)r * (K / 32) + b);
+        }
+    }
+    return 0;
+}
+
+/* The values an MX encoding stands for: out = elem(code) * 2^(scale - 127). */
+int oracle_mx_dequantize(const uint8_t *codes, const uint8_t *scales, int rows, int K, int fmt, double *out)
+{
+    if (rows < 0 || K < 32 || K % 32 != 0 || (fmt != ORACLE_FMT_MXFP8 && fmt != ORACLE_FMT_MXFP4)) return -1;
+    const int e2m1 = fmt == ORACLE_FMT_MXFP4;
+    for (size_t i = 0; i < (size_t)rows * K; ++i)
+        out[i] = ldexp(elem_value(codes[i], e2m1), (int)scales[i / 32] - 127);
+    return 0;
+}
+
+/* An activation vector as the expert GEMMs read it: stored in bf16, then MXFP8-encoded. */
+static void mx_activation(const double *v, int n, double *out)
+{
+    uint8_t codes[32], scale;
+    double blk[32];
+    for (int b = 0; b < n / 32; ++b) {
+        for (int i = 0; i < 32; ++i) blk[i] = round_bf16(v[b * 32 + i]);
+        mx_block(blk, 0, codes, &scale);
+        for (int i = 0; i < 32; ++i) out[b * 32 + i] = ldexp(elem_value(codes[i], 0), (int)scale - 127);
+    }
+}
+
+/* An MX-encoded weight matrix: codes [rows, in_dim], scales [rows, in_dim/32]. */
+typedef struct {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    int e2m1;
+} mx_matrix;
+
+/* out[o] = sum_i value(W[o, i]) * v[i] for an MX-encoded W */
+static void matvec_mx(int out_dim, int in_dim, mx_matrix W, const double *v, double *out)
+{
+    for (int o = 0; o < out_dim; ++o) {
+        const uint8_t *row = W.codes + (size_t)o * in_dim;
+        const uint8_t *sc = W.scales + (size_t)o * (in_dim / 32);
+        double s = 0.0;
+        for (int i = 0; i < in_dim; ++i) s += ldexp(elem_value(row[i], W.e2m1), (int)sc[i / 32] - 127) * v[i];
+        out[o] = s;
+    }
 }
 
 /* out[o] = sum_i W[o*in_dim + i] * v[i] */
@@ -168,13 +332,22 @@ int oracle_dispatch(int T, int top_k, int n_tot, const int32_t *idx, int32_t *co
     return 0;
 }
 
-/* One FFN expert in the latent space: o = W2_e act(W1_e z). */
-static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t *w2e, const double *z,
-                       double *u, double *h, double *o)
+/* One FFN expert in the latent space: o = W2_e act(W1_e z).  With MX expert
+ * weights (mx1/mx2 non-NULL) the encoded matrices are used and the inputs z
+ * and h pass through bf16 storage and the MXFP8 encoding first (step 9);
+ * zq and hq are scratch of L and m values. */
+static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t *w2e, const mx_matrix *mx1,
+                       const mx_matrix *mx2, const double *z, double *zq, double *u, double *h, double *hq,
+                       double *o)
 {
     const int L = c->latent, m = c->m;
     const int up_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * m : m;
-    matvec(up_rows, L, w1e, z, u);
+    if (mx1) {
+        mx_activation(z, L, zq);
+        matvec_mx(up_rows, L, *mx1, zq, u);
+    } else {
+        matvec(up_rows, L, w1e, z, u);
+    }
     for (int j = 0; j < m; ++j) {
         if (c->act == ORACLE_ACT_RELU2) {
             double r = u[j] > 0.0 ? u[j] : 0.0;
@@ -186,7 +359,12 @@ static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t 
             h[j] = u[j];
         }
     }
-    matvec(L, m, w2e, h, o);
+    if (mx2) {
+        mx_activation(h, m, hq);
+        matvec_mx(L, m, *mx2, hq, o);
+    } else {
+        matvec(L, m, w2e, h, o);
+    }
 }
 
 /*
@@ -218,7 +396,25 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
     const int s_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * ms : ms;
     const int fdim = c->latent_router ? L : d;
     const int up_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * m : m;
+    const int fmt = c->expert_fmt;
+    if (fmt != ORACLE_FMT_BF16 && fmt != ORACLE_FMT_MXFP8 && fmt != ORACLE_FMT_MXFP4) return -1;
+    if (fmt != ORACLE_FMT_BF16 && (L % 32 != 0 || m % 32 != 0)) return -1;
     int bad = 0;
+
+    /* step 9: encode the FFN experts' weights once (they are the layer's stored weights) */
+    uint8_t *c1 = NULL, *s1 = NULL, *c2 = NULL, *s2 = NULL;
+    if (fmt != ORACLE_FMT_BF16) {
+        const size_t n1 = (size_t)c->n_ffn * up_rows * L, n2 = (size_t)c->n_ffn * L * m;
+        c1 = (uint8_t *)malloc(n1 > 0 ? n1 : 1);
+        s1 = (uint8_t *)malloc(n1 / 32 > 0 ? n1 / 32 : 1);
+        c2 = (uint8_t *)malloc(n2 > 0 ? n2 : 1);
+        s2 = (uint8_t *)malloc(n2 / 32 > 0 ? n2 / 32 : 1);
+        if (!c1 || !s1 || !c2 || !s2 || oracle_mx_quantize(w1, c->n_ffn * up_rows, L, fmt, c1, s1) != 0 ||
+            oracle_mx_quantize(w2, c->n_ffn * L, m, fmt, c2, s2) != 0) {
+            free(c1); free(s1); free(c2); free(s2);
+            return -1;
+        }
+    }
 
 #pragma omp parallel reduction(| : bad)
     {
@@ -236,7 +432,10 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
         double *su = (double *)malloc(sizeof(double) * (size_t)(s_rows > 0 ? s_rows : 1));
         double *sh = (double *)malloc(sizeof(double) * (size_t)(ms > 0 ? ms : 1));
         double *so = (double *)malloc(sizeof(double) * (size_t)d);
-        if (!xt || !z || !zr || !lg || !u || !h || !o || !yl || !up || !w || !sel || !su || !sh || !so) bad = 1;
+        double *zq = (double *)malloc(sizeof(double) * (size_t)L);
+        double *hq = (double *)malloc(sizeof(double) * (size_t)m);
+        if (!xt || !z || !zr || !lg || !u || !h || !o || !yl || !up || !w || !sel || !su || !sh || !so || !zq || !hq)
+            bad = 1;
 
 #pragma omp for schedule(dynamic, 1)
         for (int t = 0; t < T; ++t) {
@@ -274,7 +473,17 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             for (int k = 0; k < K; ++k) {
                 const int e = sel[k];
                 if (e < c->n_ffn) {
-                    ffn_expert(c, w1 + (size_t)e * up_rows * L, w2 + (size_t)e * L * m, z, u, h, o);
+                    mx_matrix m1 = {0}, m2 = {0};
+                    if (fmt != ORACLE_FMT_BF16) {
+                        m1.codes = c1 + (size_t)e * up_rows * L;
+                        m1.scales = s1 + (size_t)e * up_rows * (L / 32);
+                        m2.codes = c2 + (size_t)e * L * m;
+                        m2.scales = s2 + (size_t)e * L * (m / 32);
+                        m1.e2m1 = m2.e2m1 = fmt == ORACLE_FMT_MXFP4;
+                    }
+                    ffn_expert(c, w1 + (size_t)e * up_rows * L, w2 + (size_t)e * L * m,
+                               fmt != ORACLE_FMT_BF16 ? &m1 : NULL, fmt != ORACLE_FMT_BF16 ? &m2 : NULL, z, zq, u, h,
+                               hq, o);
                 } else if (e < c->n_ffn + c->n_zero) {
                     for (int j = 0; j < L; ++j) o[j] = 0.0;
                 } else if (e < c->n_ffn + c->n_zero + c->n_copy) {
@@ -315,9 +524,10 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             if (yl_out) memcpy(yl_out + (size_t)t * L, yl, sizeof(double) * (size_t)L);
             if (logits_out) memcpy(logits_out + (size_t)t * Nt, lg, sizeof(double) * (size_t)Nt);
         }
-        free(su); free(sh); free(so);
+        free(su); free(sh); free(so); free(zq); free(hq);
         free(xt); free(z); free(zr); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
     }
+    free(c1); free(s1); free(c2); free(s2);
     return bad ? -1 : 0;
 }
 
