@@ -133,28 +133,43 @@ def dist_max(v: float, world: int, device: torch.device) -> float:
 
 
 # ----------------------------------------------------------------------------- algorithmic work
+#: bytes per stored expert weight: bf16; MXFP8 (E4M3 + one E8M0 byte per 32); MXFP4 (E2M1 + one per 32)
+WEIGHT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 0.5 + 1.0 / 32}
+#: bytes per element of the expert GEMMs' token operands (MXFP8 with block-scaled experts)
+ACT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 1.0 + 1.0 / 32}
+#: tensor-core rate of the block-scaled expert GEMMs relative to bf16 (the nominal fp8 : bf16 ratio, 4.5 : 2.25)
+MX_RATE = 2.0
+
+
 def layer_work(cfg, stats, T):
-    """F (FLOPs) and B (bytes) of one forward from its actual routing (plus the shared expert, if any)."""
+    """F (FLOPs), B (bytes) and F_eff (FLOPs at the bf16 rate that take as long) of one forward, from its actual
+    routing (plus the shared expert, if any)."""
     g = 2 if cfg.gated else 1
+    fmt = getattr(cfg, "expert_fmt", 0)
+    wb = WEIGHT_BYTES[fmt]
     R, E = stats["ffn_rows"], stats["experts_touched"]
     d, L, m, nt = cfg.d, cfg.latent, cfg.m, cfg.n_total
+    fe = 2 * (g + 1) * (L if cfg.has_proj else d) * m * R  # expert FLOPs
     if cfg.has_proj:
-        F = 2 * T * (2 * d * L + d * nt) + 2 * (g + 1) * L * m * R
-        B = 2 * ((g + 1) * L * m * E + 2 * d * L + d * nt) + 2 * 2 * T * d
+        F = 2 * T * (2 * d * L + d * nt)
+        B = wb * (g + 1) * L * m * E + 2 * (2 * d * L + d * nt) + 2 * 2 * T * d
     else:
-        F = 2 * T * d * nt + 2 * (g + 1) * d * m * R
-        B = 2 * ((g + 1) * d * m * E + d * nt) + 4 * T * d
+        F = 2 * T * d * nt
+        B = wb * (g + 1) * d * m * E + 2 * d * nt + 4 * T * d
     ms = getattr(cfg, "shared_m", 0)
     if ms:
         F += 2 * T * (g + 1) * d * ms
         B += 2 * (g + 1) * d * ms
-    return float(F), float(B)
+    F_eff = F + fe / (MX_RATE if fmt else 1.0)
+    return float(F + fe), float(B), float(F_eff)
 
 
 def phase_units(cfg, stats, T, phase):
     """Algorithmic (flops, bytes) of one launch of a phase's kernel."""
     g = 2 if cfg.gated else 1
     d, L, m, nt = cfg.d, cfg.latent, cfg.m, cfg.n_total
+    fmt = getattr(cfg, "expert_fmt", 0)
+    wb, ab = WEIGHT_BYTES[fmt], ACT_BYTES[fmt]
     fin = L  # expert input width (== d for the standard MoE)
     rows_tc = stats.get("tc_rows", 0)
     rows_st = stats.get("stream_rows", 0)
@@ -164,10 +179,10 @@ def phase_units(cfg, stats, T, phase):
         return 2.0 * rows_tc * fin * g * m, 2.0 * (g * m * fin * e_tc + rows_tc * fin + rows_tc * m)
     if phase == "expert_down_gemm":
         return 2.0 * rows_tc * m * fin, 2.0 * (fin * m * e_tc + rows_tc * m + rows_tc * fin)
-    if phase == "expert_up_stream":
-        return 2.0 * rows_st * fin * g * m, 2.0 * (g * m * fin * e_st + rows_st * fin + rows_st * m)
-    if phase == "expert_down_stream":
-        return 2.0 * rows_st * m * fin, 2.0 * (fin * m * e_st + rows_st * m + rows_st * fin)
+    if phase == "expert_up_stream":  # block-scaled: MXFP8 rows in, MXFP8 hidden rows out
+        return 2.0 * rows_st * fin * g * m, wb * g * m * fin * e_st + ab * (rows_st * fin + rows_st * m)
+    if phase == "expert_down_stream":  # bf16 rows out
+        return 2.0 * rows_st * m * fin, wb * fin * m * e_st + ab * rows_st * m + 2.0 * rows_st * fin
     if phase == "router_proj_gemm":
         n_out = (L if cfg.has_proj else 0) + nt
         return 2.0 * T * d * n_out, 2.0 * (n_out * d + T * d) + T * (L * 2 if cfg.has_proj else 0) + 4.0 * T * nt
@@ -302,11 +317,11 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     roof["traffic"] = None
     roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "")
 
-    F, B = layer_work(cfg, stats, T)
-    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9))
+    F, B, F_eff = layer_work(cfg, stats, T)
+    t_f, t_b = F_eff / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_f, t_b)
     layer_roof = {"flops": F, "bytes": B, "t_roof_us": t_roof * 1e6, "t_step_us": ms_max / steps * 1e3,
-                  "frac": t_roof / (ms_max / steps / 1e3),
-                  "bound": "tensor" if F / (peaks["bf16_tflops"] * 1e12) >= B / (peaks["hbm_gbs"] * 1e9) else "hbm"}
+                  "frac": t_roof / (ms_max / steps / 1e3), "bound": "tensor" if t_f >= t_b else "hbm"}
     mod.close()
     roof["kernel_timed_ms_per_step"] = ms_profiled / steps
     return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
@@ -369,10 +384,19 @@ def run_reference(args, cfg, rank, world):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+EXPERT_FORMATS = ["bf16", "mxfp8 (e4m3 weights and expert inputs)", "mxfp4 (e2m1 weights, mxfp8 expert inputs)"]
+
+
+def compute_dtype(cfg):
+    """The arithmetic types the path computes in: bf16 tensor-core GEMMs, plus block-scaled expert GEMMs."""
+    return ["bf16", "bf16+mxfp8", "bf16+mxfp4/mxfp8"][cfg.expert_fmt]
+
+
 def workload_config(cfg):
     return {"workload": cfg.name, "tokens": cfg.tokens, "d": cfg.d, "latent": cfg.latent, "m": cfg.m,
             "experts": cfg.n_ffn, "bypass_experts": [cfg.n_zero, cfg.n_copy, cfg.n_const], "top_k": cfg.top_k,
             "shared_expert_width": cfg.shared_m,
+            "expert_format": EXPERT_FORMATS[cfg.expert_fmt],
             "act": ["relu2", "swiglu", "identity"][cfg.act], "projection": bool(cfg.has_proj),
             "l2": "inputs larger than L2 (the touched expert weights, read every step, exceed the 126 MB L2)",
             "parallelism": "replicas (tokens shard with no exchange)"}
@@ -431,7 +455,7 @@ def main():
         value = world * T * args.steps / (res["ms"] / 1e3)
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res["ms"] / args.steps, "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "scaling": "weak", "vs_baseline": None, "dtype": compute_dtype(cfg), "data": "synthetic",
                 "config": workload_config(cfg), "roofline": res["roofline"],
                 "layer_roofline": res["layer_roofline"], "e2e": res["e2e"], "gpu_launches": res["launches"],
                 "clocks": res["clocks"],

@@ -22,6 +22,12 @@
  * gate: "LatentMoE: How MoE Made a Key Paradigm Leap in 2026", section 2,
  * closing note) adds Ws2 act(Ws1 x_t), act as for the routed experts; it runs
  * on a stream of the handle's own, concurrently with the routed path.
+ * With expert_fmt = LMOE_FMT_MXFP8 or LMOE_FMT_MXFP4 the FFN experts' W1 / W2
+ * are stored block-scaled (Open Compute Project Microscaling v1.0; the pages
+ * name MXFP4 as the Kimi K3 serving format, in the comparison table of "Two
+ * Teams, Two Practices"), and the rows those matrices multiply (z_t, and
+ * act(W1_e z_t)) are encoded in MXFP8 from their bf16 values before the
+ * multiply; see lmoe_mx_encode_weights for the format and layout.
  *
  * Conventions for every entry point:
  *   - all matrices are row-major; bf16 tensors are passed as `void *` (IEEE
@@ -65,12 +71,18 @@ extern "C" {
 #define LMOE_ACT_SWIGLU 1   /* W1_e rows [0,m) gate, [m,2m) up: h = silu(gate) * up */
 #define LMOE_ACT_IDENTITY 2 /* h = u (test use) */
 
+#define LMOE_FMT_BF16 0  /* expert weights in bf16 */
+#define LMOE_FMT_MXFP8 1 /* E4M3 elements, one E8M0 scale per 32 along K */
+#define LMOE_FMT_MXFP4 2 /* E2M1 elements, one E8M0 scale per 32 along K */
+
 /*
  * Layer shape.  Constraints (else LMOE_ERR_UNSUPPORTED_SHAPE): d, latent and m
  * multiples of 64 and at most 16384; 1 <= top_k <= min(32, n_total);
  * n_total = n_experts + n_zero + n_copy + n_const <= 1024; n_experts >= 1;
  * max_tokens >= 1; has_proj == 0 requires latent == d; shared_m is 0 or a
- * multiple of 64 up to 16384.
+ * multiple of 64 up to 16384.  A block-scaled expert_fmt also requires
+ * latent and m to be multiples of 128 and max_tokens <= 32 (the decode
+ * regime, where every expert streams its weights).
  */
 typedef struct lmoe_config {
     int32_t d;             /* model width */
@@ -86,6 +98,7 @@ typedef struct lmoe_config {
     int32_t has_proj;      /* 1: LatentMoE with W_down / W_up; 0: standard MoE */
     int32_t latent_router; /* 1: the gate reads z (latent) instead of x (d) */
     int32_t shared_m;      /* hidden width of the shared expert at d; 0: no shared expert */
+    int32_t expert_fmt;    /* LMOE_FMT_*: storage of the FFN experts' W1 / W2 */
 } lmoe_config;
 
 /* Device pointers to the layer's weights (bf16 unless stated).  n_total as above. */
@@ -94,11 +107,13 @@ typedef struct lmoe_weights {
     const float *router_bias; /* fp32 [n_total], added to the logits before selection; may be NULL */
     const void *w_down;       /* [latent, d]; NULL when has_proj == 0 */
     const void *w_up;         /* [d, latent]; NULL when has_proj == 0 */
-    const void *w1;           /* [n_experts, g*m, latent], g = 2 for SwiGLU else 1 */
-    const void *w2;           /* [n_experts, latent, m] */
+    const void *w1;           /* [n_experts, g*m, latent], g = 2 for SwiGLU else 1 (block-scaled: codes) */
+    const void *w2;           /* [n_experts, latent, m] (block-scaled: codes) */
     const void *const_vecs;   /* [n_const, latent]; may be NULL when n_const == 0 */
     const void *w_shared1;    /* [g*shared_m, d] (gate rows first when gated); NULL when shared_m == 0 */
     const void *w_shared2;    /* [d, shared_m]; NULL when shared_m == 0 */
+    const void *w1_scales;    /* block-scaled only: E8M0 scale atoms of w1 (lmoe_mx_encode_weights); else NULL */
+    const void *w2_scales;    /* block-scaled only: E8M0 scale atoms of w2; else NULL */
 } lmoe_weights;
 
 /*
@@ -255,6 +270,34 @@ LMOE_API int lmoe_gemm_bf16(const void *A, const void *B, void *C, int32_t M, in
  */
 LMOE_API int lmoe_dispatch_noalloc(const int32_t *idx, int32_t T, int32_t top_k, int32_t n_total, int32_t *counts,
                                    int32_t *offsets, int32_t *perm, int32_t *inv, void *stream);
+
+/*
+ * Block-scaled (MX) encoding of a bf16 weight matrix, for lmoe_weights.w1 /
+ * w2 with a block-scaled expert_fmt.  It follows the Open Compute Project
+ * Microscaling specification v1.0 (the pages name the format only).  Each
+ * row is split into blocks of 32 consecutive values along K.  A block shares
+ * one scale 2^s, stored as the E8M0 byte s + 127, with
+ * s = floor(log2 max|v|) - emax: emax is 8 for E4M3, 2 for E2M1; s is clamped
+ * to [-127, 127]; an all-zero block gets s = -127.  Each element is v / 2^s
+ * rounded to the nearest element value, ties to even, and saturated at
+ * +-448 (E4M3) or +-6 (E2M1).
+ *
+ *   w       device bf16 [rows, K]: an expert tensor viewed as rows, e.g. W1
+ *           as [n_experts * g * m, latent], W2 as [n_experts * latent, m]
+ *   rows    multiple of 128;  K multiple of 128
+ *   fmt     LMOE_FMT_MXFP8 or LMOE_FMT_MXFP4
+ *   codes   device, [rows, K] bytes (E4M3), or [rows, K/2] bytes (E2M1: two
+ *           per byte, element 2i in the low nibble of byte i)
+ *   scales  device, rows * K / 32 bytes, in 512-byte atoms
+ *           [rows/128][K/128][32][16]: byte (r, c) of atom (R, G) holds the
+ *           scale of row 128R + 32(c/4) + r, block 4G + c%4 (the order in
+ *           which the tensor cores read block scales)
+ *
+ * Bad sizes or format: LMOE_ERR_UNSUPPORTED_SHAPE; a NULL or misaligned
+ * pointer: LMOE_ERR_INVALID_ARG.  Asynchronous on `stream`; deterministic.
+ */
+LMOE_API int lmoe_mx_encode_weights(const void *w, int64_t rows, int32_t K, int32_t fmt, void *codes, void *scales,
+                                    void *stream);
 
 #ifdef __cplusplus
 }

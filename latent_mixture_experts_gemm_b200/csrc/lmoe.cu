@@ -20,6 +20,7 @@
 
 #include "../../include/lmoe.h"
 #include "moe_kernels.cuh"
+#include "mx.cuh"
 #include "tc_gemm.cuh"
 #include "tc_swap.cuh"
 
@@ -55,6 +56,36 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
     return r == CUDA_SUCCESS;
 }
 
+// Byte matrix [rows, cols] (row pitch `ld` bytes): E4M3 codes (box_cols = 128 with the 128-byte swizzle) or
+// block-scale rows (box_cols = 16, no swizzle).
+bool make_map_u8(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_cols,
+                 uint32_t box_rows, bool swizzle) {
+    if (!load_encode() || rows == 0) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// E2M1 codes [rows, K] packed two per byte in global memory; each load lands as 128 rows x 128 elements with
+// every 16 packed elements padded to 16 bytes, the shared-memory form the E2M1 tensor-core operand takes.
+bool make_map_e2m1(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+    if (!load_encode() || rows == 0) return false;
+    cuuint64_t dims[2] = {K, rows};
+    cuuint64_t strides[1] = {K / 2};
+    cuuint32_t box[2] = {128, 128};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 int n_total(const lmoe_config& c) { return c.n_experts + c.n_zero + c.n_copy + c.n_const; }
@@ -72,8 +103,15 @@ bool config_ok(const lmoe_config& c) {
     if (c.latent_router != 0 && c.latent_router != 1) return false;
     if (!c.has_proj && c.latent != c.d) return false;
     if (c.shared_m != 0 && !dim_ok(c.shared_m)) return false;
+    if (c.expert_fmt < LMOE_FMT_BF16 || c.expert_fmt > LMOE_FMT_MXFP4) return false;
+    if (c.expert_fmt != LMOE_FMT_BF16 && (c.latent % 128 != 0 || c.m % 128 != 0 || c.max_tokens > SMALL_MAX))
+        return false;
     return true;
 }
+
+// Row pitch (bytes) of the block-scale rows of an MXFP8 token operand with K columns: one 16-byte chunk per
+// 128-element stage (K is a multiple of 128 for block-scaled experts).
+int mx_ld_sf(int K) { return K / 128 * 16; }
 
 // Few-token path (T <= kFewTokenRows): the projections stream their weights
 // with split-K on the weight-streaming kernel.
@@ -82,7 +120,7 @@ constexpr int kFewTokenMaxSplits = 16;
 
 struct Plan {
     size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
-        partial, hs, s2, partial2, xin, yout, total;
+        partial, hs, s2, partial2, rows8, rows_sf, h8, h_sf, xin, yout, total;
     int ld_logits, nwords, mt_max;
 };
 
@@ -127,6 +165,12 @@ Plan make_plan(const lmoe_config& c) {
         p.hs = take(T * static_cast<size_t>(c.shared_m) * 2);
         p.s2 = take(T * d * 2);
         p.partial2 = take(static_cast<size_t>(kFewTokenMaxSplits) * srows * kFewTokenRows * 4);
+    }
+    if (c.expert_fmt != LMOE_FMT_BF16) {  // MXFP8 token operands of the expert GEMMs: codes and block scales
+        p.rows8 = take(R * L);
+        p.rows_sf = take(R * mx_ld_sf(static_cast<int>(L)));
+        p.h8 = take(R * m);
+        p.h_sf = take(R * mx_ld_sf(static_cast<int>(m)));
     }
     p.xin = take(T * d * 2);
     p.yout = take(T * d * 2);
@@ -174,8 +218,22 @@ bool set_swap_attr() {
                                 SwapCfg<NT, EPI>::SMEM_BYTES) == cudaSuccess;
 }
 
+template <int EPI, bool W4, bool QOUT>
+bool set_mx_attr() {
+    return cudaFuncSetAttribute(tc_swap_mx_kernel<EPI, W4, QOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                MxCfg<EPI, W4>::SMEM_BYTES) == cudaSuccess;
+}
+
 bool set_all_smem_attrs() {
     bool ok = true;
+    ok &= set_mx_attr<EPI_BF16, false, true>();
+    ok &= set_mx_attr<EPI_RELU2, false, true>();
+    ok &= set_mx_attr<EPI_SWIGLU, false, true>();
+    ok &= set_mx_attr<EPI_BF16, false, false>();
+    ok &= set_mx_attr<EPI_BF16, true, true>();
+    ok &= set_mx_attr<EPI_RELU2, true, true>();
+    ok &= set_mx_attr<EPI_SWIGLU, true, true>();
+    ok &= set_mx_attr<EPI_BF16, true, false>();
     ok &= cudaFuncSetAttribute(dispatch_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (2 * SMALL_BATCH_WORDS * 1024 + 1024) * 4) == cudaSuccess;
     ok &= set_swap_attr<16, EPI_BF16>();
@@ -285,6 +343,30 @@ void launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& 
     launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, args);
 }
 
+template <int EPI, bool W4, bool QOUT>
+void launch_mx(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf, const MxArgs& a, int grid,
+               cudaStream_t s) {
+    launch(tc_swap_mx_kernel<EPI, W4, QOUT>, grid, 192, MxCfg<EPI, W4>::SMEM_BYTES, s, w, x, xsf, a);
+}
+
+// Block-scaled expert phase: the up GEMM (activation, MXFP8 re-encoding) or the down GEMM (bf16 out).
+void launch_mx_phase(bool up, int epi, bool w4, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf,
+                     const MxArgs& a, int grid, cudaStream_t s) {
+    if (!up) {
+        if (w4) launch_mx<EPI_BF16, true, false>(w, x, xsf, a, grid, s);
+        else launch_mx<EPI_BF16, false, false>(w, x, xsf, a, grid, s);
+    } else if (epi == EPI_RELU2) {
+        if (w4) launch_mx<EPI_RELU2, true, true>(w, x, xsf, a, grid, s);
+        else launch_mx<EPI_RELU2, false, true>(w, x, xsf, a, grid, s);
+    } else if (epi == EPI_SWIGLU) {
+        if (w4) launch_mx<EPI_SWIGLU, true, true>(w, x, xsf, a, grid, s);
+        else launch_mx<EPI_SWIGLU, false, true>(w, x, xsf, a, grid, s);
+    } else {
+        if (w4) launch_mx<EPI_BF16, true, true>(w, x, xsf, a, grid, s);
+        else launch_mx<EPI_BF16, false, true>(w, x, xsf, a, grid, s);
+    }
+}
+
 }  // namespace
 
 // ====================================================================== handle
@@ -306,6 +388,8 @@ struct lmoe_handle {
     // shared expert: weights for 64/256-column tiles (gated: half-tile boxes), 128-row weight tiles,
     // its hidden rows as the A operand (128-row tiles) and as 16/32-row token tiles
     CUtensorMap ws1_64{}, ws1_256{}, ws2_64{}, ws2_256{}, ws1_128{}, ws2_128{}, a_hs{}, hs16{}, hs32{};
+    // block-scaled experts: weight codes (128 x 128 boxes) and the MXFP8 token operands with their scales
+    CUtensorMap w1q{}, w2q{}, rows8{}, rows_sf{}, h8{}, h_sf{};
     cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     // profiling
@@ -509,8 +593,10 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     }
     // Experts with at most `small` rows stream their weights; when every expert
     // must (T <= small) the grouped GEMMs are not launched at all.
+    const bool mx = c.expert_fmt != LMOE_FMT_BF16;
     int small = h->small_max;
     if (small > 0 && T <= SMALL_MAX) small = T <= 16 ? 16 : SMALL_MAX;
+    if (mx) small = SMALL_MAX;  // block-scaled experts always stream (T <= 32 is a create-time limit)
     const bool need_tc = T > small;
     h->last_small = small;
     const int nwords = (T + 31) / 32;
@@ -540,8 +626,12 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         const size_t sm = (static_cast<size_t>(2 * nwords) * nt + nt) * 4;
         launch(dispatch_small_kernel, 1, 1024, sm, s, idx, T, K, nt, c.n_experts, small, counts, offsets, mt_list,
                small_list, perm, inv, hdr);
-        launch(dispatch_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
-               feat, L, L, rows, L);
+        if (mx)
+            launch(mx_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
+                   feat, L, L, h->at<uint8_t>(p.rows8), L, h->at<uint8_t>(p.rows_sf), mx_ld_sf(L));
+        else
+            launch(dispatch_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K,
+                   c.n_experts, feat, L, L, rows, L);
     } else {
         PhaseScope ps(h, PH_DISPATCH, s, 4);
         uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
@@ -575,7 +665,26 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
             launch_gemm<256, EPI_BF16>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
         }
     }
-    if (small > 0) {
+    if (mx) {
+        PhaseScope ps(h, PH_UP_STREAM, s, 1);
+        MxArgs a{};
+        a.K = L;
+        a.n_wtiles = m / 128;
+        a.list = small_list;
+        a.count = hdr + HDR_NSMALL;
+        a.w_rows_per_expert = h->g * m;
+        a.up_offset = m;
+        a.w_sf = static_cast<const uint8_t*>(h->w.w1_scales);
+        a.n_out = m;
+        a.out8 = h->at<uint8_t>(p.h8);
+        a.out_sf = h->at<uint8_t>(p.h_sf);
+        a.ld_out8 = m;
+        a.ld_out_sf = mx_ld_sf(m);
+        a.err = hdr + HDR_ERR;
+        a.timeout_ns = h->timeout_ns;
+        const int epi = c.act == LMOE_ACT_SWIGLU ? EPI_SWIGLU : (c.act == LMOE_ACT_RELU2 ? EPI_RELU2 : EPI_BF16);
+        launch_mx_phase(true, epi, c.expert_fmt == LMOE_FMT_MXFP4, h->w1q, h->rows8, h->rows_sf, a, h->num_sms, s);
+    } else if (small > 0) {
         PhaseScope ps(h, PH_UP_STREAM, s, 1);
         SwapArgs a{};
         a.K = L;
@@ -607,7 +716,23 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.n_tiles = (L + 255) / 256;
         launch_gemm<256, EPI_BF16>(h->a_h, h->w2, h->w2, a, h->num_sms, s);
     }
-    if (small > 0) {
+    if (mx) {
+        PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
+        MxArgs a{};
+        a.K = m;
+        a.n_wtiles = L / 128;
+        a.list = small_list;
+        a.count = hdr + HDR_NSMALL;
+        a.w_rows_per_expert = L;
+        a.up_offset = 0;
+        a.w_sf = static_cast<const uint8_t*>(h->w.w2_scales);
+        a.n_out = L;
+        a.out = rows;
+        a.ld_out = L;
+        a.err = hdr + HDR_ERR;
+        a.timeout_ns = h->timeout_ns;
+        launch_mx_phase(false, EPI_BF16, c.expert_fmt == LMOE_FMT_MXFP4, h->w2q, h->h8, h->h_sf, a, h->num_sms, s);
+    } else if (small > 0) {
         PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
         SwapArgs a{};
         a.K = m;
@@ -709,9 +834,16 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     if (c.n_const > 0 && w->const_vecs == nullptr) return LMOE_ERR_INVALID_ARG;
     if (c.shared_m > 0 && (w->w_shared1 == nullptr || w->w_shared2 == nullptr)) return LMOE_ERR_INVALID_ARG;
     const void* ptrs[] = {w->w_router, w->router_bias, w->w_down, w->w_up, w->w1, w->w2, w->const_vecs,
-                          w->w_shared1, w->w_shared2};
+                          w->w_shared1, w->w_shared2, w->w1_scales, w->w2_scales};
     for (const void* q : ptrs)
         if (!aligned16(q)) return LMOE_ERR_INVALID_ARG;
+    if (c.expert_fmt != LMOE_FMT_BF16) {
+        if (w->w1_scales == nullptr || w->w2_scales == nullptr) return LMOE_ERR_INVALID_ARG;
+        // the packed E2M1 copy reads from 32-byte aligned rows
+        if (c.expert_fmt == LMOE_FMT_MXFP4 &&
+            ((reinterpret_cast<uintptr_t>(w->w1) | reinterpret_cast<uintptr_t>(w->w2)) & 31) != 0)
+            return LMOE_ERR_INVALID_ARG;
+    }
 
     lmoe_handle* h = new (std::nothrow) lmoe_handle();
     if (h == nullptr) return LMOE_ERR_INVALID_ARG;
@@ -748,12 +880,27 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
         ok &= make_map(&h->yl16, h->at<void>(p.yl), c.max_tokens, L, L, 16);
         ok &= make_map(&h->yl32, h->at<void>(p.yl), c.max_tokens, L, L, 32);
     }
-    ok &= make_map(&h->w1, w->w1, static_cast<uint64_t>(c.n_experts) * h->g * m, L, L, h->g == 2 ? 128 : 256);
-    ok &= make_map(&h->w2, w->w2, static_cast<uint64_t>(c.n_experts) * L, m, m, 256);
+    const uint64_t w1_rows = static_cast<uint64_t>(c.n_experts) * h->g * m, w2_rows = static_cast<uint64_t>(c.n_experts) * L;
+    if (c.expert_fmt == LMOE_FMT_BF16) {
+        ok &= make_map(&h->w1, w->w1, w1_rows, L, L, h->g == 2 ? 128 : 256);
+        ok &= make_map(&h->w2, w->w2, w2_rows, m, m, 256);
+        ok &= make_map(&h->w1s, w->w1, w1_rows, L, L, 128);
+        ok &= make_map(&h->w2s, w->w2, w2_rows, m, m, 128);
+    } else {
+        if (c.expert_fmt == LMOE_FMT_MXFP4) {
+            ok &= make_map_e2m1(&h->w1q, w->w1, w1_rows, L);
+            ok &= make_map_e2m1(&h->w2q, w->w2, w2_rows, m);
+        } else {
+            ok &= make_map_u8(&h->w1q, w->w1, w1_rows, L, L, 128, 128, true);
+            ok &= make_map_u8(&h->w2q, w->w2, w2_rows, m, m, 128, 128, true);
+        }
+        ok &= make_map_u8(&h->rows8, h->at<void>(p.rows8), R, L, L, 128, 32, true);
+        ok &= make_map_u8(&h->rows_sf, h->at<void>(p.rows_sf), R, mx_ld_sf(L), mx_ld_sf(L), 16, 32, false);
+        ok &= make_map_u8(&h->h8, h->at<void>(p.h8), R, m, m, 128, 32, true);
+        ok &= make_map_u8(&h->h_sf, h->at<void>(p.h_sf), R, mx_ld_sf(m), mx_ld_sf(m), 16, 32, false);
+    }
     ok &= make_map(&h->a_rows, h->at<void>(p.rows), R, L, L, 128);
     ok &= make_map(&h->a_h, h->at<void>(p.hbuf), R, m, m, 128);
-    ok &= make_map(&h->w1s, w->w1, static_cast<uint64_t>(c.n_experts) * h->g * m, L, L, 128);
-    ok &= make_map(&h->w2s, w->w2, static_cast<uint64_t>(c.n_experts) * L, m, m, 128);
     ok &= make_map(&h->rows16, h->at<void>(p.rows), R, L, L, 16);
     ok &= make_map(&h->rows32, h->at<void>(p.rows), R, L, L, 32);
     ok &= make_map(&h->h16, h->at<void>(p.hbuf), R, m, m, 16);
@@ -969,6 +1116,27 @@ int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, 
         a.n_tiles = (N + 63) / 64;
         launch_gemm<64, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);
     }
+    return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+int lmoe_mx_encode_weights(const void* w, int64_t rows, int32_t K, int32_t fmt, void* codes, void* scales,
+                           void* stream) {
+    if (fmt != LMOE_FMT_MXFP8 && fmt != LMOE_FMT_MXFP4) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows < 0 || rows % 128 != 0 || K < 128 || K % 128 != 0 || K > 65536) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0) return LMOE_OK;
+    if (w == nullptr || codes == nullptr || scales == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned16(scales)) return LMOE_ERR_INVALID_ARG;
+    const long long blocks = rows * (K / 32);
+    const unsigned grid = static_cast<unsigned>((blocks + 255) / 256);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const __nv_bfloat16* wb = static_cast<const __nv_bfloat16*>(w);
+    // a plain launch: this kernel does not wait on a predecessor (no programmatic dependent launch)
+    if (fmt == LMOE_FMT_MXFP4)
+        mx_encode_weights_kernel<true><<<grid, 256, 0, s>>>(wb, rows, K, static_cast<uint8_t*>(codes),
+                                                            static_cast<uint8_t*>(scales));
+    else
+        mx_encode_weights_kernel<false><<<grid, 256, 0, s>>>(wb, rows, K, static_cast<uint8_t*>(codes),
+                                                             static_cast<uint8_t*>(scales));
     return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 

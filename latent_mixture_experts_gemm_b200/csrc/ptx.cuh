@@ -100,6 +100,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 1-D bulk copy global -> shared (no tensor map), completion on `bar`.  Both
+// addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05
 // Shared-memory matrix descriptor for a K-major operand tile stored with the
 // 128-byte swizzle (rows of 64 bf16 = 128 B, 8-row atoms of 1024 B).
@@ -130,6 +138,56 @@ __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint6
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand without swizzle: 8-row x
+// 16-byte core matrices, `sbo` bytes between successive 8-row groups.  Used
+// as the source of tcgen05.cp (one 16-byte core-matrix column, so the leading
+// offset is never used).
+__device__ __forceinline__ uint64_t umma_desc_plain(uint32_t saddr, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;  // descriptor version for tcgen05; swizzle mode 0 (none)
+    return d;
+}
+
+// Element formats of kind::mxf8f6f4 operands.
+enum : uint32_t { MXF_E4M3 = 0, MXF_E2M1 = 5 };
+
+// Instruction descriptor of a block-scaled MMA (kind::mxf8f6f4, E8M0 scales,
+// fp32 accumulate, both operands K-major).  The scale-factor ids (which byte
+// of each 32-bit TMEM scale column the MMA reads) are OR-ed in per MMA with
+// umma_idesc_sf_ids.
+__host__ __device__ constexpr uint32_t umma_idesc_mx(int M, int N, uint32_t atype, uint32_t btype) {
+    return (atype << 7)                             // A element format
+           | (btype << 10)                          // B element format
+           | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+           | (1u << 23)                             // scale format: E8M0
+           | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
+}
+__host__ __device__ constexpr uint32_t umma_idesc_sf_ids(uint32_t a_id, uint32_t b_id) {
+    return (b_id << 4) | (a_id << 29);
+}
+
+// D (+)= (A * 2^SFA) (B * 2^SFB)^T with per-32-element block scales read from
+// TMEM at tmem_sfa / tmem_sfb.
+__device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
+        : "memory");
+}
+
+// Copy 32 rows x 16 bytes of shared memory into 4 TMEM columns of lanes 0-31,
+// repeated in each of the four 32-lane sub-partitions (the layout the MMA
+// reads its scale factors from).  Ordered before the MMAs this thread issues
+// after it.
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.

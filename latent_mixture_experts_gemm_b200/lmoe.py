@@ -16,6 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblmoe.so")
 
 LMOE_OK = 0
+LMOE_FMT_BF16, LMOE_FMT_MXFP8, LMOE_FMT_MXFP4 = 0, 1, 2
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_ARG", -2: "LMOE_ERR_UNSUPPORTED_SHAPE", -3: "LMOE_ERR_TOO_MANY_TOKENS",
           -4: "LMOE_ERR_CUDA", -5: "LMOE_ERR_TIMEOUT", -6: "LMOE_ERR_BAD_INDEX", -7: "LMOE_ERR_WORKSPACE"}
 
@@ -25,12 +26,12 @@ I32 = ctypes.c_int32
 
 class lmoe_config(ctypes.Structure):
     _fields_ = [(n, I32) for n in ("d", "latent", "m", "n_experts", "top_k", "max_tokens", "act", "n_zero", "n_copy",
-                                   "n_const", "has_proj", "latent_router", "shared_m")]
+                                   "n_const", "has_proj", "latent_router", "shared_m", "expert_fmt")]
 
 
 class lmoe_weights(ctypes.Structure):
     _fields_ = [("w_router", P), ("router_bias", P), ("w_down", P), ("w_up", P), ("w1", P), ("w2", P),
-                ("const_vecs", P), ("w_shared1", P), ("w_shared2", P)]
+                ("const_vecs", P), ("w_shared1", P), ("w_shared2", P), ("w1_scales", P), ("w2_scales", P)]
 
 
 class lmoe_debug(ctypes.Structure):
@@ -76,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
         L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
         L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
+        L.lmoe_mx_encode_weights.argtypes = [P, ctypes.c_int64, I32, I32, P, P, P]
         _lib = L
     return _lib
 
@@ -190,17 +192,36 @@ def lmoe_dispatch_noalloc(idx: torch.Tensor, n_total: int, counts: torch.Tensor,
         _p(idx), T, K, n_total, _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)))
 
 
+def lmoe_mx_encode_weights(w: torch.Tensor, fmt: int, stream=None):
+    """Block-scaled (MX) encoding of a device bf16 weight tensor viewed as rows x K (K = last dimension).
+
+    Returns ``(codes, scales)`` as new device uint8 tensors: codes [rows, K] (MXFP8) or [rows, K/2] (MXFP4,
+    element 2i in the low nibble of byte i), scales rows*K/32 bytes in the tensor-core atom order that
+    ``include/lmoe.h`` describes.
+    """
+    K = int(w.shape[-1])
+    rows = w.numel() // K
+    codes = torch.empty((rows, K if fmt == LMOE_FMT_MXFP8 else K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(rows * K // 32, dtype=torch.uint8, device=w.device)
+    _check("lmoe_mx_encode_weights", lib().lmoe_mx_encode_weights(
+        w.data_ptr(), rows, K, int(fmt), codes.data_ptr(), scales.data_ptr(), _stream(stream)))
+    return codes, scales
+
+
 # ------------------------------------------------------------------ convenience owner of a layer
 def make_config(cfg, max_tokens: int) -> lmoe_config:
     return lmoe_config(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, int(max_tokens), cfg.act, cfg.n_zero,
-                       cfg.n_copy, cfg.n_const, cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0))
+                       cfg.n_copy, cfg.n_const, cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0),
+                       getattr(cfg, "expert_fmt", 0))
 
 
 class LatentMoE:
     """A layer on one GPU: device copies of the weights, a workspace and a handle.
 
     ``cfg`` is a ``synth.LayerConfig`` (or anything with the same fields),
-    ``layer`` the dict of CPU tensors from ``synth.make_layer``.
+    ``layer`` the dict of CPU tensors from ``synth.make_layer``.  With a
+    block-scaled ``cfg.expert_fmt`` the bf16 W1 / W2 are encoded on the device
+    by ``lmoe_mx_encode_weights`` and only the encodings are kept.
     """
 
     def __init__(self, cfg, layer: Dict[str, torch.Tensor], max_tokens: int, device: str = "cuda"):
@@ -210,6 +231,13 @@ class LatentMoE:
         dev = lambda t: None if t is None else t.to(self.device).contiguous()  # noqa: E731
         self.w = {k: dev(layer.get(k)) for k in ("w_router", "bias", "w_down", "w_up", "w1", "w2", "const_vecs",
                                                   "w_shared1", "w_shared2")}
+        self.w["w1_scales"] = self.w["w2_scales"] = None
+        fmt = getattr(cfg, "expert_fmt", 0)
+        if fmt != LMOE_FMT_BF16:
+            with torch.cuda.device(self.device):
+                for k in ("w1", "w2"):
+                    self.w[k], self.w[k + "_scales"] = lmoe_mx_encode_weights(self.w[k], fmt)
+                torch.cuda.synchronize(self.device)
         self.c = make_config(cfg, self.max_tokens)
         nbytes = lmoe_workspace_bytes(self.c)
         if nbytes == 0:
@@ -217,7 +245,8 @@ class LatentMoE:
         self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.weights = lmoe_weights(_p(self.w["w_router"]), _p(self.w["bias"]), _p(self.w["w_down"]),
                                     _p(self.w["w_up"]), _p(self.w["w1"]), _p(self.w["w2"]), _p(self.w["const_vecs"]),
-                                    _p(self.w["w_shared1"]), _p(self.w["w_shared2"]))
+                                    _p(self.w["w_shared1"]), _p(self.w["w_shared2"]), _p(self.w["w1_scales"]),
+                                    _p(self.w["w2_scales"]))
         with torch.cuda.device(self.device):
             self.h = lmoe_create(self.c, self.weights, self.workspace.data_ptr(), nbytes)
 

@@ -241,11 +241,14 @@ static void mx_activation(const double *v, int n, double *out)
     }
 }
 
-/* An MX-encoded weight matrix: codes [rows, in_dim], scales [rows, in_dim/32]. */
+/* An MX-encoded weight matrix: codes [rows, in_dim], scales [rows, in_dim/32],
+ * with the value of every element code and of every scale byte tabulated
+ * (elem_value and 2^(byte - 127): the same numbers, looked up). */
 typedef struct {
     const uint8_t *codes;
     const uint8_t *scales;
-    int e2m1;
+    const double *elem; /* 256 entries */
+    const double *pow2; /* 256 entries */
 } mx_matrix;
 
 /* out[o] = sum_i value(W[o, i]) * v[i] for an MX-encoded W */
@@ -255,7 +258,7 @@ static void matvec_mx(int out_dim, int in_dim, mx_matrix W, const double *v, dou
         const uint8_t *row = W.codes + (size_t)o * in_dim;
         const uint8_t *sc = W.scales + (size_t)o * (in_dim / 32);
         double s = 0.0;
-        for (int i = 0; i < in_dim; ++i) s += ldexp(elem_value(row[i], W.e2m1), (int)sc[i / 32] - 127) * v[i];
+        for (int i = 0; i < in_dim; ++i) s += W.elem[row[i]] * W.pow2[sc[i / 32]] * v[i];
         out[o] = s;
     }
 }
@@ -403,6 +406,11 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
 
     /* step 9: encode the FFN experts' weights once (they are the layer's stored weights) */
     uint8_t *c1 = NULL, *s1 = NULL, *c2 = NULL, *s2 = NULL;
+    double elem_tab[256], pow2_tab[256];
+    for (int i = 0; i < 256; ++i) {
+        elem_tab[i] = fmt == ORACLE_FMT_MXFP4 ? (i < 16 ? elem_value((uint8_t)i, 1) : 0.0) : elem_value((uint8_t)i, 0);
+        pow2_tab[i] = ldexp(1.0, i - 127);
+    }
     if (fmt != ORACLE_FMT_BF16) {
         const size_t n1 = (size_t)c->n_ffn * up_rows * L, n2 = (size_t)c->n_ffn * L * m;
         c1 = (uint8_t *)malloc(n1 > 0 ? n1 : 1);
@@ -479,7 +487,8 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
                         m1.scales = s1 + (size_t)e * up_rows * (L / 32);
                         m2.codes = c2 + (size_t)e * L * m;
                         m2.scales = s2 + (size_t)e * L * (m / 32);
-                        m1.e2m1 = m2.e2m1 = fmt == ORACLE_FMT_MXFP4;
+                        m1.elem = m2.elem = elem_tab;
+                        m1.pow2 = m2.pow2 = pow2_tab;
                     }
                     ffn_expert(c, w1 + (size_t)e * up_rows * L, w2 + (size_t)e * L * m,
                                fmt != ORACLE_FMT_BF16 ? &m1 : NULL, fmt != ORACLE_FMT_BF16 ? &m2 : NULL, z, zq, u, h,

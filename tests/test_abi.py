@@ -91,3 +91,32 @@ def test_gemm_shape_checks():
     assert L.lmoe_gemm_bf16(0x100, 0x100, 0x100, 128, 100, 64, None, 0x100) == -2
     assert L.lmoe_gemm_bf16(0x100, 0x100, 0x100, 128, 64, 96, None, 0x100) == -2
     assert L.lmoe_gemm_bf16(0x100, 0x100, 0x100, 128, 64, 64, None, None) == -1
+
+
+def test_block_scaled_config_and_encoder_checks():
+    L = lmoe.lib()
+    ok = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp4"], 32)
+    assert lmoe.lmoe_workspace_bytes(ok) > lmoe.lmoe_workspace_bytes(lmoe.make_config(synth.WORKLOADS["nemotron_decode"], 32))
+    # block-scaled experts: decode batches only, latent and m whole 128-element stages, formats 0..2
+    for b in (dict(max_tokens=33), dict(latent=192), dict(m=320), dict(expert_fmt=3), dict(expert_fmt=-1)):
+        c = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp8"], 32)
+        for k, v in b.items():
+            setattr(c, k, v)
+        assert lmoe.lmoe_workspace_bytes(c) == 0, b
+    # a block-scaled layer without scale pointers, and MXFP4 codes off the 32-byte grid, are rejected
+    cfg = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp4"], 32)
+    big = lmoe.lmoe_workspace_bytes(cfg)
+    h = ctypes.c_void_p()
+    w = lmoe.lmoe_weights(w_router=0x10000, w_down=0x10000, w_up=0x10000, w1=0x10000, w2=0x10000)
+    assert L.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), 0x100000, big, ctypes.byref(h)) == -1
+    w = lmoe.lmoe_weights(w_router=0x10000, w_down=0x10000, w_up=0x10000, w1=0x10010, w2=0x10000,
+                          w1_scales=0x20000, w2_scales=0x20000)
+    assert L.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), 0x100000, big, ctypes.byref(h)) == -1
+    assert h.value is None
+    # the encoder checks sizes and format before anything else
+    assert L.lmoe_mx_encode_weights(0x100, 100, 128, 1, 0x100, 0x100, None) == -2
+    assert L.lmoe_mx_encode_weights(0x100, 128, 96, 2, 0x100, 0x100, None) == -2
+    assert L.lmoe_mx_encode_weights(0x100, 128, 128, 0, 0x100, 0x100, None) == -2
+    assert L.lmoe_mx_encode_weights(None, 128, 128, 1, 0x100, 0x100, None) == -1
+    assert L.lmoe_mx_encode_weights(0x108, 128, 128, 1, 0x100, 0x100, None) == -1
+    assert L.lmoe_mx_encode_weights(0x100, 0, 128, 1, None, None, None) == 0
