@@ -190,13 +190,19 @@ struct MxCfg {
     static constexpr int STAGE_BYTES = (OFF_SFB + SF_BYTES + 1023) / 1024 * 1024;
     static constexpr int TX_BYTES = NA * A_TX + B_BYTES + (NA + 1) * SF_BYTES;
     static constexpr int STAGES = (NA == 2) ? 5 : 10;
-    static constexpr int ACC_COLS = NA * NT;
-    static constexpr int SF_COL = 128;  // TMEM scale columns: weight tile 0 at +0, tile 1 at +4, tokens at +8
-    static constexpr int TMEM_COLS = 256;
+    // Two accumulation chains per weight tile (even / odd K = 32 steps), so consecutive MMAs do not wait on
+    // one another's accumulator; the epilogue adds them.  Chain c of weight tile a at column (c * NA + a) * NT.
+    static constexpr int CHAINS = 2;
+    static constexpr int ACC_COLS = CHAINS * NA * NT;  // one accumulator set (two sets: double buffering)
+    // TMEM scale columns: a ring of SF_SLOTS slots after the accumulators; a slot holds the stage's weight
+    // scales (4 columns per weight tile) and then its token scales (4 columns)
+    static constexpr int SF_COL = 2 * ACC_COLS;
+    static constexpr int SF_SLOT = 4 * (NA + 1);
+    static constexpr int SF_SLOTS = 4;
+    static constexpr int TMEM_COLS = SF_COL + SF_SLOTS * SF_SLOT <= 256 ? 256 : 512;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
-    static_assert(2 * ACC_COLS <= SF_COL, "accumulators overlap the scale columns");
-    // every scale-factor address the MMA and tcgen05.cp see (SF_COL, +4, +8) is a multiple of four columns
-    static_assert(SF_COL % 4 == 0 && SF_COL + 12 <= TMEM_COLS, "scale columns");
+    // every scale-factor address the MMA and tcgen05.cp see is a multiple of four columns
+    static_assert(SF_COL % 4 == 0 && SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "scale columns");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
@@ -205,8 +211,9 @@ struct MxCfg {
 // Per stage of 128 K elements: the weight tile(s) and the token tile by TMA
 // (E2M1 weights through the packed-to-padded 16U4 copy), the weight scale
 // atom(s) by a bulk copy, and the stage's 16-byte token-scale chunk of each
-// token row by TMA.  The MMA thread moves the scales to TMEM with tcgen05.cp and issues
-// four K = 32 block-scaled MMAs.  With QOUT the epilogue applies the
+// token row by TMA.  The MMA thread moves each stage's scales into a ring of
+// TMEM slots with tcgen05.cp and issues the stage's four K = 32 block-scaled
+// MMAs, alternating between two accumulators.  With QOUT the epilogue applies the
 // activation, stores it in bf16 precision and re-encodes it in MXFP8 (a warp
 // holds one 32-column block of each token row).  Otherwise it writes bf16.
 template <int EPI, bool W4, bool QOUT>
@@ -301,7 +308,6 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             // ------------------------------------------------ MMA issuer
             constexpr uint32_t idesc = umma_idesc_mx(128, NT, W4 ? MXF_E2M1 : MXF_E4M3, MXF_E4M3);
-            const uint32_t sf_a0 = tmem_base + C::SF_COL, sf_a1 = sf_a0 + 4, sf_b = sf_a0 + 8;
             uint32_t kc = 0;
             int it = 0;
             bool ok = true;
@@ -320,6 +326,8 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
+                    const uint32_t sf_a0 = tmem_base + C::SF_COL + (kc % C::SF_SLOTS) * C::SF_SLOT;
+                    const uint32_t sf_a1 = sf_a0 + 4, sf_b = sf_a0 + 4 * C::NA;
                     tmem_cp_32x128b_x4(sf_a0, umma_desc_plain(st + C::OFF_SFA, 128));
                     if (C::NA == 2) tmem_cp_32x128b_x4(sf_a1, umma_desc_plain(st + C::OFF_SFA + C::SF_BYTES, 128));
                     tmem_cp_32x128b_x4(sf_b, umma_desc_plain(st + C::OFF_SFB, 128));
@@ -328,10 +336,11 @@ __global__ void __launch_bounds__(192, 1)
                     const uint64_t bx = umma_desc_sw128(st + C::OFF_B);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
-                        const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+                        const uint32_t c = kk & 1;                                 // accumulation chain
+                        const uint32_t acc = (kb > 0 || kk >= C::CHAINS) ? 1u : 0u;  // first step of a chain: overwrite
                         const uint32_t id = idesc | umma_idesc_sf_ids(kk, kk);
-                        umma_mx(d0, a0 + 2 * kk, bx + 2 * kk, id, sf_a0, sf_b, acc);
-                        if (C::NA == 2) umma_mx(d0 + NT, a1 + 2 * kk, bx + 2 * kk, id, sf_a1, sf_b, acc);
+                        umma_mx(d0 + c * C::NA * NT, a0 + 2 * kk, bx + 2 * kk, id, sf_a0, sf_b, acc);
+                        if (C::NA == 2) umma_mx(d0 + (c * C::NA + 1) * NT, a1 + 2 * kk, bx + 2 * kk, id, sf_a1, sf_b, acc);
                     }
                     umma_commit(&empty[s]);
                 }
@@ -357,31 +366,49 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + buf * C::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-            uint32_t g[NT], u[NT];
+            uint32_t g[NT], u[NT], g2[NT], u2[NT];
             tmem_ld_32x32b_x32(taddr, g);
-            if (C::NA == 2) tmem_ld_32x32b_x32(taddr + NT, u);
+            tmem_ld_32x32b_x32(taddr + C::NA * NT, g2);
+            if (C::NA == 2) {
+                tmem_ld_32x32b_x32(taddr + NT, u);
+                tmem_ld_32x32b_x32(taddr + 3 * NT, u2);
+            }
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
+            // the two accumulation chains
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g2[j]));
+                if (C::NA == 2) u[j] = __float_as_uint(__uint_as_float(u[j]) + __uint_as_float(u2[j]));
+            }
             const bool valid = col < args.n_out;
             if (QOUT) {
-                uint8_t* dst = args.out8 + static_cast<size_t>(e.y) * args.ld_out8 + col;
-                uint8_t* dsf = args.out_sf + static_cast<size_t>(e.y) * args.ld_out_sf + (col >> 7) * 16 + ((col >> 5) & 3);
-#pragma unroll 4
+                // the stored (bf16) activation of each token row; then the 32 block maxima (independent warp
+                // reductions, one per row); then the codes.  Lane j writes row j's block scale.
+                float v[NT];
+#pragma unroll
                 for (int j = 0; j < NT; ++j) {
-                    float v = __uint_as_float(g[j]);
-                    if (EPI == EPI_RELU2) v = act_relu2(v);
-                    if (EPI == EPI_SWIGLU) v = act_silu_mul(v, __uint_as_float(u[j]));
-                    v = valid ? __bfloat162float(__float2bfloat16_rn(v)) : 0.f;  // the stored (bf16) activation
-                    const uint32_t amax = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v)));
-                    const int sx = mx_scale_exp(amax, 8);
-                    const uint32_t code = mx_e4m3(v * mx_exp2i(-sx));
-                    if (j < e.z) {
-                        if (valid) dst[static_cast<size_t>(j) * args.ld_out8] = static_cast<uint8_t>(code);
-                        if (lane == 0) dsf[static_cast<size_t>(j) * args.ld_out_sf] = static_cast<uint8_t>(sx + 127);
-                    }
+                    float a = __uint_as_float(g[j]);
+                    if (EPI == EPI_RELU2) a = act_relu2(a);
+                    if (EPI == EPI_SWIGLU) a = act_silu_mul(a, __uint_as_float(u[j]));
+                    v[j] = valid ? __bfloat162float(__float2bfloat16_rn(a)) : 0.f;
                 }
+                uint32_t amax[NT];
+#pragma unroll
+                for (int j = 0; j < NT; ++j) amax[j] = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
+                uint8_t* dst = args.out8 + static_cast<size_t>(e.y) * args.ld_out8 + col;
+                uint32_t my_scale = 0;
+#pragma unroll
+                for (int j = 0; j < NT; ++j) {
+                    const int sx = mx_scale_exp(amax[j], 8);
+                    if (lane == j) my_scale = static_cast<uint32_t>(sx + 127);
+                    if (j < e.z && valid) dst[static_cast<size_t>(j) * args.ld_out8] = static_cast<uint8_t>(mx_e4m3(v[j] * mx_exp2i(-sx)));
+                }
+                if (lane < e.z)
+                    args.out_sf[static_cast<size_t>(e.y + lane) * args.ld_out_sf + (col >> 7) * 16 + ((col >> 5) & 3)] =
+                        static_cast<uint8_t>(my_scale);
             } else if (valid) {
                 __nv_bfloat16* dst = args.out + static_cast<size_t>(e.y) * args.ld_out + col;
 #pragma unroll
