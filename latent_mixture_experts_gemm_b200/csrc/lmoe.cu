@@ -186,6 +186,12 @@ const char* kPhaseNames[PH_COUNT] = {"router_proj_gemm", "topk_softmax", "dispat
                                      "expert_up_stream", "expert_down_gemm", "expert_down_stream", "combine",
                                      "up_proj_gemm", "shared_expert"};
 
+template <int EPI>
+bool set_pair_attr() {
+    return cudaFuncSetAttribute(tc_gemm_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GemmPairCfg::SMEM_BYTES) == cudaSuccess;
+}
+
 template <int BN, int EPI>
 bool set_smem_attr() {
     return cudaFuncSetAttribute(tc_gemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -196,6 +202,26 @@ bool set_smem_attr() {
 // while its predecessor in the stream drains; every kernel of the layer waits
 // for its predecessor first thing (pdl_begin), so results are unchanged.
 bool g_use_pdl = true;
+
+// The same for a kernel of CTA pairs: clusters of 2 along x (grid.x even).
+template <typename... P, typename... A>
+void launch_pairs(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = g_use_pdl ? 2 : 1;
+    cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 template <typename... P, typename... A>
 void launch(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, A&&... args) {
@@ -226,6 +252,11 @@ bool set_mx_attr() {
 
 bool set_all_smem_attrs() {
     bool ok = true;
+    ok &= set_pair_attr<EPI_BF16>();
+    ok &= set_pair_attr<EPI_RELU2>();
+    ok &= set_pair_attr<EPI_SWIGLU>();
+    ok &= set_pair_attr<EPI_RESID>();
+    ok &= set_pair_attr<EPI_PROJ_ROUTER>();
     ok &= set_mx_attr<EPI_BF16, false, true>();
     ok &= set_mx_attr<EPI_RELU2, false, true>();
     ok &= set_mx_attr<EPI_SWIGLU, false, true>();
@@ -341,6 +372,14 @@ template <int BN, int EPI>
 void launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args, int grid,
                  cudaStream_t s) {
     launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, args);
+}
+
+// CTA-pair GEMM: `pair_tiles` (or, for a device-built list, an upper bound) pair tiles on up to num_sms / 2 pairs.
+template <int EPI>
+void launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args,
+                      int pair_tiles, int num_sms, cudaStream_t s) {
+    const int pairs = std::max(1, std::min(num_sms / 2, pair_tiles));
+    launch_pairs(tc_gemm_pair_kernel<EPI>, 2 * pairs, 192, GemmPairCfg::SMEM_BYTES, s, a, b, b2, args);
 }
 
 template <int EPI, bool W4, bool QOUT>
@@ -581,8 +620,8 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
             if (big) {
                 a.n_tiles0 = fused ? (L + 255) / 256 : 0;
                 a.n_tiles = a.n_tiles0 + (nt + 255) / 256;
-                launch_gemm<256, EPI_PROJ_ROUTER>(A, fused ? h->wdown256 : h->wr256, h->wr256, a,
-                                                  std::min(h->num_sms, m_tiles * a.n_tiles), s);
+                launch_gemm_pair<EPI_PROJ_ROUTER>(A, fused ? h->wdown128 : h->wr128, h->wr128, a,
+                                                  (T + 255) / 256 * a.n_tiles, h->num_sms, s);
             } else {
                 a.n_tiles0 = fused ? (L + 63) / 64 : 0;
                 a.n_tiles = a.n_tiles0 + (nt + 63) / 64;
@@ -644,6 +683,9 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     }
     // ---------------------------------------------------------------- expert up (+ activation)
     if (need_tc) {
+        // Grouped GEMMs stay on single-CTA 128-row tiles: with a few hundred rows per expert, 256-row pair
+        // tiles would need a second launch for each expert's remainder, which reads the expert's weights
+        // from HBM a second time.
         PhaseScope ps(h, PH_UP_TC, s, 1);
         GemmArgs a = base;
         a.K = L;
@@ -779,7 +821,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.ld_resid = d;
         if (m_tiles * ((d + 255) / 256) >= h->num_sms) {
             a.n_tiles = (d + 255) / 256;
-            launch_gemm<256, EPI_RESID>(h->a_yl, h->wup256, h->wup256, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
+            launch_gemm_pair<EPI_RESID>(h->a_yl, h->wup128, h->wup128, a, (T + 255) / 256 * a.n_tiles, h->num_sms, s);
         } else {
             a.n_tiles = (d + 63) / 64;
             launch_gemm<64, EPI_RESID>(h->a_yl, h->wup64, h->wup64, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
@@ -1099,7 +1141,8 @@ int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, 
     const int m_tiles = (M + 127) / 128;
     const bool big = static_cast<long long>(m_tiles) * ((N + 255) / 256) >= sms;
     CUtensorMap ma, mb;
-    if (!make_map(&ma, A, M, K, K, 128) || !make_map(&mb, B, N, K, K, big ? 256 : 64)) return LMOE_ERR_CUDA;
+    // large problems run on CTA pairs (256 x 256 tiles; each CTA loads 128 of the B rows)
+    if (!make_map(&ma, A, M, K, K, 128) || !make_map(&mb, B, N, K, K, big ? 128 : 64)) return LMOE_ERR_CUDA;
     GemmArgs a{};
     a.M = M;
     a.K = K;
@@ -1111,7 +1154,8 @@ int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (big) {
         a.n_tiles = (N + 255) / 256;
-        launch_gemm<256, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);
+        launch_gemm_pair<EPI_BF16>(ma, mb, mb, a, static_cast<int>(std::min<long long>(sms, (M + 255LL) / 256 * a.n_tiles)),
+                                   sms, s);
     } else {
         a.n_tiles = (N + 63) / 64;
         launch_gemm<64, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);

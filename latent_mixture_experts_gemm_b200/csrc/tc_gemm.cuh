@@ -131,6 +131,99 @@ __device__ __forceinline__ void epi_load_resid(const GemmArgs& a, const TileJob&
     }
 }
 
+// Epilogue of one tile for the 128 accumulator rows of this CTA: warp w (w % 4 = quad) reads TMEM
+// lanes 32*quad .. +31 at `tbase`, applies the fused epilogue and stores row `row` (when row_ok).
+// For EPI_RESID, `rs` holds the residual of the first 64 columns on entry.
+template <int BN, int EPI>
+__device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const TileJob& j, bool row_ok, size_t row,
+                                                    uint32_t tbase, uint4 (&rs)[8]) {
+    if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 2; c += 32) {
+            uint32_t g[32], u[32];
+            tmem_ld_32x32b_x32(tbase + c, g);
+            tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
+            tmem_ld_wait();
+            const int col = j.col0 + c;
+            if (row_ok && col < args.N0) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_bf16x2(act_silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                        act_silu_mul(__uint_as_float(g[2 * i + 1]),
+                                                     __uint_as_float(u[2 * i + 1])));
+                uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+            }
+        }
+    } else {
+        // 64 accumulator columns per tcgen05 wait
+#pragma unroll 1
+        for (int pc = 0; pc < BN; pc += 64) {
+            uint32_t v2[2][32];
+            tmem_ld_32x32b_x32(tbase + pc, v2[0]);
+            tmem_ld_32x32b_x32(tbase + pc + 32, v2[1]);
+            uint4 rs_now[8];
+            if (EPI == EPI_RESID) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) rs_now[i] = rs[i];
+                if (pc + 64 < BN) epi_load_resid<BN>(args, j, pc + 64, row_ok, row, rs);
+            }
+            tmem_ld_wait();
+            if (!row_ok) continue;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t(&v)[32] = v2[h];
+                const int col = j.col0 + pc + 32 * h;
+                if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
+                    float* dst = args.out1 + row * args.ld1 + col;
+                    if (col + 32 <= args.N1) {
+                        float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                                __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (col + i < args.N1) dst[i] = __uint_as_float(v[i]);
+                    }
+                    continue;
+                }
+                if (col >= args.N0) continue;
+                float f[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+                if (EPI == EPI_RELU2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
+                }
+                if (EPI == EPI_RESID) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint4 q = rs_now[4 * h + i];
+                        f[8 * i + 0] += bf16lo(q.x);
+                        f[8 * i + 1] += bf16hi(q.x);
+                        f[8 * i + 2] += bf16lo(q.y);
+                        f[8 * i + 3] += bf16hi(q.y);
+                        f[8 * i + 4] += bf16lo(q.z);
+                        f[8 * i + 5] += bf16hi(q.z);
+                        f[8 * i + 6] += bf16lo(q.w);
+                        f[8 * i + 7] += bf16hi(q.w);
+                    }
+                }
+                uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    dst[i] = make_uint4(pack_bf16x2(f[8 * i + 0], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
+                                        pack_bf16x2(f[8 * i + 4], f[8 * i + 5]), pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
+            }
+        }
+    }
+}
+
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -277,91 +370,7 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quad * 32) << 16);
-            if (EPI == EPI_SWIGLU) {
-#pragma unroll 1
-                for (int c = 0; c < BN / 2; c += 32) {
-                    uint32_t g[32], u[32];
-                    tmem_ld_32x32b_x32(tbase + c, g);
-                    tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
-                    tmem_ld_wait();
-                    const int col = j.col0 + c;
-                    if (row_ok && col < args.N0) {
-                        uint32_t pk[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16x2(act_silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                                act_silu_mul(__uint_as_float(g[2 * i + 1]),
-                                                             __uint_as_float(u[2 * i + 1])));
-                        uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                    }
-                }
-            } else {
-                // 64 accumulator columns per tcgen05 wait
-#pragma unroll 1
-                for (int pc = 0; pc < BN; pc += 64) {
-                    uint32_t v2[2][32];
-                    tmem_ld_32x32b_x32(tbase + pc, v2[0]);
-                    tmem_ld_32x32b_x32(tbase + pc + 32, v2[1]);
-                    uint4 rs_now[8];
-                    if (EPI == EPI_RESID) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) rs_now[i] = rs[i];
-                        if (pc + 64 < BN) epi_load_resid<BN>(args, j, pc + 64, row_ok, row, rs);
-                    }
-                    tmem_ld_wait();
-                    if (!row_ok) continue;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint32_t(&v)[32] = v2[h];
-                        const int col = j.col0 + pc + 32 * h;
-                        if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
-                            float* dst = args.out1 + row * args.ld1 + col;
-                            if (col + 32 <= args.N1) {
-                                float4* d4 = reinterpret_cast<float4*>(dst);
-#pragma unroll
-                                for (int i = 0; i < 8; ++i)
-                                    d4[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                                        __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
-                            } else {
-#pragma unroll
-                                for (int i = 0; i < 32; ++i)
-                                    if (col + i < args.N1) dst[i] = __uint_as_float(v[i]);
-                            }
-                            continue;
-                        }
-                        if (col >= args.N0) continue;
-                        float f[32];
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
-                        if (EPI == EPI_RELU2) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
-                        }
-                        if (EPI == EPI_RESID) {
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const uint4 q = rs_now[4 * h + i];
-                                f[8 * i + 0] += bf16lo(q.x);
-                                f[8 * i + 1] += bf16hi(q.x);
-                                f[8 * i + 2] += bf16lo(q.y);
-                                f[8 * i + 3] += bf16hi(q.y);
-                                f[8 * i + 4] += bf16lo(q.z);
-                                f[8 * i + 5] += bf16hi(q.z);
-                                f[8 * i + 6] += bf16lo(q.w);
-                                f[8 * i + 7] += bf16hi(q.w);
-                            }
-                        }
-                        uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
-#pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pack_bf16x2(f[8 * i + 0], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
-                                                pack_bf16x2(f[8 * i + 4], f[8 * i + 5]), pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
-                    }
-                }
-            }
+            gemm_epilogue_store<BN, EPI>(args, j, row_ok, row, tbase, rs);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
@@ -374,6 +383,238 @@ __global__ void __launch_bounds__(192, 1)
     if (warp == 1) {
         __syncwarp();
         tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+// ============================================================================ CTA-pair GEMM
+// The same GEMM on pairs of CTAs (a cluster of 2) issuing cta_group::2 MMAs:
+// a pair tile is 256 rows x 256 columns.  Each CTA loads its own 128 A rows
+// and half of the tile's B rows (128), so an SM brings in 32 KB per 64-deep K
+// stage instead of 48 KB for the same multiply-adds: the operand bytes per MAC
+// fall by a third, which is what bounds the single-CTA kernel (its operand
+// loads are latency-bound).  One thread of the first CTA issues the MMAs; each
+// CTA's tensor memory receives its own 128 rows of the 256 x 256 accumulator
+// and its own epilogue stores them.
+//
+// Synchronisation of the pair:
+//   full[s]   first CTA only: its producer posts the stage's bytes of both
+//             CTAs; both CTAs' copies complete on it (its cluster address);
+//   empty[s]  both CTAs: the MMA thread's commit arrives on both (multicast);
+//   tfull[b]  both CTAs: the commit after a tile's last stage (multicast);
+//   tempty[b] first CTA only: the 8 epilogue warps of both CTAs arrive on it.
+// Every wait is bounded, so each thread reaches the cluster barrier before the
+// CTAs free their tensor memory, even after a timeout.
+//
+// Tile maps: dense -- ceil(M/256) x n_tiles; grouped -- the pair list
+// (expert, first row, rows <= 256).  For EPI_SWIGLU the first CTA loads the
+// gate rows and the second the matching up rows, so accumulator columns
+// [0,128) are gate and [128,256) up, as in the single-CTA kernel's layout.
+struct GemmPairCfg {
+    static constexpr int BN = 256;
+    static constexpr int BK = 64;
+    static constexpr int A_BYTES = 128 * BK * 2;       // this CTA's 128 A rows
+    static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the B rows
+    static constexpr int STAGES = 6;
+    static constexpr int TMEM_COLS = 2 * BN;
+    static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 + 256;
+};
+
+template <int EPI>
+__device__ __forceinline__ void tile_job_pair(const GemmArgs& a, int t, int rank, TileJob& j) {
+    const int mt = t / a.n_tiles, nt = t % a.n_tiles;
+    int row0, rows;
+    j.seg = 0;
+    j.b_row1 = 0;
+    if (a.mt_list != nullptr) {
+        const int4 e = a.mt_list[mt];
+        row0 = e.y;
+        rows = e.z;
+        const int base = e.x * a.b_rows_per_expert;
+        if (EPI == EPI_SWIGLU) {
+            j.col0 = nt * 128;
+            j.b_row0 = base + j.col0 + (rank ? a.up_offset : 0);
+        } else {
+            j.col0 = nt * 256;
+            j.b_row0 = base + j.col0 + 128 * rank;
+        }
+    } else {
+        row0 = mt * 256;
+        rows = min(256, a.M - row0);
+        if (EPI == EPI_PROJ_ROUTER && nt >= a.n_tiles0) {
+            j.seg = 1;
+            j.col0 = (nt - a.n_tiles0) * 256;
+        } else {
+            j.col0 = (EPI == EPI_SWIGLU) ? nt * 128 : nt * 256;
+        }
+        j.b_row0 = (EPI == EPI_SWIGLU) ? j.col0 + (rank ? a.up_offset : 0) : j.col0 + 128 * rank;
+    }
+    j.a_row0 = row0 + 128 * rank;
+    j.rows = max(0, min(128, rows - 128 * rank));
+}
+
+__device__ __forceinline__ int total_tiles_pair(const GemmArgs& a) {
+    if (a.mt_list != nullptr) return (*a.mt_count) * a.n_tiles;
+    return ((a.M + 255) / 256) * a.n_tiles;
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(192, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
+    pdl_begin();
+    using C = GemmPairCfg;
+    constexpr int BN = C::BN;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::STAGES * C::A_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+    uint64_t* empty = full + C::STAGES;
+    uint64_t* tfull = empty + C::STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* mma_done = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pid = static_cast<int>(blockIdx.x >> 1), npid = static_cast<int>(gridDim.x >> 1);
+    const int ntiles = total_tiles_pair(args);
+    if (pid >= ntiles) return;  // both CTAs of the pair leave together, before any pair set-up
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 8);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tmA);
+        tma_prefetch_desc(&tmB);
+        if (EPI == EPI_PROJ_ROUTER) tma_prefetch_desc(&tmB2);
+    }
+    if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers initialised before any copy or arrive reaches them
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int nkb = args.K / C::BK;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ------------------------------------------------ TMA producer (both CTAs)
+            uint32_t kc = 0;
+            uint32_t last_parity[C::STAGES];
+            bool issued[C::STAGES];
+            for (int s = 0; s < C::STAGES; ++s) issued[s] = false, last_parity[s] = 0;
+            bool ok = true;
+            for (int t = pid; t < ntiles && ok; t += npid) {
+                TileJob j;
+                tile_job_pair<EPI>(args, t, static_cast<int>(rank), j);
+                const CUtensorMap* bmap = (EPI == EPI_PROJ_ROUTER && j.seg == 1) ? &tmB2 : &tmB;
+                for (int kb = 0; kb < nkb; ++kb, ++kc) {
+                    const int s = kc % C::STAGES;
+                    const uint32_t ph = (kc / C::STAGES) & 1;
+                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.err, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::A_BYTES + C::B_BYTES));
+                    const uint32_t fb = mapa_shared(&full[s], 0);
+                    tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, fb, kb * C::BK, j.a_row0);
+                    tma_load_2d_pair(sB + s * C::B_BYTES, bmap, fb, kb * C::BK, j.b_row0);
+                    issued[s] = true;
+                    last_parity[s] = ph;
+                }
+            }
+            // The first CTA's full barriers count both CTAs' bytes: waiting for the last phase of each
+            // stage there means no copy of either CTA is still in flight.  The second CTA leaves only
+            // after the final cluster barrier, which the first passes after this drain.
+            if (rank == 0)
+                for (int s = 0; s < C::STAGES; ++s)
+                    if (issued[s]) {
+                        int no_abort = 0;
+                        mbar_wait_bounded(&full[s], last_parity[s], &no_abort, args.err, drain_ns(args));
+                    }
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && rank == 0) {
+            // ------------------------------------------------ MMA issuer (first CTA)
+            constexpr uint32_t idesc = umma_idesc_bf16(256, BN);
+            uint32_t kc = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = pid; t < ntiles && ok; t += npid, ++it) {
+                const int buf = it & 1;
+                const uint32_t use = (it >> 1) & 1;
+                if (!mbar_wait_bounded(&tempty[buf], use ^ 1, abort_flag, args.err, args.timeout_ns)) break;
+                tc_fence_after();
+                const uint32_t dtmem = tmem_base + buf * BN;
+                for (int kb = 0; kb < nkb; ++kb, ++kc) {
+                    const int s = kc % C::STAGES;
+                    const uint32_t ph = (kc / C::STAGES) & 1;
+                    if (!mbar_wait_bounded(&full[s], ph, abort_flag, args.err, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint64_t ad = umma_desc_sw128(smem_u32(sA + s * C::A_BYTES));
+                    const uint64_t bd = umma_desc_sw128(smem_u32(sB + s * C::B_BYTES));
+#pragma unroll
+                    for (int kk = 0; kk < C::BK / 16; ++kk)
+                        umma_bf16_pair(dtmem, ad + 2 * kk, bd + 2 * kk, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit_pair_mc(&empty[s], 0x3);
+                }
+                if (ok) umma_commit_pair_mc(&tfull[buf], 0x3);
+            }
+            // every MMA of the pair done before the tensor memory of either CTA is freed
+            umma_commit_pair(mma_done);
+            int no_abort = 0;
+            mbar_wait_bounded(mma_done, 0, &no_abort, args.err, drain_ns(args));
+        }
+    } else {
+        // ---------------------------------------------------- epilogue (both CTAs, own 128 rows)
+        const int quad = warp & 3;
+        const int row_in_tile = quad * 32 + lane;
+        int it = 0;
+        for (int t = pid; t < ntiles; t += npid, ++it) {
+            TileJob j;
+            tile_job_pair<EPI>(args, t, static_cast<int>(rank), j);
+            const int buf = it & 1;
+            const uint32_t use = (it >> 1) & 1;
+            const bool row_ok = row_in_tile < j.rows;
+            const size_t row = static_cast<size_t>(j.a_row0) + row_in_tile;
+            uint4 rs[8];
+            if (EPI == EPI_RESID) epi_load_resid<BN>(args, j, 0, row_ok, row, rs);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(&tfull[buf], use, abort_flag, args.err, args.timeout_ns) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quad * 32) << 16);
+            gemm_epilogue_store<BN, EPI>(args, j, row_ok, row, tbase, rs);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty[buf], 0));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    tc_fence_after();
+    if (warp == 1) {
+        __syncwarp();
+        tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
     }
 }
 

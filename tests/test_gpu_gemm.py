@@ -1,5 +1,6 @@
 """The tcgen05 GEMM kernel alone (C = A B^T, bf16 in/out, fp32 accumulate) against an fp64 matmul
-of the same bf16 inputs, on shapes that exercise partial M tiles, both column-tile widths and long K."""
+of the same bf16 inputs, on shapes that exercise partial M tiles, both column-tile widths, long K and the
+CTA-pair kernel (large shapes)."""
 import numpy as np
 import pytest
 import torch
@@ -11,7 +12,10 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("M,N,K", [(128, 64, 64), (1, 64, 64), (37, 512, 128), (200, 192, 320), (1000, 256, 1024),
-                                   (4096, 1024, 512), (8192, 4096, 1024), (300, 64, 4096)])
+                                   (4096, 1024, 512), (8192, 4096, 1024), (300, 64, 4096),
+                                   # CTA-pair tiles (256 x 256): a ragged last pair (the second CTA gets 104 rows),
+                                   # and a ragged last column tile (the second CTA's B rows are all past N)
+                                   (1000, 8192, 256), (2500, 2368, 320)])
 def test_gemm_matches_fp64(M, N, K):
     g = torch.Generator().manual_seed(M * 31 + N * 7 + K)
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)

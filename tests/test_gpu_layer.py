@@ -37,6 +37,10 @@ CASES = {
     "medium_standard_moe_shared": MEDIUM.with_(latent=512, has_proj=0, shared_m=192, seed=36),
     "tiny_decode_shared_swiglu": synth.WORKLOADS["tiny"].with_(tokens=9, act="swiglu", shared_m=64, seed=37),
     "tiny_decode_latent_router": synth.WORKLOADS["tiny"].with_(tokens=12, latent_router=1, seed=38),
+    # hundreds of rows per expert (several full 128-row tiles and a ragged one), plain and gated with skew
+    "medium_500_rows_per_expert": MEDIUM.with_(tokens=2000, n_ffn=16, top_k=4, seed=40),
+    "medium_300_rows_per_expert_swiglu_skew": MEDIUM.with_(tokens=1300, n_ffn=16, top_k=4, act="swiglu", zipf=1.1,
+                                                           n_zero=1, seed=41),
     "nemotron_decode": synth.WORKLOADS["nemotron_decode"],
     "std_decode": synth.WORKLOADS["std_decode"],
 }
