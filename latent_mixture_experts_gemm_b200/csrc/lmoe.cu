@@ -649,7 +649,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     // ---------------------------------------------------------------- top-K' + softmax
     {
         PhaseScope ps(h, PH_TOPK, s, 1);
-        const dim3 grid((T + 7) / 8), block(256);
+        const dim3 grid((T + 3) / 4), block(128);  // one warp per token, 4 per block (few tokens: more SMs)
 #define LMOE_TOPK(N) launch(topk_softmax_kernel<N>, grid, block, 0, s, logits, p.ld_logits, bias, T, nt, K, idx, wts)
         if (npl <= 1) LMOE_TOPK(1);
         else if (npl <= 2) LMOE_TOPK(2);

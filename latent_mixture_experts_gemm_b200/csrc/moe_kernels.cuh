@@ -78,12 +78,20 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ row, co
                                                int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     const int lane = threadIdx.x & 31;
     const uint32_t below = (1u << lane) - 1u;
+    // all loads first, so that they are in flight together (the row sits in L2: one round trip, not NPL)
+    float lv[NPL], bv[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+        const int e = lane + 32 * i;
+        lv[i] = e < n_tot ? __ldg(row + e) : 0.0f;
+        bv[i] = (bias != nullptr && e < n_tot) ? __ldg(bias + e) : 0.0f;
+    }
     uint32_t key[NPL];
     uint32_t lmax = 0;
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        key[i] = e < n_tot ? order_key(row[e] + (bias != nullptr ? bias[e] : 0.0f)) : 0u;  // 0: no expert
+        key[i] = e < n_tot ? order_key(lv[i] + bv[i]) : 0u;  // 0: no expert
         lmax = max(lmax, key[i]);
     }
     // K'-th largest lane maximum (descending bitonic sort of the 32 maxima by key)
@@ -191,11 +199,11 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ row, co
 }
 
 template <int NPL>
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits, int ld,
+__global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restrict__ logits, int ld,
                                                            const float* __restrict__ bias, int T, int n_tot, int K,
                                                            int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
     pdl_begin();
-    __shared__ uint32_t s_key[8][64], s_id[8][64];
+    __shared__ uint32_t s_key[4][64], s_id[4][64];
     const int warp = threadIdx.x >> 5;
     const int t = blockIdx.x * (blockDim.x >> 5) + warp;
     if (t >= T) return;
