@@ -368,18 +368,25 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
     return 2;
 }
 
+// `out` (optional): TMA map of the bf16 output (box 32 rows x 64 columns, 128-byte swizzle); the epilogue
+// then stores whole 32-row blocks with TMA (BN = 256).  Without it every thread stores its own row.
 template <int BN, int EPI>
 void launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args, int grid,
-                 cudaStream_t s) {
-    launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, args);
+                 cudaStream_t s, const CUtensorMap* out = nullptr) {
+    GemmArgs g = args;
+    g.tma_store = (out != nullptr && BN == 256) ? 1 : 0;
+    launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, out != nullptr ? *out : a, g);
 }
 
 // CTA-pair GEMM: `pair_tiles` (or, for a device-built list, an upper bound) pair tiles on up to num_sms / 2 pairs.
 template <int EPI>
 void launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args,
-                      int pair_tiles, int num_sms, cudaStream_t s) {
+                      int pair_tiles, int num_sms, cudaStream_t s, const CUtensorMap* out = nullptr) {
     const int pairs = std::max(1, std::min(num_sms / 2, pair_tiles));
-    launch_pairs(tc_gemm_pair_kernel<EPI>, 2 * pairs, 192, GemmPairCfg::SMEM_BYTES, s, a, b, b2, args);
+    GemmArgs g = args;
+    g.tma_store = out != nullptr ? 1 : 0;
+    launch_pairs(tc_gemm_pair_kernel<EPI>, 2 * pairs, 192, GemmPairCfg::SMEM_BYTES, s, a, b, b2,
+                 out != nullptr ? *out : a, g);
 }
 
 template <int EPI, bool W4, bool QOUT>
@@ -429,6 +436,8 @@ struct lmoe_handle {
     CUtensorMap ws1_64{}, ws1_256{}, ws2_64{}, ws2_256{}, ws1_128{}, ws2_128{}, a_hs{}, hs16{}, hs32{};
     // block-scaled experts: weight codes (128 x 128 boxes) and the MXFP8 token operands with their scales
     CUtensorMap w1q{}, w2q{}, rows8{}, rows_sf{}, h8{}, h_sf{};
+    // TMA store maps of bf16 GEMM outputs (32-row x 64-column boxes): hidden rows, expert outputs, z
+    CUtensorMap o_h{}, o_rows{}, o_z{};
     cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     // profiling
@@ -621,7 +630,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
                 a.n_tiles0 = fused ? (L + 255) / 256 : 0;
                 a.n_tiles = a.n_tiles0 + (nt + 255) / 256;
                 launch_gemm_pair<EPI_PROJ_ROUTER>(A, fused ? h->wdown128 : h->wr128, h->wr128, a,
-                                                  (T + 255) / 256 * a.n_tiles, h->num_sms, s);
+                                                  (T + 255) / 256 * a.n_tiles, h->num_sms, s, fused ? &h->o_z : nullptr);
             } else {
                 a.n_tiles0 = fused ? (L + 63) / 64 : 0;
                 a.n_tiles = a.n_tiles0 + (nt + 63) / 64;
@@ -698,13 +707,13 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.ld0 = m;
         if (c.act == LMOE_ACT_SWIGLU) {
             a.n_tiles = (m + 127) / 128;
-            launch_gemm<256, EPI_SWIGLU>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
+            launch_gemm<256, EPI_SWIGLU>(h->a_rows, h->w1, h->w1, a, h->num_sms, s, &h->o_h);
         } else if (c.act == LMOE_ACT_RELU2) {
             a.n_tiles = (m + 255) / 256;
-            launch_gemm<256, EPI_RELU2>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
+            launch_gemm<256, EPI_RELU2>(h->a_rows, h->w1, h->w1, a, h->num_sms, s, &h->o_h);
         } else {
             a.n_tiles = (m + 255) / 256;
-            launch_gemm<256, EPI_BF16>(h->a_rows, h->w1, h->w1, a, h->num_sms, s);
+            launch_gemm<256, EPI_BF16>(h->a_rows, h->w1, h->w1, a, h->num_sms, s, &h->o_h);
         }
     }
     if (mx) {
@@ -756,7 +765,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.out0 = rows;
         a.ld0 = L;
         a.n_tiles = (L + 255) / 256;
-        launch_gemm<256, EPI_BF16>(h->a_h, h->w2, h->w2, a, h->num_sms, s);
+        launch_gemm<256, EPI_BF16>(h->a_h, h->w2, h->w2, a, h->num_sms, s, &h->o_rows);
     }
     if (mx) {
         PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
@@ -821,7 +830,10 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.ld_resid = d;
         if (m_tiles * ((d + 255) / 256) >= h->num_sms) {
             a.n_tiles = (d + 255) / 256;
-            launch_gemm_pair<EPI_RESID>(h->a_yl, h->wup128, h->wup128, a, (T + 255) / 256 * a.n_tiles, h->num_sms, s);
+            CUtensorMap o_y;
+            if (!make_map(&o_y, y, T, d, d, 32)) return LMOE_ERR_CUDA;
+            launch_gemm_pair<EPI_RESID>(h->a_yl, h->wup128, h->wup128, a, (T + 255) / 256 * a.n_tiles, h->num_sms, s,
+                                        &o_y);
         } else {
             a.n_tiles = (d + 63) / 64;
             launch_gemm<64, EPI_RESID>(h->a_yl, h->wup64, h->wup64, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
@@ -943,6 +955,9 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     }
     ok &= make_map(&h->a_rows, h->at<void>(p.rows), R, L, L, 128);
     ok &= make_map(&h->a_h, h->at<void>(p.hbuf), R, m, m, 128);
+    ok &= make_map(&h->o_h, h->at<void>(p.hbuf), R, m, m, 32);
+    ok &= make_map(&h->o_rows, h->at<void>(p.rows), R, L, L, 32);
+    if (c.has_proj) ok &= make_map(&h->o_z, h->at<void>(p.z), c.max_tokens, L, L, 32);
     ok &= make_map(&h->rows16, h->at<void>(p.rows), R, L, L, 16);
     ok &= make_map(&h->rows32, h->at<void>(p.rows), R, L, L, 32);
     ok &= make_map(&h->h16, h->at<void>(p.hbuf), R, m, m, 16);
@@ -1142,7 +1157,9 @@ int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, 
     const bool big = static_cast<long long>(m_tiles) * ((N + 255) / 256) >= sms;
     CUtensorMap ma, mb;
     // large problems run on CTA pairs (256 x 256 tiles; each CTA loads 128 of the B rows)
-    if (!make_map(&ma, A, M, K, K, 128) || !make_map(&mb, B, N, K, K, big ? 128 : 64)) return LMOE_ERR_CUDA;
+    CUtensorMap mc;
+    if (!make_map(&ma, A, M, K, K, 128) || !make_map(&mb, B, N, K, K, big ? 128 : 64) || !make_map(&mc, C, M, N, N, 32))
+        return LMOE_ERR_CUDA;
     GemmArgs a{};
     a.M = M;
     a.K = K;
@@ -1155,7 +1172,7 @@ int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, 
     if (big) {
         a.n_tiles = (N + 255) / 256;
         launch_gemm_pair<EPI_BF16>(ma, mb, mb, a, static_cast<int>(std::min<long long>(sms, (M + 255LL) / 256 * a.n_tiles)),
-                                   sms, s);
+                                   sms, s, &mc);
     } else {
         a.n_tiles = (N + 63) / 64;
         launch_gemm<64, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);

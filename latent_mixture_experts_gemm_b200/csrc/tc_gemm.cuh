@@ -46,9 +46,15 @@ struct GemmArgs {
     int ld1;
     const __nv_bfloat16* resid;
     int ld_resid;
+    int tma_store;         // 1: bf16 out0 rows leave through shared-memory staging and TMA stores (BN = 256)
     int* err;
     unsigned long long timeout_ns;
 };
+
+// Output staging for TMA stores: each epilogue warp owns two 4 KB buffers of 32 rows x 64 bf16
+// columns.  Row r sits at r * 128 bytes with its 16-byte chunk c at position c ^ (r % 8): the
+// 128-byte swizzle of the output map (buffers are 1024-byte aligned).
+constexpr int OUT_STAGE_BYTES = 4 * 2 * 32 * 128;
 
 template <int BN>
 struct GemmCfg {
@@ -58,7 +64,8 @@ struct GemmCfg {
     static constexpr int B_BYTES = BN * BK * 2;
     static constexpr int STAGES = (BN >= 256) ? 4 : (BN >= 128 ? 6 : 8);
     static constexpr int TMEM_COLS = 2 * BN;  // power of two for BN in {64,128,256}
-    static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+    static constexpr int SMEM_BYTES =
+        STAGES * (A_BYTES + B_BYTES) + OUT_STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 };
 
 struct TileJob {
@@ -131,13 +138,45 @@ __device__ __forceinline__ void epi_load_resid(const GemmArgs& a, const TileJob&
     }
 }
 
+__device__ __forceinline__ void stage_row64(uint8_t* buf, int lane, const uint4 (&q)[8]) {
+    uint8_t* rowp = buf + lane * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(rowp + ((c ^ (lane & 7)) << 4)) = q[c];
+}
+
+// Hand this warp's staged 32 x 64 block to the TMA unit once every lane has written it.
+__device__ __forceinline__ void store_block64(const CUtensorMap* map, const uint8_t* buf, int lane, int col, int row0) {
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+        tma_store_2d(map, buf, col, row0);
+        bulk_commit_group();
+    }
+}
+
+// Before rewriting a staging buffer: the store issued from it one block earlier has read it.
+__device__ __forceinline__ void staging_acquire(int lane) {
+    if (lane == 0) bulk_wait_group_read<1>();
+    __syncwarp();
+}
+
+__device__ __forceinline__ uint4 pack8(const float* f) {
+    return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+}
+
 // Epilogue of one tile for the 128 accumulator rows of this CTA: warp w (w % 4 = quad) reads TMEM
 // lanes 32*quad .. +31 at `tbase`, applies the fused epilogue and stores row `row` (when row_ok).
-// For EPI_RESID, `rs` holds the residual of the first 64 columns on entry.
+// For EPI_RESID, `rs` holds the residual of the first 64 columns on entry.  With `tma_rows` (all
+// 32 rows of this warp valid, and a bf16 output map), the bf16 outputs go out in 64-column blocks
+// through this warp's staging buffers `sout` and TMA stores to `tmOut` at rows warp_row0 ..;
+// otherwise every thread stores its own row.
 template <int BN, int EPI>
 __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const TileJob& j, bool row_ok, size_t row,
-                                                    uint32_t tbase, uint4 (&rs)[8]) {
+                                                    uint32_t tbase, uint4 (&rs)[8], const CUtensorMap* tmOut,
+                                                    uint8_t* sout, uint32_t& sbuf, bool tma_rows, int warp_row0,
+                                                    int lane) {
     if (EPI == EPI_SWIGLU) {
+        uint32_t pk_prev[16];
 #pragma unroll 1
         for (int c = 0; c < BN / 2; c += 32) {
             uint32_t g[32], u[32];
@@ -145,17 +184,32 @@ __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const 
             tmem_ld_32x32b_x32(tbase + BN / 2 + c, u);
             tmem_ld_wait();
             const int col = j.col0 + c;
-            if (row_ok && col < args.N0) {
-                uint32_t pk[16];
+            uint32_t pk[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(act_silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                                        act_silu_mul(__uint_as_float(g[2 * i + 1]),
-                                                     __uint_as_float(u[2 * i + 1])));
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pack_bf16x2(act_silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                                    act_silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+            if (tma_rows) {
+                if ((c & 32) == 0) {  // first half of a 64-column block
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pk_prev[i] = pk[i];
+                } else if (col - 32 < args.N0) {
+                    uint4 q[8];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        q[i] = make_uint4(pk_prev[4 * i], pk_prev[4 * i + 1], pk_prev[4 * i + 2], pk_prev[4 * i + 3]);
+                        q[4 + i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
+                    staging_acquire(lane);
+                    uint8_t* buf = sout + sbuf * 4096;
+                    stage_row64(buf, lane, q);
+                    store_block64(tmOut, buf, lane, col - 32, warp_row0);
+                    sbuf ^= 1u;
+                }
+            } else if (row_ok && col < args.N0) {
                 uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
             }
         }
     } else {
@@ -172,14 +226,15 @@ __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const 
                 if (pc + 64 < BN) epi_load_resid<BN>(args, j, pc + 64, row_ok, row, rs);
             }
             tmem_ld_wait();
-            if (!row_ok) continue;
+            if (!row_ok) continue;  // (with tma_rows every lane's row is valid: no divergence)
+            const int col = j.col0 + pc;
+            if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const uint32_t(&v)[32] = v2[h];
-                const int col = j.col0 + pc + 32 * h;
-                if (EPI == EPI_PROJ_ROUTER && j.seg == 1) {
-                    float* dst = args.out1 + row * args.ld1 + col;
-                    if (col + 32 <= args.N1) {
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t(&v)[32] = v2[h];
+                    const int ch = col + 32 * h;
+                    float* dst = args.out1 + row * args.ld1 + ch;
+                    if (ch + 32 <= args.N1) {
                         float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
@@ -188,14 +243,18 @@ __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const 
                     } else {
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            if (col + i < args.N1) dst[i] = __uint_as_float(v[i]);
+                            if (ch + i < args.N1) dst[i] = __uint_as_float(v[i]);
                     }
-                    continue;
                 }
-                if (col >= args.N0) continue;
+                continue;
+            }
+            if (col >= args.N0) continue;
+            uint4 q[8];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
                 float f[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
+                for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v2[h][i]);
                 if (EPI == EPI_RELU2) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
@@ -203,22 +262,30 @@ __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const 
                 if (EPI == EPI_RESID) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const uint4 q = rs_now[4 * h + i];
-                        f[8 * i + 0] += bf16lo(q.x);
-                        f[8 * i + 1] += bf16hi(q.x);
-                        f[8 * i + 2] += bf16lo(q.y);
-                        f[8 * i + 3] += bf16hi(q.y);
-                        f[8 * i + 4] += bf16lo(q.z);
-                        f[8 * i + 5] += bf16hi(q.z);
-                        f[8 * i + 6] += bf16lo(q.w);
-                        f[8 * i + 7] += bf16hi(q.w);
+                        const uint4 r4 = rs_now[4 * h + i];
+                        f[8 * i + 0] += bf16lo(r4.x);
+                        f[8 * i + 1] += bf16hi(r4.x);
+                        f[8 * i + 2] += bf16lo(r4.y);
+                        f[8 * i + 3] += bf16hi(r4.y);
+                        f[8 * i + 4] += bf16lo(r4.z);
+                        f[8 * i + 5] += bf16hi(r4.z);
+                        f[8 * i + 6] += bf16lo(r4.w);
+                        f[8 * i + 7] += bf16hi(r4.w);
                     }
                 }
+#pragma unroll
+                for (int i = 0; i < 4; ++i) q[4 * h + i] = pack8(f + 8 * i);
+            }
+            if (tma_rows) {
+                staging_acquire(lane);
+                uint8_t* buf = sout + sbuf * 4096;
+                stage_row64(buf, lane, q);
+                store_block64(tmOut, buf, lane, col, warp_row0);
+                sbuf ^= 1u;
+            } else {
                 uint4* dst = reinterpret_cast<uint4*>(args.out0 + row * args.ld0 + col);
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    dst[i] = make_uint4(pack_bf16x2(f[8 * i + 0], f[8 * i + 1]), pack_bf16x2(f[8 * i + 2], f[8 * i + 3]),
-                                        pack_bf16x2(f[8 * i + 4], f[8 * i + 5]), pack_bf16x2(f[8 * i + 6], f[8 * i + 7]));
+                for (int i = 0; i < 8; ++i) dst[i] = q[i];
             }
         }
     }
@@ -227,14 +294,16 @@ __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const 
 template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
+                   const GemmArgs args) {
     pdl_begin();
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+    uint8_t* sOut = sB + C::STAGES * C::B_BYTES;  // epilogue staging (1024-aligned)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_STAGE_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* tfull = empty + C::STAGES;
     uint64_t* tempty = tfull + 2;
@@ -350,6 +419,7 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------------------------------------------- epilogue
         const int quad = warp & 3;
         const int row_in_tile = quad * 32 + lane;
+        uint32_t sbuf = 0;
         int it = 0;
         for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
             TileJob j;
@@ -370,11 +440,15 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quad * 32) << 16);
-            gemm_epilogue_store<BN, EPI>(args, j, row_ok, row, tbase, rs);
+            const bool tma_rows = BN == 256 && args.tma_store != 0 && j.rows >= quad * 32 + 32 &&
+                                  !(EPI == EPI_PROJ_ROUTER && j.seg == 1);
+            gemm_epilogue_store<BN, EPI>(args, j, row_ok, row, tbase, rs, &tmOut, sOut + quad * 8192, sbuf, tma_rows,
+                                         j.a_row0 + quad * 32, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[buf]);
         }
+        if (lane == 0) bulk_wait_group_all();  // the tile stores are complete before the CTA can exit
     }
 
     tc_fence_before();
@@ -416,7 +490,8 @@ struct GemmPairCfg {
     static constexpr int B_BYTES = (BN / 2) * BK * 2;  // this CTA's half of the B rows
     static constexpr int STAGES = 6;
     static constexpr int TMEM_COLS = 2 * BN;
-    static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 + 256;
+    static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + OUT_STAGE_BYTES + 1024 + 256;
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 template <int EPI>
@@ -460,7 +535,8 @@ __device__ __forceinline__ int total_tiles_pair(const GemmArgs& a) {
 template <int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmB2, const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
+                        const GemmArgs args) {
     pdl_begin();
     using C = GemmPairCfg;
     constexpr int BN = C::BN;
@@ -468,7 +544,8 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + C::STAGES * C::A_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sB + C::STAGES * C::B_BYTES);
+    uint8_t* sOut = sB + C::STAGES * C::B_BYTES;  // epilogue staging (1024-aligned)
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + OUT_STAGE_BYTES);
     uint64_t* empty = full + C::STAGES;
     uint64_t* tfull = empty + C::STAGES;
     uint64_t* tempty = tfull + 2;
@@ -585,6 +662,7 @@ __global__ void __launch_bounds__(192, 1)
         // ---------------------------------------------------- epilogue (both CTAs, own 128 rows)
         const int quad = warp & 3;
         const int row_in_tile = quad * 32 + lane;
+        uint32_t sbuf = 0;
         int it = 0;
         for (int t = pid; t < ntiles; t += npid, ++it) {
             TileJob j;
@@ -601,11 +679,15 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + buf * BN + (static_cast<uint32_t>(quad * 32) << 16);
-            gemm_epilogue_store<BN, EPI>(args, j, row_ok, row, tbase, rs);
+            const bool tma_rows = BN == 256 && args.tma_store != 0 && j.rows >= quad * 32 + 32 &&
+                                  !(EPI == EPI_PROJ_ROUTER && j.seg == 1);
+            gemm_epilogue_store<BN, EPI>(args, j, row_ok, row, tbase, rs, &tmOut, sOut + quad * 8192, sbuf, tma_rows,
+                                         j.a_row0 + quad * 32, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(mapa_shared(&tempty[buf], 0));
         }
+        if (lane == 0) bulk_wait_group_all();
     }
 
     tc_fence_before();
