@@ -141,6 +141,13 @@ ACT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 1.0 + 1.0 / 32}
 MX_RATE = 2.0
 
 
+#: DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of that kernel as it is now
+#: (profiles/traffic_tc_swap_nemotron_decode.md).  A kernel that changes drops out of this table.
+NCU_TRAFFIC = {
+    ("nemotron_decode", "expert_up_stream"): 806.1e6,
+}
+
+
 def layer_work(cfg, stats, T):
     """F (FLOPs), B (bytes) and F_eff (FLOPs at the bf16 rate that take as long) of one forward, from its actual
     routing (plus the shared expert, if any)."""
@@ -314,7 +321,7 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     roof["kernel"] = dom
     roof["launch_ms"] = per_launch_ms
     roof["algorithmic_per_launch"] = {"flops": flops, "bytes": nbytes}
-    roof["traffic"] = None
+    roof["traffic"] = NCU_TRAFFIC.get((cfg.name, dom))
     roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "")
 
     F, B, F_eff = layer_work(cfg, stats, T)
