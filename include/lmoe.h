@@ -66,6 +66,7 @@ extern "C" {
 #define LMOE_ERR_TIMEOUT (-5)           /* device: a bounded wait inside a kernel gave up */
 #define LMOE_ERR_BAD_INDEX (-6)         /* device: an expert id outside [0, n_total) */
 #define LMOE_ERR_WORKSPACE (-7)         /* workspace missing or smaller than lmoe_workspace_bytes */
+#define LMOE_ERR_BAD_COUNTS (-8)        /* device: received row counts of lmoe_ep_experts inconsistent */
 
 #define LMOE_ACT_RELU2 0    /* h = relu(u)^2 (non-gated) */
 #define LMOE_ACT_SWIGLU 1   /* W1_e rows [0,m) gate, [m,2m) up: h = silu(gate) * up */
@@ -83,6 +84,11 @@ extern "C" {
  * multiple of 64 up to 16384.  A block-scaled expert_fmt also requires
  * latent and m to be multiples of 128 and max_tokens <= 32 (the decode
  * regime, where every expert streams its weights).
+ * Expert parallelism (see lmoe_ep_dispatch): ep_size 0 or 1 means none;
+ * otherwise 2 <= ep_size <= n_experts, n_experts a multiple of ep_size,
+ * 0 <= ep_rank < ep_size, expert_fmt == LMOE_FMT_BF16, and
+ * ep_size * max_tokens * min(top_k, n_local) <= 2^30, with
+ * n_local = n_experts / ep_size.
  */
 typedef struct lmoe_config {
     int32_t d;             /* model width */
@@ -99,16 +105,24 @@ typedef struct lmoe_config {
     int32_t latent_router; /* 1: the gate reads z (latent) instead of x (d) */
     int32_t shared_m;      /* hidden width of the shared expert at d; 0: no shared expert */
     int32_t expert_fmt;    /* LMOE_FMT_*: storage of the FFN experts' W1 / W2 */
+    int32_t ep_size;       /* ranks the FFN experts are split over (0 or 1: all experts on this device) */
+    int32_t ep_rank;       /* this rank: it holds FFN experts ep_rank * n_local .. (ep_rank + 1) * n_local - 1 */
 } lmoe_config;
 
-/* Device pointers to the layer's weights (bf16 unless stated).  n_total as above. */
+/*
+ * Device pointers to the layer's weights (bf16 unless stated).  n_total as
+ * above; n_local = n_experts / ep_size (n_experts without expert
+ * parallelism): w1, w2 and their scales hold this rank's experts only, local
+ * expert j being FFN expert ep_rank * n_local + j.  The router, projections,
+ * constant vectors and shared expert are whole on every rank.
+ */
 typedef struct lmoe_weights {
     const void *w_router;     /* [n_total, d], or [n_total, latent] with latent_router */
     const float *router_bias; /* fp32 [n_total], added to the logits before selection; may be NULL */
     const void *w_down;       /* [latent, d]; NULL when has_proj == 0 */
     const void *w_up;         /* [d, latent]; NULL when has_proj == 0 */
-    const void *w1;           /* [n_experts, g*m, latent], g = 2 for SwiGLU else 1 (block-scaled: codes) */
-    const void *w2;           /* [n_experts, latent, m] (block-scaled: codes) */
+    const void *w1;           /* [n_local, g*m, latent], g = 2 for SwiGLU else 1 (block-scaled: codes) */
+    const void *w2;           /* [n_local, latent, m] (block-scaled: codes) */
     const void *const_vecs;   /* [n_const, latent]; may be NULL when n_const == 0 */
     const void *w_shared1;    /* [g*shared_m, d] (gate rows first when gated); NULL when shared_m == 0 */
     const void *w_shared2;    /* [d, shared_m]; NULL when shared_m == 0 */
@@ -148,6 +162,8 @@ LMOE_API int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *wo
 
 /*
  * y = LatentMoE(x) for T tokens: x, y device bf16 [T, d], must not overlap.
+ * Rejected (LMOE_ERR_INVALID_ARG) on a handle with ep_size > 1, which holds
+ * only its rank's experts: use the lmoe_ep_* stages there.
  * 0 <= T <= max_tokens (T == 0 enqueues nothing and accepts NULL x / y).  Asynchronous on `stream`;
  * concurrent forwards on one handle share its workspace and must be ordered
  * by the caller (same stream).  Device-side faults (a bounded wait that gave
@@ -167,8 +183,8 @@ LMOE_API int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host,
 /*
  * Read and clear the device error word of the handle's workspace (blocking
  * copy; synchronise the forward's stream first).  Returns LMOE_OK,
- * LMOE_ERR_TIMEOUT or LMOE_ERR_BAD_INDEX (the first set, in that order), or
- * LMOE_ERR_CUDA if the read failed.
+ * LMOE_ERR_TIMEOUT, LMOE_ERR_BAD_INDEX or LMOE_ERR_BAD_COUNTS (the first set,
+ * in that order), or LMOE_ERR_CUDA if the read failed.
  */
 LMOE_API int lmoe_last_error(lmoe_handle *h);
 
@@ -298,6 +314,82 @@ LMOE_API int lmoe_dispatch_noalloc(const int32_t *idx, int32_t T, int32_t top_k,
  */
 LMOE_API int lmoe_mx_encode_weights(const void *w, int64_t rows, int32_t K, int32_t fmt, void *codes, void *scales,
                                     void *stream);
+
+/*
+ * Expert parallelism: the forward split at the two all-to-all exchanges that
+ * the pages put between routing and the experts and between the experts and
+ * the aggregation (Kimi K3 / Nemotron 3 Super article, "MoE 遇到了什么问题？";
+ * Nemotron-3 article section 2.2: the exchanged rows are latent-wide, which is
+ * the 4x saving in communication volume the LatentMoE design is built on).
+ * The library does no communication: the caller moves the rows between the
+ * stages (NCCL all-to-all over NVLink, for instance).  One forward on one rank:
+ *
+ *   lmoe_ep_dispatch   router, W_down, top-K', counting sort; the latent rows
+ *                      of slots routed to FFN experts, grouped by expert id,
+ *                      hence by destination rank, go to send_rows.
+ *   (caller)           all-to-all of send_counts, then of the rows: rank r's
+ *                      block of send_rows goes to rank r.
+ *   lmoe_ep_experts    this rank's experts on the rows it received.
+ *   (caller)           the reverse all-to-all of the expert outputs.
+ *   lmoe_ep_combine    aggregation in the latent width (MoE++ bypass experts
+ *                      included; they need no exchange), W_up and residual.
+ *
+ * The result of dispatch -> exchange -> experts -> exchange -> combine on
+ * ep_size ranks equals, token for token, lmoe_forward of the whole layer.
+ * The stages need expert_fmt == LMOE_FMT_BF16 (else LMOE_ERR_UNSUPPORTED_SHAPE).
+ * The three stages keep state in the handle's workspace: a handle serves one
+ * forward at a time, dispatch before combine, all on one stream.  The experts
+ * stage uses workspace that dispatch and combine do not, so it may run
+ * between them (it normally does: it serves the other ranks' tokens).
+ */
+
+/*
+ * Stage 1.  x device bf16 [T, d], 0 <= T <= max_tokens, unchanged until
+ * lmoe_ep_combine has run (the residual and the shared expert read it).
+ *   send_rows    device bf16 [T * top_k, latent] (capacity): rows 0 .. n_send-1
+ *                receive the latent rows (z_t, or x_t for the standard MoE)
+ *                of every (token, slot) routed to an FFN expert, ordered by
+ *                expert id, then token, then slot.  n_send = sum(send_counts).
+ *   send_counts  device int32 [n_experts]: rows per FFN expert.  Viewed as
+ *                [ep_size][n_local], row r counts the rows for rank r, which
+ *                are the r-th consecutive block of send_rows.
+ * T == 0 only zeroes send_counts.  Asynchronous on `stream`.
+ */
+LMOE_API int lmoe_ep_dispatch(lmoe_handle *h, const void *x, int32_t T, void *send_rows, int32_t *send_counts,
+                              void *stream);
+
+/*
+ * Stage 2: this rank's FFN experts on the rows it received.
+ *   recv_rows    device bf16 [n_recv, latent]: ep_size consecutive blocks,
+ *                block s being rank s's rows for this rank (its send_rows
+ *                block ep_rank), in rank s's order.
+ *   recv_counts  device int32 [ep_size, n_local]: recv_counts[s][j] = rank s's
+ *                send_counts[ep_rank * n_local + j].
+ *   n_recv       sum of recv_counts (host value), 0 .. ep_size * max_tokens *
+ *                min(top_k, n_local).
+ *   rows_bound   an upper bound of the rows any one local expert received (for
+ *                instance the tokens of all ranks together, or the exact
+ *                maximum of the column sums of recv_counts).  At most 32 lets
+ *                every expert take the weight-streaming GEMM (the same rule
+ *                lmoe_set_small_rows states for T); above 32 the grouped GEMM
+ *                runs too.  Must be >= 1 when n_recv > 0.
+ *   out_rows     device bf16 [n_recv, latent]: row i = o_e(recv row i), e its
+ *                expert.  May be recv_rows itself.
+ * The device checks recv_counts: a negative count, a sum other than n_recv, or
+ * an expert with more rows than rows_bound sets LMOE_ERR_BAD_COUNTS (see
+ * lmoe_last_error) and the stage then computes nothing.  Asynchronous.
+ */
+LMOE_API int lmoe_ep_experts(lmoe_handle *h, const void *recv_rows, const int32_t *recv_counts, int32_t n_recv,
+                             int32_t rows_bound, void *out_rows, void *stream);
+
+/*
+ * Stage 3.  ret_rows device bf16 [n_send, latent]: the expert outputs of
+ * send_rows, in the same order (the reverse exchange's result).  y device
+ * bf16 [T, d] (T of the dispatch), not overlapping x.  Requires a dispatch on
+ * this handle since the last combine (else LMOE_ERR_INVALID_ARG).  With T == 0
+ * it only closes the forward.  Asynchronous.
+ */
+LMOE_API int lmoe_ep_combine(lmoe_handle *h, const void *ret_rows, void *y, void *stream);
 
 #ifdef __cplusplus
 }

@@ -21,6 +21,7 @@
 #include "../../include/lmoe.h"
 #include "moe_kernels.cuh"
 #include "mx.cuh"
+#include "ep.cuh"
 #include "tc_gemm.cuh"
 #include "tc_swap.cuh"
 
@@ -106,6 +107,16 @@ bool config_ok(const lmoe_config& c) {
     if (c.expert_fmt < LMOE_FMT_BF16 || c.expert_fmt > LMOE_FMT_MXFP4) return false;
     if (c.expert_fmt != LMOE_FMT_BF16 && (c.latent % 128 != 0 || c.m % 128 != 0 || c.max_tokens > SMALL_MAX))
         return false;
+    if (c.ep_size < 0 || c.ep_size > 1024) return false;
+    if (c.ep_size > 1) {  // expert parallelism: whole local expert sets, bf16 experts
+        if (c.n_experts % c.ep_size != 0 || c.ep_rank < 0 || c.ep_rank >= c.ep_size) return false;
+        if (c.expert_fmt != LMOE_FMT_BF16) return false;
+        const long long n_local = c.n_experts / c.ep_size;
+        if (static_cast<long long>(c.ep_size) * c.max_tokens * std::min<long long>(c.top_k, n_local) > (1LL << 30))
+            return false;
+    } else if (c.ep_rank != 0) {
+        return false;
+    }
     return true;
 }
 
@@ -118,9 +129,16 @@ int mx_ld_sf(int K) { return K / 128 * 16; }
 constexpr int kFewTokenRows = 32;
 constexpr int kFewTokenMaxSplits = 16;
 
+// Expert-parallel ranks and local FFN experts of a configuration (1 and n_experts without expert parallelism).
+int ep_ranks(const lmoe_config& c) { return c.ep_size > 1 ? c.ep_size : 1; }
+int n_local_experts(const lmoe_config& c) { return c.n_experts / ep_ranks(c); }
+
 struct Plan {
     size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
-        partial, hs, s2, partial2, rows8, rows_sf, h8, h_sf, xin, yout, total;
+        partial, hs, s2, partial2, rows8, rows_sf, h8, h_sf, xin, yout, ep_map, ep_src, ep_dst, ep_counts,
+        ep_offsets, total;
+    size_t rows_cap;  // rows of the expert-side buffers: a forward's slots, or the most an experts stage receives
+    size_t ep_cap;    // rows an expert-parallel experts stage may receive
     int ld_logits, nwords, mt_max;
 };
 
@@ -135,9 +153,13 @@ Plan make_plan(const lmoe_config& c) {
     const size_t T = c.max_tokens, K = c.top_k, L = c.latent, d = c.d, m = c.m;
     const size_t nt = n_total(c);
     const size_t R = T * K;
+    const size_t n_local = n_local_experts(c);
+    p.ep_cap = static_cast<size_t>(ep_ranks(c)) * T * std::min(K, n_local);
+    p.rows_cap = std::max(R, p.ep_cap);
+    const size_t RC = p.rows_cap;
     p.ld_logits = static_cast<int>(round_up(nt, 64));
     p.nwords = static_cast<int>((T + 31) / 32);
-    p.mt_max = static_cast<int>((R + 127) / 128 + c.n_experts);
+    p.mt_max = static_cast<int>((RC + 127) / 128 + c.n_experts);
     p.hdr = take(HDR_WORDS * 4);
     p.logits = take(T * p.ld_logits * 4);
     p.z = c.has_proj ? take(T * L * 2) : 0;
@@ -151,8 +173,8 @@ Plan make_plan(const lmoe_config& c) {
     p.inv = take(R * 4);
     p.mt_list = take(static_cast<size_t>(p.mt_max) * 16);
     p.small_list = take(static_cast<size_t>(c.n_experts) * 16);
-    p.rows = take(R * L * 2);  // gathered expert inputs, then (reused) expert outputs
-    p.hbuf = take(R * m * 2);
+    p.rows = take(RC * L * 2);  // gathered expert inputs, then (reused) expert outputs
+    p.hbuf = take(RC * m * 2);
     p.yl = c.has_proj ? take(T * L * 2) : 0;
     {   // split-K partial sums of the few-token projections: [splits][128-row tiles][32 tokens] fp32
         auto up128 = [](size_t v) { return (v + 127) / 128 * 128; };
@@ -174,6 +196,12 @@ Plan make_plan(const lmoe_config& c) {
     }
     p.xin = take(T * d * 2);
     p.yout = take(T * d * 2);
+    // expert-parallel experts stage: received row -> expert-major row, segment tables, local counts / offsets
+    p.ep_map = take(p.ep_cap * 4);
+    p.ep_src = take((static_cast<size_t>(c.n_experts) + 1) * 4);
+    p.ep_dst = take(static_cast<size_t>(c.n_experts) * 4);
+    p.ep_counts = take(n_local * 4);
+    p.ep_offsets = take((n_local + 1) * 4);
     p.total = off;
     return p;
 }
@@ -181,10 +209,10 @@ Plan make_plan(const lmoe_config& c) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 enum Phase : int { PH_ROUTER = 0, PH_TOPK, PH_DISPATCH, PH_UP_TC, PH_UP_STREAM, PH_DOWN_TC, PH_DOWN_STREAM, PH_COMBINE,
-                   PH_WUP, PH_SHARED, PH_COUNT };
+                   PH_WUP, PH_SHARED, PH_EP_REGROUP, PH_COUNT };
 const char* kPhaseNames[PH_COUNT] = {"router_proj_gemm", "topk_softmax", "dispatch", "expert_up_gemm",
                                      "expert_up_stream", "expert_down_gemm", "expert_down_stream", "combine",
-                                     "up_proj_gemm", "shared_expert"};
+                                     "up_proj_gemm", "shared_expert", "ep_regroup"};
 
 template <int EPI>
 bool set_pair_attr() {
@@ -422,7 +450,11 @@ struct lmoe_handle {
     uint8_t* ws = nullptr;
     Plan p{};
     int n_tot = 0, g = 1, num_sms = 148, small_max = 16, device = 0;
+    int n_local = 1;      // FFN experts whose weights this handle holds
     int last_small = 16;  // threshold the last forward used
+    // expert-parallel forward in progress: the dispatch's x and T (ep_T < 0: none)
+    const void* ep_x = nullptr;
+    int ep_T = -1;
     unsigned long long timeout_ns = 1000000000ull;
     // weight descriptors: router/projection operands for both column tiles, expert weights, workspace operands
     CUtensorMap wdown64{}, wdown256{}, wr64{}, wr256{}, wup64{}, wup256{}, w1{}, w2{};
@@ -477,23 +509,33 @@ void free_events(lmoe_handle* h) {
     h->prof_max = h->prof_n = 0;
 }
 
-int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, const lmoe_debug* dbg) {
+// Shared expert (forked to the side stream), router (+ W_down), top-K' and the
+// counting sort by expert.  The feature rows of slots routed to FFN experts are
+// gathered in sorted order to `rows_dst` (ld = latent), or encoded as the MXFP8
+// token operand for block-scaled experts; `small` shapes the tile lists.
+int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat16* rows_dst, int small) {
     const lmoe_config& c = h->c;
     const Plan& p = h->p;
-    const int K = c.top_k, L = c.latent, d = c.d, m = c.m, nt = h->n_tot;
+    const int K = c.top_k, L = c.latent, d = c.d, nt = h->n_tot;
     const bool proj = c.has_proj != 0;
+    const bool mx = c.expert_fmt != LMOE_FMT_BF16;
     int* hdr = h->at<int>(p.hdr);
     float* logits = h->at<float>(p.logits);
     __nv_bfloat16* z = proj ? h->at<__nv_bfloat16>(p.z) : nullptr;
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
-    __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(y);
     const __nv_bfloat16* feat = proj ? z : xb;  // what the experts read (latent z, or x for the standard MoE)
     int32_t* idx = h->at<int32_t>(p.idx);
     float* wts = h->at<float>(p.w);
-    __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
-    __nv_bfloat16* hbuf = h->at<__nv_bfloat16>(p.hbuf);
     int4* mt_list = h->at<int4>(p.mt_list);
     int4* small_list = h->at<int4>(p.small_list);
+    const int nwords = (T + 31) / 32;
+    int* counts = h->at<int>(p.counts);
+    int* offsets = h->at<int>(p.offsets);
+    int32_t* perm = h->at<int32_t>(p.perm);
+    int32_t* inv = h->at<int32_t>(p.inv);
+    const long slots = static_cast<long>(T) * K;
+    const int npl = (nt + 31) / 32;
+    const float* bias = h->w.router_bias;
 
     CUtensorMap a_x;
     if (!make_map(&a_x, x, T, d, d, 128)) return LMOE_ERR_CUDA;
@@ -506,7 +548,6 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     // ---------------------------------------------------------------- shared expert (side stream)
     // s2 = x + Ws2 act(Ws1 x) runs concurrently with the routed path; the up-projection
     // (or, for the standard MoE, the combine) waits for it and adds s2 instead of x.
-    const __nv_bfloat16* resid = xb;
     if (c.shared_m > 0) {
         const int ms = c.shared_m, srows = h->g * ms;
         __nv_bfloat16* hs = h->at<__nv_bfloat16>(p.hs);
@@ -569,7 +610,6 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
             }
         }
         if (cudaEventRecord(h->ev_join, h->side) != cudaSuccess) return LMOE_ERR_CUDA;
-        resid = s2;
     }
 
     // ---------------------------------------------------------------- router (+ W_down)
@@ -639,22 +679,6 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
             }
         }
     }
-    // Experts with at most `small` rows stream their weights; when every expert
-    // must (T <= small) the grouped GEMMs are not launched at all.
-    const bool mx = c.expert_fmt != LMOE_FMT_BF16;
-    int small = h->small_max;
-    if (small > 0 && T <= SMALL_MAX) small = T <= 16 ? 16 : SMALL_MAX;
-    if (mx) small = SMALL_MAX;  // block-scaled experts always stream (T <= 32 is a create-time limit)
-    const bool need_tc = T > small;
-    h->last_small = small;
-    const int nwords = (T + 31) / 32;
-    int* counts = h->at<int>(p.counts);
-    int* offsets = h->at<int>(p.offsets);
-    int32_t* perm = h->at<int32_t>(p.perm);
-    int32_t* inv = h->at<int32_t>(p.inv);
-    const long slots = static_cast<long>(T) * K;
-    const int npl = (nt + 31) / 32;
-    const float* bias = h->w.router_bias;
     // ---------------------------------------------------------------- top-K' + softmax
     {
         PhaseScope ps(h, PH_TOPK, s, 1);
@@ -679,7 +703,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
                    feat, L, L, h->at<uint8_t>(p.rows8), L, h->at<uint8_t>(p.rows_sf), mx_ld_sf(L));
         else
             launch(dispatch_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K,
-                   c.n_experts, feat, L, L, rows, L);
+                   c.n_experts, feat, L, L, rows_dst, L);
     } else {
         PhaseScope ps(h, PH_DISPATCH, s, 4);
         uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
@@ -688,8 +712,29 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         launch(dispatch_expert_scan_kernel, (nt + 7) / 8, 256, 0, s, bitmap, T, nt, prefix, counts);
         launch(dispatch_offsets_kernel, 1, 1024, 0, s, counts, nt, c.n_experts, small, offsets, mt_list, small_list, hdr);
         launch(dispatch_scatter_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, T, K, nt, c.n_experts,
-               bitmap, prefix, offsets, feat, L, L, rows, L, perm, inv);
+               bitmap, prefix, offsets, feat, L, L, rows_dst, L, perm, inv);
     }
+    return LMOE_OK;
+}
+
+// Expert up (+ activation) and down GEMMs over the sorted rows in the
+// workspace, by the tile lists and counts in its header; the outputs replace
+// the rows.  need_tc: some expert has more than `small` rows (the grouped GEMMs
+// run).
+int run_experts(lmoe_handle* h, int small, bool need_tc, cudaStream_t s) {
+    const lmoe_config& c = h->c;
+    const Plan& p = h->p;
+    const int L = c.latent, m = c.m;
+    const bool mx = c.expert_fmt != LMOE_FMT_BF16;
+    int* hdr = h->at<int>(p.hdr);
+    __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
+    __nv_bfloat16* hbuf = h->at<__nv_bfloat16>(p.hbuf);
+    int4* mt_list = h->at<int4>(p.mt_list);
+    int4* small_list = h->at<int4>(p.small_list);
+    GemmArgs base{};
+    base.err = hdr + HDR_ERR;
+    base.timeout_ns = h->timeout_ns;
+
     // ---------------------------------------------------------------- expert up (+ activation)
     if (need_tc) {
         // Grouped GEMMs stay on single-CTA 128-row tiles: with a few hundred rows per expert, 256-row pair
@@ -800,13 +845,37 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
         a.timeout_ns = h->timeout_ns;
         launch_stream(small, EPI_BF16, h->w2s, h->h16, h->h32, a, h->num_sms, s);
     }
+    return LMOE_OK;
+}
+
+// Combine in the latent width of the expert outputs O (the sorted rows of the
+// FFN-expert slots, ld = latent), then W_up + residual (joining the shared
+// expert's side stream).
+int run_back(lmoe_handle* h, const __nv_bfloat16* O, const void* x, void* y, int T, cudaStream_t s) {
+    const lmoe_config& c = h->c;
+    const Plan& p = h->p;
+    const int K = c.top_k, L = c.latent, d = c.d;
+    const bool proj = c.has_proj != 0;
+    int* hdr = h->at<int>(p.hdr);
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(y);
+    const __nv_bfloat16* feat = proj ? h->at<__nv_bfloat16>(p.z) : xb;
+    const __nv_bfloat16* resid = c.shared_m > 0 ? h->at<__nv_bfloat16>(p.s2) : xb;  // x + shared expert, or x
+    const int32_t* idx = h->at<int32_t>(p.idx);
+    const float* wts = h->at<float>(p.w);
+    const int32_t* inv = h->at<int32_t>(p.inv);
+    const int m_tiles = (T + 127) / 128;
+    GemmArgs base{};
+    base.err = hdr + HDR_ERR;
+    base.timeout_ns = h->timeout_ns;
+
     // ---------------------------------------------------------------- combine in the latent width
     {
         PhaseScope ps(h, PH_COMBINE, s, 1);
         __nv_bfloat16* out = proj ? h->at<__nv_bfloat16>(p.yl) : yb;
         if (!proj && c.shared_m > 0 && cudaStreamWaitEvent(s, h->ev_join, 0) != cudaSuccess) return LMOE_ERR_CUDA;
         auto kern = T <= 256 ? combine_kernel<32> : combine_kernel<8>;
-        launch(kern, T, 128, 0, s, static_cast<const __nv_bfloat16*>(rows), L,
+        launch(kern, T, 128, 0, s, O, L,
                static_cast<const int32_t*>(inv), static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
                feat, L, static_cast<const __nv_bfloat16*>(h->w.const_vecs), T, K, L, c.n_experts, c.n_zero, c.n_copy,
                proj ? static_cast<const __nv_bfloat16*>(nullptr) : resid, d, out, proj ? L : d);
@@ -841,23 +910,50 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     }
     if (cudaGetLastError() != cudaSuccess) return LMOE_ERR_CUDA;
     if (h->prof && h->prof_n < h->prof_max) ++h->prof_n;
+    return LMOE_OK;
+}
+
+// Experts with at most `small` rows stream their weights.  rows_bound bounds
+// the rows of any one expert (the token count of a forward); when every expert
+// must stream (rows_bound <= small) the grouped GEMMs are not launched at all.
+int choose_small(const lmoe_handle* h, long rows_bound) {
+    int small = h->small_max;
+    if (small > 0 && rows_bound <= SMALL_MAX) small = rows_bound <= 16 ? 16 : SMALL_MAX;
+    if (h->c.expert_fmt != LMOE_FMT_BF16) small = SMALL_MAX;  // block-scaled experts always stream (T <= 32)
+    return small;
+}
+
+int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, const lmoe_debug* dbg) {
+    const lmoe_config& c = h->c;
+    const Plan& p = h->p;
+    const int K = c.top_k, L = c.latent, nt = h->n_tot;
+    const bool proj = c.has_proj != 0;
+    const int small = choose_small(h, T);
+    h->last_small = small;
+    __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
+    int st = run_front(h, x, T, s, rows, small);
+    if (st != LMOE_OK) return st;
+    st = run_experts(h, small, T > small, s);
+    if (st != LMOE_OK) return st;
+    st = run_back(h, rows, x, y, T, s);
+    if (st != LMOE_OK) return st;
 
     if (dbg != nullptr) {
         bool ok = true;
         auto cp = [&](void* dst, const void* src, size_t bytes) {
             if (dst) ok &= cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
         };
-        cp(dbg->topk_idx, idx, static_cast<size_t>(T) * K * 4);
-        cp(dbg->topk_w, wts, static_cast<size_t>(T) * K * 4);
+        cp(dbg->topk_idx, h->at<int32_t>(p.idx), static_cast<size_t>(T) * K * 4);
+        cp(dbg->topk_w, h->at<float>(p.w), static_cast<size_t>(T) * K * 4);
         cp(dbg->counts, h->at<int>(p.counts), static_cast<size_t>(nt) * 4);
         cp(dbg->offsets, h->at<int>(p.offsets), static_cast<size_t>(nt + 1) * 4);
         cp(dbg->perm, h->at<int32_t>(p.perm), static_cast<size_t>(T) * K * 4);
         if (proj) {
-            cp(dbg->z, z, static_cast<size_t>(T) * L * 2);
+            cp(dbg->z, h->at<__nv_bfloat16>(p.z), static_cast<size_t>(T) * L * 2);
             cp(dbg->yl, h->at<__nv_bfloat16>(p.yl), static_cast<size_t>(T) * L * 2);
         }
         if (dbg->logits)
-            ok &= cudaMemcpy2DAsync(dbg->logits, static_cast<size_t>(nt) * 4, logits, static_cast<size_t>(p.ld_logits) * 4,
+            ok &= cudaMemcpy2DAsync(dbg->logits, static_cast<size_t>(nt) * 4, h->at<float>(p.logits), static_cast<size_t>(p.ld_logits) * 4,
                                     static_cast<size_t>(nt) * 4, T, cudaMemcpyDeviceToDevice, s) == cudaSuccess;
         if (!ok) return LMOE_ERR_CUDA;
     }
@@ -906,6 +1002,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     h->ws = static_cast<uint8_t*>(workspace);
     h->p = p;
     h->n_tot = n_total(c);
+    h->n_local = n_local_experts(c);
     h->g = c.act == LMOE_ACT_SWIGLU ? 2 : 1;
     if (cudaGetDevice(&h->device) != cudaSuccess ||
         cudaDeviceGetAttribute(&h->num_sms, cudaDevAttrMultiProcessorCount, h->device) != cudaSuccess ||
@@ -916,6 +1013,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     const int L = c.latent, d = c.d, m = c.m, nt = h->n_tot;
     const int fdim = c.latent_router ? L : d;
     const uint64_t R = static_cast<uint64_t>(c.max_tokens) * c.top_k;
+    const uint64_t RC = p.rows_cap;
     bool ok = true;
     ok &= make_map(&h->wr128, w->w_router, nt, fdim, fdim, 128);
     ok &= make_map(&h->wr64, w->w_router, nt, fdim, fdim, 64);
@@ -934,7 +1032,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
         ok &= make_map(&h->yl16, h->at<void>(p.yl), c.max_tokens, L, L, 16);
         ok &= make_map(&h->yl32, h->at<void>(p.yl), c.max_tokens, L, L, 32);
     }
-    const uint64_t w1_rows = static_cast<uint64_t>(c.n_experts) * h->g * m, w2_rows = static_cast<uint64_t>(c.n_experts) * L;
+    const uint64_t w1_rows = static_cast<uint64_t>(h->n_local) * h->g * m, w2_rows = static_cast<uint64_t>(h->n_local) * L;
     if (c.expert_fmt == LMOE_FMT_BF16) {
         ok &= make_map(&h->w1, w->w1, w1_rows, L, L, h->g == 2 ? 128 : 256);
         ok &= make_map(&h->w2, w->w2, w2_rows, m, m, 256);
@@ -953,15 +1051,15 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
         ok &= make_map_u8(&h->h8, h->at<void>(p.h8), R, m, m, 128, 32, true);
         ok &= make_map_u8(&h->h_sf, h->at<void>(p.h_sf), R, mx_ld_sf(m), mx_ld_sf(m), 16, 32, false);
     }
-    ok &= make_map(&h->a_rows, h->at<void>(p.rows), R, L, L, 128);
-    ok &= make_map(&h->a_h, h->at<void>(p.hbuf), R, m, m, 128);
-    ok &= make_map(&h->o_h, h->at<void>(p.hbuf), R, m, m, 32);
-    ok &= make_map(&h->o_rows, h->at<void>(p.rows), R, L, L, 32);
+    ok &= make_map(&h->a_rows, h->at<void>(p.rows), RC, L, L, 128);
+    ok &= make_map(&h->a_h, h->at<void>(p.hbuf), RC, m, m, 128);
+    ok &= make_map(&h->o_h, h->at<void>(p.hbuf), RC, m, m, 32);
+    ok &= make_map(&h->o_rows, h->at<void>(p.rows), RC, L, L, 32);
     if (c.has_proj) ok &= make_map(&h->o_z, h->at<void>(p.z), c.max_tokens, L, L, 32);
-    ok &= make_map(&h->rows16, h->at<void>(p.rows), R, L, L, 16);
-    ok &= make_map(&h->rows32, h->at<void>(p.rows), R, L, L, 32);
-    ok &= make_map(&h->h16, h->at<void>(p.hbuf), R, m, m, 16);
-    ok &= make_map(&h->h32, h->at<void>(p.hbuf), R, m, m, 32);
+    ok &= make_map(&h->rows16, h->at<void>(p.rows), RC, L, L, 16);
+    ok &= make_map(&h->rows32, h->at<void>(p.rows), RC, L, L, 32);
+    ok &= make_map(&h->h16, h->at<void>(p.hbuf), RC, m, m, 16);
+    ok &= make_map(&h->h32, h->at<void>(p.hbuf), RC, m, m, 32);
     if (c.shared_m > 0) {
         const int ms = c.shared_m, srows = h->g * ms;
         ok &= make_map(&h->ws1_64, w->w_shared1, srows, d, d, h->g == 2 ? 32 : 64);
@@ -987,7 +1085,7 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
 }
 
 int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, void* stream, const lmoe_debug* dbg) {
-    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (h == nullptr || h->c.ep_size > 1) return LMOE_ERR_INVALID_ARG;
     if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
     if (T == 0) return LMOE_OK;
     if (x == nullptr || y == nullptr) return LMOE_ERR_INVALID_ARG;
@@ -999,7 +1097,7 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, void* stream
 }
 
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, void* stream) {
-    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (h == nullptr || h->c.ep_size > 1) return LMOE_ERR_INVALID_ARG;
     if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
     if (T == 0) return LMOE_OK;
     if (x_host == nullptr || y_host == nullptr) return LMOE_ERR_INVALID_ARG;
@@ -1014,6 +1112,93 @@ int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t 
     return LMOE_OK;
 }
 
+int lmoe_ep_dispatch(lmoe_handle* h, const void* x, int32_t T, void* send_rows, int32_t* send_counts, void* stream) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (h->c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
+    if (send_counts == nullptr || !aligned16(send_counts)) return LMOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(send_counts, 0, static_cast<size_t>(h->c.n_experts) * 4, s) != cudaSuccess)
+            return LMOE_ERR_CUDA;
+        h->ep_x = nullptr;
+        h->ep_T = 0;
+        return LMOE_OK;
+    }
+    if (x == nullptr || send_rows == nullptr || !aligned16(x) || !aligned16(send_rows)) return LMOE_ERR_INVALID_ARG;
+    // the tile lists the sort builds are not used here: the experts stage rebuilds them for the rows it receives
+    const int st = run_front(h, x, T, s, static_cast<__nv_bfloat16*>(send_rows), h->small_max);
+    if (st != LMOE_OK) return st;
+    if (cudaMemcpyAsync(send_counts, h->at<int>(h->p.counts), static_cast<size_t>(h->c.n_experts) * 4,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return LMOE_ERR_CUDA;
+    h->ep_x = x;
+    h->ep_T = T;
+    return LMOE_OK;
+}
+
+int lmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const int32_t* recv_counts, int32_t n_recv,
+                    int32_t rows_bound, void* out_rows, void* stream) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    const lmoe_config& c = h->c;
+    if (c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (n_recv < 0 || static_cast<size_t>(n_recv) > h->p.ep_cap) return LMOE_ERR_TOO_MANY_TOKENS;
+    if (n_recv == 0) return LMOE_OK;
+    if (rows_bound < 1) return LMOE_ERR_INVALID_ARG;
+    if (recv_rows == nullptr || recv_counts == nullptr || out_rows == nullptr || !aligned16(recv_rows) ||
+        !aligned16(recv_counts) || !aligned16(out_rows))
+        return LMOE_ERR_INVALID_ARG;
+    const Plan& p = h->p;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int ep = ep_ranks(c), nl = h->n_local, L = c.latent;
+    const int small = choose_small(h, rows_bound);
+    h->last_small = small;
+    int* hdr = h->at<int>(p.hdr);
+    int* src_off = h->at<int>(p.ep_src);
+    int* dst_base = h->at<int>(p.ep_dst);
+    int32_t* map = h->at<int32_t>(p.ep_map);
+    __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
+    const int n_seg = ep * nl;
+    const unsigned grid = static_cast<unsigned>(
+        std::min<long>((n_recv + EP_ROWS_PER_PASS - 1) / EP_ROWS_PER_PASS, 8L * h->num_sms));
+    {
+        PhaseScope ps(h, PH_EP_REGROUP, s, 2);
+        launch(ep_prep_kernel, 1, 1024, 0, s, recv_counts, ep, nl, static_cast<int>(n_recv),
+               static_cast<int>(rows_bound), small, h->at<int>(p.ep_counts), h->at<int>(p.ep_offsets),
+               h->at<int4>(p.mt_list), h->at<int4>(p.small_list), src_off, dst_base, hdr);
+        launch(ep_regroup_kernel, grid, 32 * EP_ROWS_PER_PASS, static_cast<size_t>(2 * n_seg + 1) * 4, s,
+               static_cast<const __nv_bfloat16*>(recv_rows), static_cast<int>(n_recv), L,
+               static_cast<const int*>(src_off), static_cast<const int*>(dst_base), n_seg,
+               static_cast<const int*>(hdr), rows, map);
+    }
+    const int st = run_experts(h, small, rows_bound > small, s);
+    if (st != LMOE_OK) return st;
+    {
+        PhaseScope ps(h, PH_EP_REGROUP, s, 1);
+        launch(ep_unregroup_kernel, grid, 32 * EP_ROWS_PER_PASS, 0, s, static_cast<const __nv_bfloat16*>(rows),
+               static_cast<const int32_t*>(map), static_cast<int>(n_recv), L, static_cast<const int*>(hdr),
+               static_cast<__nv_bfloat16*>(out_rows));
+    }
+    return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+int lmoe_ep_combine(lmoe_handle* h, const void* ret_rows, void* y, void* stream) {
+    if (h == nullptr || h->ep_T < 0) return LMOE_ERR_INVALID_ARG;
+    if (h->c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    const int T = h->ep_T;
+    const void* x = h->ep_x;
+    if (T == 0) {
+        h->ep_T = -1;
+        return LMOE_OK;
+    }
+    if (ret_rows == nullptr || y == nullptr || !aligned16(ret_rows) || !aligned16(y)) return LMOE_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(T) * h->c.d * 2;
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+    if (xa < ya + bytes && ya < xa + bytes) return LMOE_ERR_INVALID_ARG;
+    h->ep_T = -1;
+    return run_back(h, static_cast<const __nv_bfloat16*>(ret_rows), x, y, T, static_cast<cudaStream_t>(stream));
+}
+
 int lmoe_last_error(lmoe_handle* h) {
     if (h == nullptr) return LMOE_ERR_INVALID_ARG;
     int err = 0;
@@ -1022,6 +1207,7 @@ int lmoe_last_error(lmoe_handle* h) {
     if (err != 0 && cudaMemset(dev, 0, 4) != cudaSuccess) return LMOE_ERR_CUDA;
     if (err & DEVERR_TIMEOUT) return LMOE_ERR_TIMEOUT;
     if (err & DEVERR_BAD_INDEX) return LMOE_ERR_BAD_INDEX;
+    if (err & DEVERR_BAD_COUNTS) return LMOE_ERR_BAD_COUNTS;
     return LMOE_OK;
 }
 
@@ -1044,6 +1230,7 @@ const char* lmoe_status_string(int status) {
         case LMOE_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up";
         case LMOE_ERR_BAD_INDEX: return "expert id out of range";
         case LMOE_ERR_WORKSPACE: return "workspace missing or too small";
+        case LMOE_ERR_BAD_COUNTS: return "received row counts inconsistent";
         default: return "unknown status";
     }
 }

@@ -17,6 +17,7 @@ enum : int {
     HDR_ROWS = 1,       // R: (token, slot) pairs routed to FFN experts
     HDR_MT = 2,         // entries of the tensor-core M-tile list
     HDR_NSMALL = 3,     // entries of the weight-streaming list
+    HDR_EP_BAD = 4,     // 1: the received counts of the expert-parallel experts stage were rejected
     HDR_WORDS = 16,
 };
 
@@ -301,17 +302,15 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
     return out;
 }
 
-// Single block of 1024 threads: offsets (exclusive scan of counts), the
-// tensor-core M-tile list (experts with more than `small_max` rows, split in
-// 128-row tiles) and the weight-streaming list (experts with 1..small_max rows).
-static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __restrict__ counts, int n_tot, int n_ffn,
-                                                                int small_max, int* __restrict__ offsets,
-                                                                int4* __restrict__ mt_list, int4* __restrict__ small_list,
-                                                                int* __restrict__ hdr) {
-    pdl_begin();
-    __shared__ int scratch[33];
+// Offsets (exclusive scan of counts), the tensor-core M-tile list (experts
+// with more than `small_max` rows, split in 128-row tiles) and the
+// weight-streaming list (experts with 1..small_max rows).  Body for a single
+// block of 1024 threads, thread e holding expert e's row count c (0 for
+// e >= n_tot); returns offsets[e].
+__device__ __forceinline__ int offsets_and_tiles(int c, int n_tot, int n_ffn, int small_max, int* __restrict__ offsets,
+                                                 int4* __restrict__ mt_list, int4* __restrict__ small_list,
+                                                 int* __restrict__ hdr, int* scratch) {
     const int e = threadIdx.x;
-    const int c = e < n_tot ? counts[e] : 0;
     int total;
     const int off = block_exclusive_scan(c, scratch, &total);
     if (e < n_tot) offsets[e] = off;
@@ -333,6 +332,18 @@ static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int
         hdr[HDR_MT] = mt_total;
         hdr[HDR_NSMALL] = small_total;
     }
+    return off;
+}
+
+// The same as a kernel of one block of 1024 threads, over counts[] in memory.
+static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __restrict__ counts, int n_tot, int n_ffn,
+                                                                int small_max, int* __restrict__ offsets,
+                                                                int4* __restrict__ mt_list, int4* __restrict__ small_list,
+                                                                int* __restrict__ hdr) {
+    pdl_begin();
+    __shared__ int scratch[33];
+    const int e = threadIdx.x;
+    offsets_and_tiles(e < n_tot ? counts[e] : 0, n_tot, n_ffn, small_max, offsets, mt_list, small_list, hdr, scratch);
 }
 
 // Small batches (T <= 256): bitmap, per-expert prefix, offsets, tile lists and

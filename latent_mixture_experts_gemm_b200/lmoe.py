@@ -18,7 +18,8 @@ LIB_PATH = os.path.join(HERE, "liblmoe.so")
 LMOE_OK = 0
 LMOE_FMT_BF16, LMOE_FMT_MXFP8, LMOE_FMT_MXFP4 = 0, 1, 2
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_ARG", -2: "LMOE_ERR_UNSUPPORTED_SHAPE", -3: "LMOE_ERR_TOO_MANY_TOKENS",
-          -4: "LMOE_ERR_CUDA", -5: "LMOE_ERR_TIMEOUT", -6: "LMOE_ERR_BAD_INDEX", -7: "LMOE_ERR_WORKSPACE"}
+          -4: "LMOE_ERR_CUDA", -5: "LMOE_ERR_TIMEOUT", -6: "LMOE_ERR_BAD_INDEX", -7: "LMOE_ERR_WORKSPACE",
+          -8: "LMOE_ERR_BAD_COUNTS"}
 
 P = ctypes.c_void_p
 I32 = ctypes.c_int32
@@ -26,7 +27,8 @@ I32 = ctypes.c_int32
 
 class lmoe_config(ctypes.Structure):
     _fields_ = [(n, I32) for n in ("d", "latent", "m", "n_experts", "top_k", "max_tokens", "act", "n_zero", "n_copy",
-                                   "n_const", "has_proj", "latent_router", "shared_m", "expert_fmt")]
+                                   "n_const", "has_proj", "latent_router", "shared_m", "expert_fmt", "ep_size",
+                                   "ep_rank")]
 
 
 class lmoe_weights(ctypes.Structure):
@@ -78,6 +80,9 @@ def lib() -> ctypes.CDLL:
         L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
         L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
         L.lmoe_mx_encode_weights.argtypes = [P, ctypes.c_int64, I32, I32, P, P, P]
+        L.lmoe_ep_dispatch.argtypes = [P, P, I32, P, P, P]
+        L.lmoe_ep_experts.argtypes = [P, P, P, I32, I32, P, P]
+        L.lmoe_ep_combine.argtypes = [P, P, P, P]
         _lib = L
     return _lib
 
@@ -208,11 +213,30 @@ def lmoe_mx_encode_weights(w: torch.Tensor, fmt: int, stream=None):
     return codes, scales
 
 
+def lmoe_ep_dispatch(h: int, x: torch.Tensor, send_rows: torch.Tensor, send_counts: torch.Tensor,
+                     stream=None) -> None:
+    """Expert-parallel stage 1 for the rows of ``x`` (device bf16 [T, d])."""
+    _check("lmoe_ep_dispatch", lib().lmoe_ep_dispatch(h, x.data_ptr(), int(x.shape[0]), send_rows.data_ptr(),
+                                                      send_counts.data_ptr(), _stream(stream)))
+
+
+def lmoe_ep_experts(h: int, recv_rows: torch.Tensor, recv_counts: torch.Tensor, n_recv: int, rows_bound: int,
+                    out_rows: torch.Tensor, stream=None) -> None:
+    """Expert-parallel stage 2: this rank's experts on ``n_recv`` received rows."""
+    _check("lmoe_ep_experts", lib().lmoe_ep_experts(h, recv_rows.data_ptr(), recv_counts.data_ptr(), int(n_recv),
+                                                    int(rows_bound), out_rows.data_ptr(), _stream(stream)))
+
+
+def lmoe_ep_combine(h: int, ret_rows: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """Expert-parallel stage 3: aggregation, W_up and residual into ``y``."""
+    _check("lmoe_ep_combine", lib().lmoe_ep_combine(h, ret_rows.data_ptr(), y.data_ptr(), _stream(stream)))
+
+
 # ------------------------------------------------------------------ convenience owner of a layer
-def make_config(cfg, max_tokens: int) -> lmoe_config:
+def make_config(cfg, max_tokens: int, ep_size: int = 0, ep_rank: int = 0) -> lmoe_config:
     return lmoe_config(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, int(max_tokens), cfg.act, cfg.n_zero,
                        cfg.n_copy, cfg.n_const, cfg.has_proj, cfg.latent_router, getattr(cfg, "shared_m", 0),
-                       getattr(cfg, "expert_fmt", 0))
+                       getattr(cfg, "expert_fmt", 0), int(ep_size), int(ep_rank))
 
 
 class LatentMoE:
@@ -221,10 +245,14 @@ class LatentMoE:
     ``cfg`` is a ``synth.LayerConfig`` (or anything with the same fields),
     ``layer`` the dict of CPU tensors from ``synth.make_layer``.  With a
     block-scaled ``cfg.expert_fmt`` the bf16 W1 / W2 are encoded on the device
-    by ``lmoe_mx_encode_weights`` and only the encodings are kept.
+    by ``lmoe_mx_encode_weights`` and only the encodings are kept.  With
+    ``ep_size`` > 1 the handle is one rank of an expert-parallel layer:
+    ``layer['w1']`` / ``layer['w2']`` must then hold that rank's experts only
+    (see ``expert_parallel``).
     """
 
-    def __init__(self, cfg, layer: Dict[str, torch.Tensor], max_tokens: int, device: str = "cuda"):
+    def __init__(self, cfg, layer: Dict[str, torch.Tensor], max_tokens: int, device: str = "cuda",
+                 ep_size: int = 0, ep_rank: int = 0):
         self.cfg = cfg
         self.device = torch.device(device)
         self.max_tokens = int(max_tokens)
@@ -238,7 +266,7 @@ class LatentMoE:
                 for k in ("w1", "w2"):
                     self.w[k], self.w[k + "_scales"] = lmoe_mx_encode_weights(self.w[k], fmt)
                 torch.cuda.synchronize(self.device)
-        self.c = make_config(cfg, self.max_tokens)
+        self.c = make_config(cfg, self.max_tokens, ep_size, ep_rank)
         nbytes = lmoe_workspace_bytes(self.c)
         if nbytes == 0:
             raise LmoeError("lmoe_workspace_bytes", -2)

@@ -82,7 +82,11 @@ def test_null_handle_calls_are_rejected():
     assert L.lmoe_last_error(None) == -1
     assert L.lmoe_set_profiling(None, 1, 1) == -1
     L.lmoe_destroy(None)
-    assert lmoe.lmoe_num_phases() == 10
+    assert L.lmoe_ep_dispatch(None, None, 1, None, None, None) == -1
+    assert L.lmoe_ep_experts(None, None, None, 1, 1, None, None) == -1
+    assert L.lmoe_ep_combine(None, None, None, None) == -1
+    assert lmoe.lmoe_num_phases() == 11
+    assert lmoe.lmoe_phase_name(10) == "ep_regroup"
     assert [lmoe.lmoe_phase_name(i) for i in range(3)] == ["router_proj_gemm", "topk_softmax", "dispatch"]
 
 
@@ -120,3 +124,17 @@ def test_block_scaled_config_and_encoder_checks():
     assert L.lmoe_mx_encode_weights(None, 128, 128, 1, 0x100, 0x100, None) == -1
     assert L.lmoe_mx_encode_weights(0x108, 128, 128, 1, 0x100, 0x100, None) == -1
     assert L.lmoe_mx_encode_weights(0x100, 0, 128, 1, None, None, None) == 0
+
+
+def test_expert_parallel_config_checks():
+    wl = synth.WORKLOADS["nemotron_prefill"]          # 512 FFN experts, top-22
+    one = lmoe.lmoe_workspace_bytes(lmoe.make_config(wl, 8192))
+    ep8 = lmoe.lmoe_workspace_bytes(lmoe.make_config(wl, 8192, ep_size=8, ep_rank=7))
+    # the expert side holds up to 8 ranks x 8192 tokens x 22 rows, each a latent row and a hidden row
+    assert ep8 > one + 7 * 8192 * 22 * (1024 + 1024) * 2
+    assert lmoe.lmoe_workspace_bytes(lmoe.make_config(wl, 8192, ep_size=1)) == one
+    for ep, rank in ((3, 0), (8, 8), (8, -1), (-1, 0), (0, 1), (1, 1), (2048, 0), (1024, 0)):
+        assert lmoe.lmoe_workspace_bytes(lmoe.make_config(wl, 8192, ep_size=ep, ep_rank=rank)) == 0, (ep, rank)
+    # block-scaled experts are not split; the expert-side capacity must stay below 2^30 rows
+    assert lmoe.lmoe_workspace_bytes(lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp8"], 32, ep_size=2)) == 0
+    assert lmoe.lmoe_workspace_bytes(lmoe.make_config(wl, 1 << 25, ep_size=8)) == 0
