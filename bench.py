@@ -4,11 +4,15 @@ One step = one full layer forward (router GEMM, top-K' + softmax, counting
 sort, expert up / down GEMMs, combine, up-projection + residual) over one
 batch of seeded synthetic tokens, with weights and inputs resident in HBM.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference] [--ep]
 
 Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank runs an
 independent replica of the layer on its own tokens (the layer shards by
 tokens with no exchange step), so per-GPU work is fixed: weak scaling.
+With --ep the ranks instead split the FFN experts (expert parallelism): each
+rank routes its own tokens and the latent rows cross ranks by NCCL all-to-all
+before and after the experts; with one rank nothing moves and the step times
+the three stages of that forward alone.
 """
 from __future__ import annotations
 
@@ -201,7 +205,40 @@ def phase_units(cfg, stats, T, phase):
         return 2.0 * T * (g + 1) * d * ms, 2.0 * ((g + 1) * d * ms + T * (d + ms) + T * (ms + 2 * d))
     if phase == "combine":
         return 2.0 * T * cfg.top_k * L, 2.0 * (rows_tc + rows_st) * L + 2.0 * T * L
+    if phase == "ep_regroup":  # three launches: counts, rows to expert-major order (read + write), and back
+        return 0.0, 2.0 * 2 * 2 * (rows_tc + rows_st) * L / 3
     return 0.0, 0.0
+
+
+def rooflines(cfg, stats, T, phases, peaks, step_ms):
+    """The dominant kernel's roofline (from its phase time per launch) and the whole step's, plus the number of
+    the library's kernel launches per step."""
+    launches = sum(n for _, n in phases.values())
+    dom = max(phases, key=lambda k: phases[k][0])
+    dom_ms, dom_n = phases[dom]
+    flops, nbytes = phase_units(cfg, stats, T, dom)
+    per_launch_ms = dom_ms / max(dom_n, 1)
+    intensity = flops / max(nbytes, 1.0)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if "gemm" in dom and intensity >= ridge:
+        roof = {"bound": "tensor", "achieved": flops / (per_launch_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": nbytes / (per_launch_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["kernel"] = dom
+    roof["launch_ms"] = per_launch_ms
+    roof["algorithmic_per_launch"] = {"flops": flops, "bytes": nbytes}
+    roof["traffic"] = NCU_TRAFFIC.get((cfg.name, dom))
+    roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "")
+
+    F, B, F_eff = layer_work(cfg, stats, T)
+    t_f, t_b = F_eff / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9)
+    t_roof = max(t_f, t_b)
+    layer_roof = {"flops": F, "bytes": B, "t_roof_us": t_roof * 1e6, "t_step_us": step_ms * 1e3,
+                  "frac": t_roof / (step_ms / 1e3), "bound": "tensor" if t_f >= t_b else "hbm"}
+    return roof, layer_roof, launches
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -304,36 +341,119 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
                "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
                "d2h_bytes_per_step": int(yh.numel() * yh.element_size()), "ms_per_step": e2e_ms / steps}
 
-    # ---------------------------------------------------------------- roofline of the dominant kernel
-    launches = sum(n for _, n in phases.values())
-    dom = max(phases, key=lambda k: phases[k][0])
-    dom_ms, dom_n = phases[dom]
-    flops, nbytes = phase_units(cfg, stats, T, dom)
-    per_launch_ms = dom_ms / max(dom_n, 1)
-    intensity = flops / max(nbytes, 1.0)
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if "gemm" in dom and intensity >= ridge:
-        roof = {"bound": "tensor", "achieved": flops / (per_launch_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": nbytes / (per_launch_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["kernel"] = dom
-    roof["launch_ms"] = per_launch_ms
-    roof["algorithmic_per_launch"] = {"flops": flops, "bytes": nbytes}
-    roof["traffic"] = NCU_TRAFFIC.get((cfg.name, dom))
-    roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "")
-
-    F, B, F_eff = layer_work(cfg, stats, T)
-    t_f, t_b = F_eff / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9)
-    t_roof = max(t_f, t_b)
-    layer_roof = {"flops": F, "bytes": B, "t_roof_us": t_roof * 1e6, "t_step_us": ms_max / steps * 1e3,
-                  "frac": t_roof / (ms_max / steps / 1e3), "bound": "tensor" if t_f >= t_b else "hbm"}
+    roof, layer_roof, launches = rooflines(cfg, stats, T, phases, peaks, ms_max / steps)
     mod.close()
     roof["kernel_timed_ms_per_step"] = ms_profiled / steps
     return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
             "e2e": e2e, "clocks": clk, "stats": stats}
+
+
+def run_ep(cfg, steps, warmup, rank, world, device, peaks):
+    """Expert-parallel steps: this rank holds n_ffn / world experts and routes its own tokens.
+
+    Rows cross ranks by NCCL all-to-all; with one rank nothing moves. A step includes the one host wait of the
+    exchange (the counts that size it).
+    """
+    from latent_mixture_experts_gemm_b200 import expert_parallel as xp
+    torch.cuda.set_device(device)
+    layer, xs = setup_layer(cfg, rank, device)
+    T = cfg.tokens
+    rk = xp.ExpertParallelLatentMoE(cfg, layer, max_tokens=T, ep_size=world, ep_rank=rank, device=f"cuda:{device}")
+    xd = [x.to(f"cuda:{device}") for x in xs]
+    yd = torch.empty_like(xd[0])
+    stream = torch.cuda.current_stream()
+    dev = torch.device(f"cuda:{device}")
+    barrier = lambda: dist_barrier(world)  # noqa: E731
+    max_over_ranks = lambda v: dist_max(v, world, dev)  # noqa: E731
+
+    def check(where):
+        status = rk.last_error()
+        if status != 0:
+            raise RuntimeError(f"device error {where}: {lmoe.lmoe_status_string(status)}")
+
+    # expert-side routing statistics (rows this rank's experts received) and the rows sent to other ranks
+    acc, sent_away = {}, 0.0
+    nl = cfg.n_ffn // world
+    for xb in xd:
+        rk.forward(xb, yd)
+        torch.cuda.synchronize()
+        for k, v in lmoe.lmoe_routing_stats(rk.mod.h).items():
+            acc[k] = acc.get(k, 0) + v / len(xd)
+        sc = rk.send_counts.cpu().view(world, nl).sum(1)
+        sent_away += float(sc.sum() - sc[rank]) / len(xd)
+    stats = acc
+    for i in range(warmup):
+        rk.forward(xd[i % N_INPUT_BATCHES], yd)
+    torch.cuda.synchronize()
+    check("during warm-up")
+
+    clocks = ClockSampler(_smi_id(device))
+    clocks.start()
+    time.sleep(0.3)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(steps):
+        rk.forward(xd[i % N_INPUT_BATCHES], yd)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = ev0.elapsed_time(ev1)
+    clk = clocks.stop()
+    check("in the timed region")
+    ms_max = max_over_ranks(ms)
+
+    lmoe.lmoe_set_profiling(rk.mod.h, True, steps)
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(steps):
+        rk.forward(xd[i % N_INPUT_BATCHES], yd)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms_profiled = ev0.elapsed_time(ev1)
+    phases = lmoe.lmoe_phase_times(rk.mod.h)
+    lmoe.lmoe_set_profiling(rk.mod.h, False)
+    check("in the kernel-timed region")
+
+    # end to end: pinned host tokens in, host output back, every step
+    xh = [x.pin_memory() for x in xs]
+    yh = torch.empty_like(xh[0]).pin_memory()
+    xin = torch.empty_like(xd[0])
+
+    def host_step(i):
+        xin.copy_(xh[i % N_INPUT_BATCHES], non_blocking=True)
+        rk.forward(xin, yd)
+        yh.copy_(yd, non_blocking=True)
+
+    for i in range(warmup):
+        host_step(i)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(steps):
+        host_step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    check("in the end-to-end region")
+    e2e = {"value": world * T * steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
+           "d2h_bytes_per_step": int(yh.numel() * yh.element_size()), "ms_per_step": e2e_ms / steps}
+
+    roof, layer_roof, launches = rooflines(cfg, stats, T, phases, peaks, ms_max / steps)
+    roof["kernel_timed_ms_per_step"] = ms_profiled / steps
+    exchange = {"ranks": world, "rows_sent_to_other_ranks_per_step": sent_away,
+                "bytes_over_nvlink_per_step": 2 * 2 * sent_away * cfg.latent,
+                "collective": "NCCL all_to_all_single (counts, rows, rows back)" if world > 1 else "none (one rank)"}
+    rk.close()
+    return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
+            "e2e": e2e, "clocks": clk, "stats": stats, "exchange": exchange}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
@@ -421,6 +541,7 @@ def main():
     ap.add_argument("--impl", default="lmoe", choices=["lmoe", "reference"])
     ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -446,9 +567,12 @@ def main():
                                  device_id=torch.device(f"cuda:{local}"))
     peaks = load_peaks()
     try:
-        res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks)
+        if args.ep:
+            res = run_ep(cfg, args.steps, args.warmup, rank, world, local, peaks)
+        else:
+            res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks)
         secondary = None
-        if not args.no_secondary and args.workload != SECONDARY_WORKLOAD:
+        if not args.ep and not args.no_secondary and args.workload != SECONDARY_WORKLOAD:
             sc = synth.WORKLOADS[SECONDARY_WORKLOAD]
             s_steps = max(3, min(args.steps, 20))
             r2 = run_gpu(sc, s_steps, args.warmup, rank, world, local, peaks, with_e2e=False, with_clocks=False)
@@ -471,6 +595,10 @@ def main():
                 "routing": res["stats"]}
         if secondary is not None:
             line["secondary"] = secondary
+        if args.ep:
+            line["config"]["parallelism"] = (f"ep{world}: each rank holds {cfg.n_ffn // world} of the {cfg.n_ffn} "
+                                             "FFN experts and routes its own tokens")
+            line["exchange"] = res["exchange"]
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)

@@ -209,12 +209,13 @@ LMOE_API const char *lmoe_phase_name(int phase);
 
 /*
  * Sizes of the last forward's routing, read back from the device (blocking;
- * synchronise first).  out8[0] rows routed to FFN experts, [1] FFN experts
- * with at least one row, [2] tensor-core M-tiles, [3] experts on the
- * weight-streaming path, [4] rows on that path, [5] experts on the grouped
- * tensor-core path, [6] rows on that path, [7] the row threshold the forward
- * used (see lmoe_set_small_rows).  Used to compute the algorithmic work of a
- * forward.
+ * synchronise first).  After lmoe_ep_experts they describe the rows that
+ * stage received for this rank's experts instead.  out8[0] rows routed to
+ * FFN experts, [1] FFN experts with at least one row, [2] tensor-core
+ * M-tiles, [3] experts on the weight-streaming path, [4] rows on that path,
+ * [5] experts on the grouped tensor-core path, [6] rows on that path, [7] the
+ * row threshold the forward used (see lmoe_set_small_rows).  Used to compute
+ * the algorithmic work of a forward.
  */
 LMOE_API int lmoe_routing_stats(lmoe_handle *h, int32_t *out8);
 

@@ -455,6 +455,7 @@ struct lmoe_handle {
     // expert-parallel forward in progress: the dispatch's x and T (ep_T < 0: none)
     const void* ep_x = nullptr;
     int ep_T = -1;
+    bool stats_ep = false;  // the header's row / tile counts are those of the last experts stage
     unsigned long long timeout_ns = 1000000000ull;
     // weight descriptors: router/projection operands for both column tiles, expert weights, workspace operands
     CUtensorMap wdown64{}, wdown256{}, wr64{}, wr256{}, wup64{}, wup256{}, w1{}, w2{};
@@ -930,6 +931,7 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     const bool proj = c.has_proj != 0;
     const int small = choose_small(h, T);
     h->last_small = small;
+    h->stats_ep = false;
     __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
     int st = run_front(h, x, T, s, rows, small);
     if (st != LMOE_OK) return st;
@@ -1143,7 +1145,14 @@ int lmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const int32_t* recv_c
     const lmoe_config& c = h->c;
     if (c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
     if (n_recv < 0 || static_cast<size_t>(n_recv) > h->p.ep_cap) return LMOE_ERR_TOO_MANY_TOKENS;
-    if (n_recv == 0) return LMOE_OK;
+    if (n_recv == 0) {  // nothing to compute; the routing statistics show an empty stage
+        cudaStream_t s0 = static_cast<cudaStream_t>(stream);
+        if (cudaMemsetAsync(h->at<int>(h->p.ep_counts), 0, static_cast<size_t>(h->n_local) * 4, s0) != cudaSuccess ||
+            cudaMemsetAsync(h->at<int>(h->p.hdr) + HDR_ROWS, 0, 3 * 4, s0) != cudaSuccess)
+            return LMOE_ERR_CUDA;
+        h->stats_ep = true;
+        return LMOE_OK;
+    }
     if (rows_bound < 1) return LMOE_ERR_INVALID_ARG;
     if (recv_rows == nullptr || recv_counts == nullptr || out_rows == nullptr || !aligned16(recv_rows) ||
         !aligned16(recv_counts) || !aligned16(out_rows))
@@ -1153,6 +1162,7 @@ int lmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const int32_t* recv_c
     const int ep = ep_ranks(c), nl = h->n_local, L = c.latent;
     const int small = choose_small(h, rows_bound);
     h->last_small = small;
+    h->stats_ep = true;
     int* hdr = h->at<int>(p.hdr);
     int* src_off = h->at<int>(p.ep_src);
     int* dst_base = h->at<int>(p.ep_dst);
@@ -1283,12 +1293,15 @@ const char* lmoe_phase_name(int phase) { return (phase >= 0 && phase < PH_COUNT)
 int lmoe_routing_stats(lmoe_handle* h, int32_t* out8) {
     if (h == nullptr || out8 == nullptr) return LMOE_ERR_INVALID_ARG;
     int hdr[HDR_WORDS];
-    std::vector<int> counts(h->n_tot);
+    // after an expert-parallel experts stage: the local experts' received rows; else the forward's routing
+    const int n_ffn = h->stats_ep ? h->n_local : h->c.n_experts;
+    std::vector<int> counts(n_ffn);
     if (cudaMemcpy(hdr, h->at<int>(h->p.hdr), sizeof hdr, cudaMemcpyDeviceToHost) != cudaSuccess ||
-        cudaMemcpy(counts.data(), h->at<int>(h->p.counts), counts.size() * 4, cudaMemcpyDeviceToHost) != cudaSuccess)
+        cudaMemcpy(counts.data(), h->at<int>(h->stats_ep ? h->p.ep_counts : h->p.counts), counts.size() * 4,
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
         return LMOE_ERR_CUDA;
     int touched = 0, st_experts = 0, st_rows = 0, tc_experts = 0, tc_rows = 0;
-    for (int e = 0; e < h->c.n_experts; ++e) {
+    for (int e = 0; e < n_ffn; ++e) {
         const int n = counts[e];
         touched += n > 0;
         if (n > 0 && n <= h->last_small) {

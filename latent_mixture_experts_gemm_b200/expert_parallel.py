@@ -28,16 +28,18 @@ from __future__ import annotations
 
 from typing import Dict, List, Optional, Tuple
 
+import numpy as np
 import torch
 import torch.distributed as dist
 
 from . import lmoe
 
 
-def split_plan(send_counts: torch.Tensor, recv_counts: torch.Tensor, ep: int) -> Tuple[List[int], List[int], int, int, int]:
+def split_plan(send_counts, recv_counts, ep: int) -> Tuple[List[int], List[int], int, int, int]:
     """Host-side sizes of one exchange.
 
-    The inputs are the count matrices ``[ep, n_local]`` on the host: what this
+    The inputs are the count matrices ``[ep, n_local]`` on the host (CPU
+    tensors or arrays, any shape of ep * n_local entries): what this
     rank sends to each rank's experts, and what each rank sends to this rank's
     experts. Returns a tuple of:
     * ``in_splits``: rows sent to each rank;
@@ -45,11 +47,11 @@ def split_plan(send_counts: torch.Tensor, recv_counts: torch.Tensor, ep: int) ->
     * ``n_send``, ``n_recv``: their totals;
     * ``rows_bound``: the most rows any local expert receives.
     """
-    sc = send_counts.reshape(ep, -1).to(torch.int64)
-    rc = recv_counts.reshape(ep, -1).to(torch.int64)
-    in_splits = [int(v) for v in sc.sum(1)]
-    out_splits = [int(v) for v in rc.sum(1)]
-    rows_bound = int(rc.sum(0).max()) if rc.numel() else 0
+    sc = np.asarray(send_counts, dtype=np.int64).reshape(ep, -1)
+    rc = np.asarray(recv_counts, dtype=np.int64).reshape(ep, -1)
+    in_splits = sc.sum(1).tolist()
+    out_splits = rc.sum(1).tolist()
+    rows_bound = int(rc.sum(0).max()) if rc.size else 0
     return in_splits, out_splits, sum(in_splits), sum(out_splits), rows_bound
 
 
@@ -93,8 +95,10 @@ def ep_forward(stages, exchange, x: torch.Tensor, y: Optional[torch.Tensor] = No
     """
     send_rows, send_counts = stages.dispatch(x)
     recv_counts = exchange.counts(send_counts)
-    host = torch.stack([send_counts, recv_counts]).cpu()  # the forward's one wait on the device
-    in_splits, out_splits, n_send, n_recv, rows_bound = split_plan(host[0], host[1], exchange.world)
+    n = send_counts.numel()
+    both = send_counts if recv_counts is send_counts else torch.cat([send_counts, recv_counts])
+    host = both.cpu().numpy()  # the forward's one wait on the device
+    in_splits, out_splits, n_send, n_recv, rows_bound = split_plan(host[:n], host[-n:], exchange.world)
     recv = exchange.rows(stages.recv_buffer(n_recv), send_rows[:n_send], out_splits, in_splits)
     out = stages.experts(recv, recv_counts, n_recv, rows_bound)
     ret = exchange.rows(stages.ret_buffer(n_send), out, in_splits, out_splits)
