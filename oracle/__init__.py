@@ -45,6 +45,12 @@ def lib():
         L.oracle_mx_quantize.restype = ctypes.c_int
         L.oracle_mx_dequantize.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, P]
         L.oracle_mx_dequantize.restype = ctypes.c_int
+        L.oracle_nv_tensor_scale.argtypes = [P, ctypes.c_longlong]
+        L.oracle_nv_tensor_scale.restype = ctypes.c_float
+        L.oracle_nv_quantize.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_float, P, P]
+        L.oracle_nv_quantize.restype = ctypes.c_int
+        L.oracle_nv_dequantize.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_float, P]
+        L.oracle_nv_dequantize.restype = ctypes.c_int
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_set_num_threads.argtypes = [ctypes.c_int]
         _lib = L
@@ -145,8 +151,8 @@ def dispatch(idx: np.ndarray, n_total: int):
     return counts, offsets, perm, inv
 
 
-#: MX block formats of the expert weights (``expert_fmt``)
-FMT_BF16, FMT_MXFP8, FMT_MXFP4 = 0, 1, 2
+#: block-scaled formats of the expert weights (``expert_fmt``)
+FMT_BF16, FMT_MXFP8, FMT_MXFP4, FMT_NVFP4 = 0, 1, 2, 3
 
 
 def mx_quantize(w: torch.Tensor, fmt: int):
@@ -174,4 +180,37 @@ def mx_dequantize(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray
     out = np.empty((rows, K), np.float64)
     if lib().oracle_mx_dequantize(c.ctypes.data, s.ctypes.data, rows, K, int(fmt), out.ctypes.data) != 0:
         raise ValueError("oracle_mx_dequantize rejected its arguments")
+    return out
+
+
+def nv_tensor_scale(w: torch.Tensor) -> float:
+    """NVFP4 fp32 tensor scale of a bf16 tensor: amax / (6 * 448), 1 when all zero."""
+    wb = _bits(w.reshape(-1))
+    return float(lib().oracle_nv_tensor_scale(wb.ctypes.data, wb.size))
+
+
+def nv_quantize(w: torch.Tensor, g: float):
+    """NVFP4 encoding of a bf16 matrix [rows, K] (K a multiple of 16) with tensor scale ``g``.
+
+    Returns ``(codes, scales)``: uint8 [rows, K] E2M1 codes, one per byte, and
+    uint8 [rows, K/16] E4M3 block-scale bytes.
+    """
+    w2 = w.reshape(-1, w.shape[-1])
+    rows, K = int(w2.shape[0]), int(w2.shape[1])
+    wb = _bits(w2)
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, max(K // 16, 1)), np.uint8)
+    if lib().oracle_nv_quantize(wb.ctypes.data, rows, K, float(g), codes.ctypes.data, scales.ctypes.data) != 0:
+        raise ValueError("oracle_nv_quantize rejected its arguments")
+    return codes, scales
+
+
+def nv_dequantize(codes: np.ndarray, scales: np.ndarray, g: float) -> np.ndarray:
+    """The fp64 values an NVFP4 encoding from :func:`nv_quantize` stands for."""
+    c = np.ascontiguousarray(codes, dtype=np.uint8)
+    s = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = c.shape
+    out = np.empty((rows, K), np.float64)
+    if lib().oracle_nv_dequantize(c.ctypes.data, s.ctypes.data, rows, K, float(g), out.ctypes.data) != 0:
+        raise ValueError("oracle_nv_dequantize rejected its arguments")
     return out

@@ -43,8 +43,10 @@
  *      and W2_e are first encoded in that MX format (see the MX section
  *      below) and used at their encoded values; the inputs of both expert
  *      matrices (z, and the activation h) are stored in bf16 and then
- *      encoded in MXFP8 before the multiply.  The router, the projections
- *      and the shared expert stay in bf16.
+ *      encoded in MXFP8 before the multiply.  With expert_fmt = NVFP4 the
+ *      weights and both inputs are NVFP4-encoded instead (see the NVFP4
+ *      section).  The router, the projections and the shared expert stay in
+ *      bf16.
  *
  * Everything is computed in double precision on the bf16 inputs widened
  * exactly; nothing is rounded in between except the MX encodings of step 9
@@ -75,11 +77,11 @@ typedef struct {
     int32_t has_proj;      /* 1: W_down / W_up present */
     int32_t latent_router; /* 1: gate reads z instead of x */
     int32_t shared_m;      /* hidden width of the shared expert at d (0: none) */
-    int32_t expert_fmt;    /* 0 bf16 expert weights, 1 MXFP8, 2 MXFP4 */
+    int32_t expert_fmt;    /* 0 bf16 expert weights, 1 MXFP8, 2 MXFP4, 3 NVFP4 */
 } oracle_cfg;
 
 enum { ORACLE_ACT_RELU2 = 0, ORACLE_ACT_SWIGLU = 1, ORACLE_ACT_IDENTITY = 2 };
-enum { ORACLE_FMT_BF16 = 0, ORACLE_FMT_MXFP8 = 1, ORACLE_FMT_MXFP4 = 2 };
+enum { ORACLE_FMT_BF16 = 0, ORACLE_FMT_MXFP8 = 1, ORACLE_FMT_MXFP4 = 2, ORACLE_FMT_NVFP4 = 3 };
 
 static double widen(uint16_t h)
 {
@@ -241,25 +243,121 @@ static void mx_activation(const double *v, int n, double *out)
     }
 }
 
-/* An MX-encoded weight matrix: codes [rows, in_dim], scales [rows, in_dim/32],
+/* ------------------------------------------------------------------ NVFP4
+ *
+ * The pages name NVFP4 only: Nemotron 3 Super trains in it (the training
+ * note of the outlook section).  The definition used is NVIDIA's published
+ * two-level one:
+ *   - elements are E2M1 (as for MXFP4), codes one per byte;
+ *   - a block is 16 consecutive values along K; it shares one positive E4M3
+ *     scale sb (a byte with the sign bit clear);
+ *   - a whole tensor shares one fp32 scale g.  A weight matrix takes
+ *     g = amax / (6 * 448): the block that holds the matrix's largest
+ *     magnitude then gets the largest E4M3 scale.  An all-zero matrix takes
+ *     g = 1.  Here each expert's W1_e and each W2_e is one tensor.  The
+ *     activations take g = 1 (reading R16);
+ *   - sb = E4M3(amax_block / (g * 6)), nearest even, saturated at 448;
+ *   - element = E2M1(v / (sb * g)), nearest even, saturated at 6;
+ *   - a block whose scale rounds to zero encodes zeros;
+ *   - the value of an element is element * sb * g.
+ * The products g * 6 and sb * g and the two quotients are taken in fp32:
+ * they decide integer codes, and the kernels take the same steps in fp32.
+ */
+
+/* fp32 tensor scale of a bf16 tensor of n values: amax / (6 * 448), or 1 when all are zero. */
+float oracle_nv_tensor_scale(const uint16_t *w, long long n)
+{
+    float amax = 0.0f;
+    for (long long i = 0; i < n; ++i) {
+        const float a = (float)fabs(widen(w[i]));
+        amax = a > amax ? a : amax;
+    }
+    return amax == 0.0f ? 1.0f : amax / 2688.0f;
+}
+
+/* Encode one block of 16 bf16-exact values with tensor scale g. */
+static void nv_block(const double *v, float g, uint8_t *codes, uint8_t *scale)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        const float a = (float)fabs(v[i]);
+        amax = a > amax ? a : amax;
+    }
+    const float d = g * 6.0f;
+    const float x = amax / d;
+    const double sb = round_elem((double)x, 0); /* E4M3: nearest even, saturated at 448 */
+    *scale = elem_code(sb, 0, 0);
+    const float sg = (float)sb * g;
+    for (int i = 0; i < 16; ++i) {
+        if (sb == 0.0) {
+            codes[i] = 0;
+            continue;
+        }
+        const float q = (float)v[i] / sg;
+        codes[i] = elem_code(round_elem(fabs((double)q), 1), signbit(q) != 0, 1);
+    }
+}
+
+/* NVFP4 encoding of a bf16 matrix [rows, K] (K a multiple of 16) with tensor
+ * scale g > 0: codes [rows, K] one per byte (E2M1), scales [rows, K/16] as
+ * E4M3 bytes.  Returns 0, or -1 on bad arguments. */
+int oracle_nv_quantize(const uint16_t *w, int rows, int K, float g, uint8_t *codes, uint8_t *scales)
+{
+    if (rows < 0 || K < 16 || K % 16 != 0 || !(g > 0.0f)) return -1;
+#pragma omp parallel for schedule(static)
+    for (int r = 0; r < rows; ++r) {
+        double v[16];
+        for (int b = 0; b < K / 16; ++b) {
+            for (int i = 0; i < 16; ++i) v[i] = widen(w[(size_t)r * K + b * 16 + i]);
+            nv_block(v, g, codes + (size_t)r * K + b * 16, scales + (size_t)r * (K / 16) + b);
+        }
+    }
+    return 0;
+}
+
+/* The values an NVFP4 encoding stands for: out = elem(code) * e4m3(scale) * g. */
+int oracle_nv_dequantize(const uint8_t *codes, const uint8_t *scales, int rows, int K, float g, double *out)
+{
+    if (rows < 0 || K < 16 || K % 16 != 0) return -1;
+    for (size_t i = 0; i < (size_t)rows * K; ++i)
+        out[i] = elem_value(codes[i], 1) * elem_value(scales[i / 16], 0) * (double)g;
+    return 0;
+}
+
+/* An activation vector as NVFP4 expert GEMMs read it: stored in bf16, then NVFP4-encoded with g = 1. */
+static void nv_activation(const double *v, int n, double *out)
+{
+    uint8_t codes[16], scale;
+    double blk[16];
+    for (int b = 0; b < n / 16; ++b) {
+        for (int i = 0; i < 16; ++i) blk[i] = round_bf16(v[b * 16 + i]);
+        nv_block(blk, 1.0f, codes, &scale);
+        for (int i = 0; i < 16; ++i) out[b * 16 + i] = elem_value(codes[i], 1) * elem_value(scale, 0);
+    }
+}
+
+/* A block-scaled weight matrix: codes [rows, in_dim], scales [rows, in_dim / block],
  * with the value of every element code and of every scale byte tabulated
- * (elem_value and 2^(byte - 127): the same numbers, looked up). */
+ * (elem_value, and 2^(byte - 127) for MX or the E4M3 value for NVFP4: the
+ * same numbers, looked up), and the tensor scale g (1 for MX). */
 typedef struct {
     const uint8_t *codes;
     const uint8_t *scales;
     const double *elem; /* 256 entries */
-    const double *pow2; /* 256 entries */
+    const double *sval; /* 256 entries */
+    int block;          /* 32 (MX) or 16 (NVFP4) */
+    double g;
 } mx_matrix;
 
-/* out[o] = sum_i value(W[o, i]) * v[i] for an MX-encoded W */
+/* out[o] = sum_i value(W[o, i]) * v[i] for a block-scaled W */
 static void matvec_mx(int out_dim, int in_dim, mx_matrix W, const double *v, double *out)
 {
     for (int o = 0; o < out_dim; ++o) {
         const uint8_t *row = W.codes + (size_t)o * in_dim;
-        const uint8_t *sc = W.scales + (size_t)o * (in_dim / 32);
+        const uint8_t *sc = W.scales + (size_t)o * (in_dim / W.block);
         double s = 0.0;
-        for (int i = 0; i < in_dim; ++i) s += W.elem[row[i]] * W.pow2[sc[i / 32]] * v[i];
-        out[o] = s;
+        for (int i = 0; i < in_dim; ++i) s += W.elem[row[i]] * W.sval[sc[i / W.block]] * v[i];
+        out[o] = s * W.g;
     }
 }
 
@@ -346,7 +444,8 @@ static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t 
     const int L = c->latent, m = c->m;
     const int up_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * m : m;
     if (mx1) {
-        mx_activation(z, L, zq);
+        if (c->expert_fmt == ORACLE_FMT_NVFP4) nv_activation(z, L, zq);
+        else mx_activation(z, L, zq);
         matvec_mx(up_rows, L, *mx1, zq, u);
     } else {
         matvec(up_rows, L, w1e, z, u);
@@ -363,7 +462,8 @@ static void ffn_expert(const oracle_cfg *c, const uint16_t *w1e, const uint16_t 
         }
     }
     if (mx2) {
-        mx_activation(h, m, hq);
+        if (c->expert_fmt == ORACLE_FMT_NVFP4) nv_activation(h, m, hq);
+        else mx_activation(h, m, hq);
         matvec_mx(L, m, *mx2, hq, o);
     } else {
         matvec(L, m, w2e, h, o);
@@ -400,26 +500,45 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
     const int fdim = c->latent_router ? L : d;
     const int up_rows = c->act == ORACLE_ACT_SWIGLU ? 2 * m : m;
     const int fmt = c->expert_fmt;
-    if (fmt != ORACLE_FMT_BF16 && fmt != ORACLE_FMT_MXFP8 && fmt != ORACLE_FMT_MXFP4) return -1;
-    if (fmt != ORACLE_FMT_BF16 && (L % 32 != 0 || m % 32 != 0)) return -1;
+    if (fmt != ORACLE_FMT_BF16 && fmt != ORACLE_FMT_MXFP8 && fmt != ORACLE_FMT_MXFP4 && fmt != ORACLE_FMT_NVFP4)
+        return -1;
+    const int nv = fmt == ORACLE_FMT_NVFP4;
+    const int blk = nv ? 16 : 32; /* block length along K */
+    if (fmt != ORACLE_FMT_BF16 && (L % blk != 0 || m % blk != 0)) return -1;
     int bad = 0;
 
     /* step 9: encode the FFN experts' weights once (they are the layer's stored weights) */
     uint8_t *c1 = NULL, *s1 = NULL, *c2 = NULL, *s2 = NULL;
-    double elem_tab[256], pow2_tab[256];
+    float *g1 = NULL, *g2 = NULL; /* NVFP4: tensor scale of each expert's W1_e / W2_e */
+    double elem_tab[256], sval_tab[256];
     for (int i = 0; i < 256; ++i) {
-        elem_tab[i] = fmt == ORACLE_FMT_MXFP4 ? (i < 16 ? elem_value((uint8_t)i, 1) : 0.0) : elem_value((uint8_t)i, 0);
-        pow2_tab[i] = ldexp(1.0, i - 127);
+        const int e2m1 = fmt == ORACLE_FMT_MXFP4 || nv;
+        elem_tab[i] = e2m1 ? (i < 16 ? elem_value((uint8_t)i, 1) : 0.0) : elem_value((uint8_t)i, 0);
+        sval_tab[i] = nv ? elem_value((uint8_t)i, 0) : ldexp(1.0, i - 127);
     }
     if (fmt != ORACLE_FMT_BF16) {
         const size_t n1 = (size_t)c->n_ffn * up_rows * L, n2 = (size_t)c->n_ffn * L * m;
         c1 = (uint8_t *)malloc(n1 > 0 ? n1 : 1);
-        s1 = (uint8_t *)malloc(n1 / 32 > 0 ? n1 / 32 : 1);
+        s1 = (uint8_t *)malloc(n1 / blk > 0 ? n1 / blk : 1);
         c2 = (uint8_t *)malloc(n2 > 0 ? n2 : 1);
-        s2 = (uint8_t *)malloc(n2 / 32 > 0 ? n2 / 32 : 1);
-        if (!c1 || !s1 || !c2 || !s2 || oracle_mx_quantize(w1, c->n_ffn * up_rows, L, fmt, c1, s1) != 0 ||
-            oracle_mx_quantize(w2, c->n_ffn * L, m, fmt, c2, s2) != 0) {
-            free(c1); free(s1); free(c2); free(s2);
+        s2 = (uint8_t *)malloc(n2 / blk > 0 ? n2 / blk : 1);
+        g1 = (float *)malloc(sizeof(float) * (size_t)(c->n_ffn > 0 ? c->n_ffn : 1));
+        g2 = (float *)malloc(sizeof(float) * (size_t)(c->n_ffn > 0 ? c->n_ffn : 1));
+        int enc_bad = !c1 || !s1 || !c2 || !s2 || !g1 || !g2;
+        if (!enc_bad && !nv) {
+            enc_bad = oracle_mx_quantize(w1, c->n_ffn * up_rows, L, fmt, c1, s1) != 0 ||
+                      oracle_mx_quantize(w2, c->n_ffn * L, m, fmt, c2, s2) != 0;
+            for (int e = 0; e < c->n_ffn; ++e) g1[e] = g2[e] = 1.0f;
+        }
+        for (int e = 0; !enc_bad && nv && e < c->n_ffn; ++e) {
+            const size_t o1 = (size_t)e * up_rows * L, o2 = (size_t)e * L * m;
+            g1[e] = oracle_nv_tensor_scale(w1 + o1, (long long)up_rows * L);
+            g2[e] = oracle_nv_tensor_scale(w2 + o2, (long long)L * m);
+            enc_bad = oracle_nv_quantize(w1 + o1, up_rows, L, g1[e], c1 + o1, s1 + o1 / 16) != 0 ||
+                      oracle_nv_quantize(w2 + o2, L, m, g2[e], c2 + o2, s2 + o2 / 16) != 0;
+        }
+        if (enc_bad) {
+            free(c1); free(s1); free(c2); free(s2); free(g1); free(g2);
             return -1;
         }
     }
@@ -484,11 +603,14 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
                     mx_matrix m1 = {0}, m2 = {0};
                     if (fmt != ORACLE_FMT_BF16) {
                         m1.codes = c1 + (size_t)e * up_rows * L;
-                        m1.scales = s1 + (size_t)e * up_rows * (L / 32);
+                        m1.scales = s1 + (size_t)e * up_rows * (L / blk);
                         m2.codes = c2 + (size_t)e * L * m;
-                        m2.scales = s2 + (size_t)e * L * (m / 32);
+                        m2.scales = s2 + (size_t)e * L * (m / blk);
                         m1.elem = m2.elem = elem_tab;
-                        m1.pow2 = m2.pow2 = pow2_tab;
+                        m1.sval = m2.sval = sval_tab;
+                        m1.block = m2.block = blk;
+                        m1.g = g1[e];
+                        m2.g = g2[e];
                     }
                     ffn_expert(c, w1 + (size_t)e * up_rows * L, w2 + (size_t)e * L * m,
                                fmt != ORACLE_FMT_BF16 ? &m1 : NULL, fmt != ORACLE_FMT_BF16 ? &m2 : NULL, z, zq, u, h,
@@ -536,7 +658,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
         free(su); free(sh); free(so); free(zq); free(hq);
         free(xt); free(z); free(zr); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
     }
-    free(c1); free(s1); free(c2); free(s2);
+    free(c1); free(s1); free(c2); free(s2); free(g1); free(g2);
     return bad ? -1 : 0;
 }
 
