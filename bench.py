@@ -137,12 +137,14 @@ def dist_max(v: float, world: int, device: torch.device) -> float:
 
 
 # ----------------------------------------------------------------------------- algorithmic work
-#: bytes per stored expert weight: bf16; MXFP8 (E4M3 + one E8M0 byte per 32); MXFP4 (E2M1 + one per 32)
-WEIGHT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 0.5 + 1.0 / 32}
-#: bytes per element of the expert GEMMs' token operands (MXFP8 with block-scaled experts)
-ACT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 1.0 + 1.0 / 32}
-#: tensor-core rate of the block-scaled expert GEMMs relative to bf16 (the nominal fp8 : bf16 ratio, 4.5 : 2.25)
-MX_RATE = 2.0
+#: bytes per stored expert weight: bf16; MXFP8 (E4M3 + one E8M0 byte per 32); MXFP4 (E2M1 + one per 32);
+#: NVFP4 (E2M1 + one E4M3 byte per 16; the fp32 scale per expert matrix is negligible)
+WEIGHT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 0.5 + 1.0 / 32, 3: 0.5 + 1.0 / 16}
+#: bytes per element of the expert GEMMs' token operands (MXFP8 with MX experts, NVFP4 with NVFP4 experts)
+ACT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 1.0 + 1.0 / 32, 3: 0.5 + 1.0 / 16}
+#: tensor-core rate of the expert GEMMs relative to bf16: the nominal fp8 : bf16 ratio (4.5 : 2.25) for the
+#: MX kinds (E2M1 weights meet E4M3 inputs there), fp4 : bf16 (9 : 2.25) for NVFP4
+EXPERT_RATE = {0: 1.0, 1: 2.0, 2: 2.0, 3: 4.0}
 
 
 #: DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of that kernel as it is now:
@@ -172,7 +174,7 @@ def layer_work(cfg, stats, T):
     if ms:
         F += 2 * T * (g + 1) * d * ms
         B += 2 * (g + 1) * d * ms
-    F_eff = F + fe / (MX_RATE if fmt else 1.0)
+    F_eff = F + fe / EXPERT_RATE[fmt]
     return float(F + fe), float(B), float(F_eff)
 
 
@@ -512,12 +514,13 @@ def run_reference(args, cfg, rank, world):
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
-EXPERT_FORMATS = ["bf16", "mxfp8 (e4m3 weights and expert inputs)", "mxfp4 (e2m1 weights, mxfp8 expert inputs)"]
+EXPERT_FORMATS = ["bf16", "mxfp8 (e4m3 weights and expert inputs)", "mxfp4 (e2m1 weights, mxfp8 expert inputs)",
+                  "nvfp4 (e2m1 weights and expert inputs, e4m3 scale per 16, fp32 scale per expert matrix)"]
 
 
 def compute_dtype(cfg):
     """The arithmetic types the path computes in: bf16 tensor-core GEMMs, plus block-scaled expert GEMMs."""
-    return ["bf16", "bf16+mxfp8", "bf16+mxfp4/mxfp8"][cfg.expert_fmt]
+    return ["bf16", "bf16+mxfp8", "bf16+mxfp4/mxfp8", "bf16+nvfp4"][cfg.expert_fmt]
 
 
 def workload_config(cfg):

@@ -27,7 +27,10 @@
  * name MXFP4 as the Kimi K3 serving format, in the comparison table of "Two
  * Teams, Two Practices"), and the rows those matrices multiply (z_t, and
  * act(W1_e z_t)) are encoded in MXFP8 from their bf16 values before the
- * multiply; see lmoe_mx_encode_weights for the format and layout.
+ * multiply; see lmoe_mx_encode_weights for the format and layout.  With
+ * LMOE_FMT_NVFP4 (the pages name it as Nemotron 3 Super's training format,
+ * in the training note of the outlook section) the weights and those rows
+ * are NVFP4; see lmoe_nvfp4_encode_weights.
  *
  * Conventions for every entry point:
  *   - all matrices are row-major; bf16 tensors are passed as `void *` (IEEE
@@ -75,6 +78,7 @@ extern "C" {
 #define LMOE_FMT_BF16 0  /* expert weights in bf16 */
 #define LMOE_FMT_MXFP8 1 /* E4M3 elements, one E8M0 scale per 32 along K */
 #define LMOE_FMT_MXFP4 2 /* E2M1 elements, one E8M0 scale per 32 along K */
+#define LMOE_FMT_NVFP4 3 /* E2M1 elements, one E4M3 scale per 16 along K, one fp32 scale per expert matrix */
 
 /*
  * Layer shape.  Constraints (else LMOE_ERR_UNSUPPORTED_SHAPE): d, latent and m
@@ -82,8 +86,8 @@ extern "C" {
  * n_total = n_experts + n_zero + n_copy + n_const <= 1024; n_experts >= 1;
  * max_tokens >= 1; has_proj == 0 requires latent == d; shared_m is 0 or a
  * multiple of 64 up to 16384.  A block-scaled expert_fmt also requires
- * latent and m to be multiples of 128 and max_tokens <= 32 (the decode
- * regime, where every expert streams its weights).
+ * latent and m to be multiples of 128 (256 for NVFP4) and max_tokens <= 32
+ * (the decode regime, where every expert streams its weights).
  * Expert parallelism (see lmoe_ep_dispatch): ep_size 0 or 1 means none;
  * otherwise 2 <= ep_size <= n_experts, n_experts a multiple of ep_size,
  * 0 <= ep_rank < ep_size, expert_fmt == LMOE_FMT_BF16, and
@@ -126,8 +130,11 @@ typedef struct lmoe_weights {
     const void *const_vecs;   /* [n_const, latent]; may be NULL when n_const == 0 */
     const void *w_shared1;    /* [g*shared_m, d] (gate rows first when gated); NULL when shared_m == 0 */
     const void *w_shared2;    /* [d, shared_m]; NULL when shared_m == 0 */
-    const void *w1_scales;    /* block-scaled only: E8M0 scale atoms of w1 (lmoe_mx_encode_weights); else NULL */
-    const void *w2_scales;    /* block-scaled only: E8M0 scale atoms of w2; else NULL */
+    const void *w1_scales;    /* block-scaled only: scale atoms of w1 (lmoe_mx_encode_weights or
+                                 lmoe_nvfp4_encode_weights: E8M0 or E4M3 bytes); else NULL */
+    const void *w2_scales;    /* block-scaled only: scale atoms of w2; else NULL */
+    const float *w1_gscale;   /* NVFP4 only: fp32 [n_local] tensor scale of each expert's W1_e; else NULL */
+    const float *w2_gscale;   /* NVFP4 only: fp32 [n_local] tensor scale of each expert's W2_e; else NULL */
 } lmoe_weights;
 
 /*
@@ -315,6 +322,37 @@ LMOE_API int lmoe_dispatch_noalloc(const int32_t *idx, int32_t T, int32_t top_k,
  */
 LMOE_API int lmoe_mx_encode_weights(const void *w, int64_t rows, int32_t K, int32_t fmt, void *codes, void *scales,
                                     void *stream);
+
+/*
+ * NVFP4 encoding of bf16 weight matrices, for lmoe_weights.w1 / w2 with
+ * expert_fmt = LMOE_FMT_NVFP4.  It follows NVIDIA's published two-level
+ * definition (the pages name the format only).  Each of the n_mats matrices
+ * (an expert's W1_e or W2_e, rows_per_mat rows of K values) takes one fp32
+ * tensor scale g = amax / (6 * 448), or 1 when all its values are zero.  Each
+ * row is split into blocks of 16 consecutive values along K; a block shares
+ * one positive E4M3 scale sb = E4M3(amax_block / (g * 6)), and each element
+ * is E2M1(v / (sb * g)); both round to nearest even and saturate (448, 6),
+ * and a block whose scale is zero encodes zeros.  The products g * 6 and
+ * sb * g and both quotients are fp32 operations.  An element stands for
+ * e2m1 * sb * g.
+ *
+ *   w             device bf16 [n_mats * rows_per_mat, K]
+ *   n_mats        1 .. 65535;  rows_per_mat a multiple of 128;  K a multiple
+ *                 of 64 (the layer's kernels need multiples of 256)
+ *   codes         device, [n_mats * rows_per_mat, K/2] bytes, two elements
+ *                 per byte, element 2i in the low nibble of byte i
+ *   scales        device, rows * K / 16 bytes, in 512-byte atoms
+ *                 [rows/128][K/64][32][16]: byte (r, c) of atom (R, G) holds
+ *                 the scale of row 128R + 32(c/4) + r, block 4G + c%4 (one
+ *                 atom per 64 values of 128 rows: the order in which the
+ *                 tensor cores read the scales of one K = 64 MMA)
+ *   gscale        device fp32 [n_mats]: the tensor scales (written)
+ *
+ * Bad sizes: LMOE_ERR_UNSUPPORTED_SHAPE; a NULL or misaligned pointer:
+ * LMOE_ERR_INVALID_ARG.  Asynchronous on `stream`; deterministic.
+ */
+LMOE_API int lmoe_nvfp4_encode_weights(const void *w, int32_t n_mats, int64_t rows_per_mat, int32_t K, void *codes,
+                                       void *scales, float *gscale, void *stream);
 
 /*
  * Expert parallelism: the forward split at the two all-to-all exchanges that

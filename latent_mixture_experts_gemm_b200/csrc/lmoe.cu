@@ -21,6 +21,7 @@
 #include "../../include/lmoe.h"
 #include "moe_kernels.cuh"
 #include "mx.cuh"
+#include "nv.cuh"
 #include "ep.cuh"
 #include "tc_gemm.cuh"
 #include "tc_swap.cuh"
@@ -87,6 +88,20 @@ bool make_map_e2m1(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) 
     return r == CUDA_SUCCESS;
 }
 
+// NVFP4 token scale chunks, planar [chunks][rows][16] bytes; a box is 4 chunks x 32 rows x 16 bytes (the
+// four 512-byte scale atoms of one 256-element stage, first 32 rows).
+bool make_map_nv_sf(CUtensorMap* m, const void* base, uint64_t rows, uint64_t chunks) {
+    if (!load_encode() || rows == 0) return false;
+    cuuint64_t dims[3] = {16, rows, chunks};
+    cuuint64_t strides[2] = {16, rows * 16};
+    cuuint32_t box[3] = {16, 32, 4};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 int n_total(const lmoe_config& c) { return c.n_experts + c.n_zero + c.n_copy + c.n_const; }
@@ -104,8 +119,10 @@ bool config_ok(const lmoe_config& c) {
     if (c.latent_router != 0 && c.latent_router != 1) return false;
     if (!c.has_proj && c.latent != c.d) return false;
     if (c.shared_m != 0 && !dim_ok(c.shared_m)) return false;
-    if (c.expert_fmt < LMOE_FMT_BF16 || c.expert_fmt > LMOE_FMT_MXFP4) return false;
-    if (c.expert_fmt != LMOE_FMT_BF16 && (c.latent % 128 != 0 || c.m % 128 != 0 || c.max_tokens > SMALL_MAX))
+    if (c.expert_fmt < LMOE_FMT_BF16 || c.expert_fmt > LMOE_FMT_NVFP4) return false;
+    // block-scaled experts stream their weights (decode batches) in stages of 128 (MX) or 256 (NVFP4) elements
+    const int stage = c.expert_fmt == LMOE_FMT_NVFP4 ? 256 : 128;
+    if (c.expert_fmt != LMOE_FMT_BF16 && (c.latent % stage != 0 || c.m % stage != 0 || c.max_tokens > SMALL_MAX))
         return false;
     if (c.ep_size < 0 || c.ep_size > 1024) return false;
     if (c.ep_size > 1) {  // expert parallelism: whole local expert sets, bf16 experts
@@ -135,7 +152,8 @@ int n_local_experts(const lmoe_config& c) { return c.n_experts / ep_ranks(c); }
 
 struct Plan {
     size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
-        partial, hs, s2, partial2, rows8, rows_sf, h8, h_sf, xin, yout, ep_map, ep_src, ep_dst, ep_counts,
+        partial, hs, s2, partial2, rows4, rows_sf4, h4, h_sf4, rows8, rows_sf, h8, h_sf, xin, yout, ep_map, ep_src,
+        ep_dst, ep_counts,
         ep_offsets, total;
     size_t rows_cap;  // rows of the expert-side buffers: a forward's slots, or the most an experts stage receives
     size_t ep_cap;    // rows an expert-parallel experts stage may receive
@@ -188,7 +206,12 @@ Plan make_plan(const lmoe_config& c) {
         p.s2 = take(T * d * 2);
         p.partial2 = take(static_cast<size_t>(kFewTokenMaxSplits) * srows * kFewTokenRows * 4);
     }
-    if (c.expert_fmt != LMOE_FMT_BF16) {  // MXFP8 token operands of the expert GEMMs: codes and block scales
+    if (c.expert_fmt == LMOE_FMT_NVFP4) {  // NVFP4 token operands: packed codes, planar scale chunks
+        p.rows4 = take(R * L / 2);
+        p.rows_sf4 = take(L / 64 * R * 16);
+        p.h4 = take(R * m / 2);
+        p.h_sf4 = take(m / 64 * R * 16);
+    } else if (c.expert_fmt != LMOE_FMT_BF16) {  // MXFP8 token operands of the expert GEMMs: codes and block scales
         p.rows8 = take(R * L);
         p.rows_sf = take(R * mx_ld_sf(static_cast<int>(L)));
         p.h8 = take(R * m);
@@ -278,8 +301,18 @@ bool set_mx_attr() {
                                 MxCfg<EPI, W4>::SMEM_BYTES) == cudaSuccess;
 }
 
+template <int EPI, bool QOUT>
+bool set_nv_attr() {
+    return cudaFuncSetAttribute(tc_swap_nv_kernel<EPI, QOUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                NvCfg<EPI>::SMEM_BYTES) == cudaSuccess;
+}
+
 bool set_all_smem_attrs() {
     bool ok = true;
+    ok &= set_nv_attr<EPI_BF16, true>();
+    ok &= set_nv_attr<EPI_RELU2, true>();
+    ok &= set_nv_attr<EPI_SWIGLU, true>();
+    ok &= set_nv_attr<EPI_BF16, false>();
     ok &= set_pair_attr<EPI_BF16>();
     ok &= set_pair_attr<EPI_RELU2>();
     ok &= set_pair_attr<EPI_SWIGLU>();
@@ -424,6 +457,18 @@ void launch_mx(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs
 }
 
 // Block-scaled expert phase: the up GEMM (activation, MXFP8 re-encoding) or the down GEMM (bf16 out).
+template <int EPI, bool QOUT>
+void launch_nv(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf, const NvArgs& a, int grid,
+               cudaStream_t s) {
+    launch(tc_swap_nv_kernel<EPI, QOUT>, grid, 192, NvCfg<EPI>::SMEM_BYTES, s, w, x, xsf, a);
+}
+void launch_nv_phase(bool up, int epi, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf,
+                     const NvArgs& a, int grid, cudaStream_t s) {
+    if (!up) launch_nv<EPI_BF16, false>(w, x, xsf, a, grid, s);
+    else if (epi == EPI_RELU2) launch_nv<EPI_RELU2, true>(w, x, xsf, a, grid, s);
+    else if (epi == EPI_SWIGLU) launch_nv<EPI_SWIGLU, true>(w, x, xsf, a, grid, s);
+    else launch_nv<EPI_BF16, true>(w, x, xsf, a, grid, s);
+}
 void launch_mx_phase(bool up, int epi, bool w4, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf,
                      const MxArgs& a, int grid, cudaStream_t s) {
     if (!up) {
@@ -469,6 +514,9 @@ struct lmoe_handle {
     CUtensorMap ws1_64{}, ws1_256{}, ws2_64{}, ws2_256{}, ws1_128{}, ws2_128{}, a_hs{}, hs16{}, hs32{};
     // block-scaled experts: weight codes (128 x 128 boxes) and the MXFP8 token operands with their scales
     CUtensorMap w1q{}, w2q{}, rows8{}, rows_sf{}, h8{}, h_sf{};
+    // NVFP4 experts: packed weight codes (128 x 128-byte boxes), token codes (32 x 128-byte boxes) and the
+    // token scale chunks (4 chunks x 32 rows x 16 bytes)
+    CUtensorMap w1n{}, w2n{}, rows4{}, rows_sf4{}, h4{}, h_sf4{};
     // TMA store maps of bf16 GEMM outputs (32-row x 64-column boxes): hidden rows, expert outputs, z
     CUtensorMap o_h{}, o_rows{}, o_z{};
     cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
@@ -699,7 +747,10 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
         const size_t sm = (static_cast<size_t>(2 * nwords) * nt + nt) * 4;
         launch(dispatch_small_kernel, 1, 1024, sm, s, idx, T, K, nt, c.n_experts, small, counts, offsets, mt_list,
                small_list, perm, inv, hdr);
-        if (mx)
+        if (c.expert_fmt == LMOE_FMT_NVFP4)
+            launch(nv_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
+                   feat, L, L, h->at<uint8_t>(p.rows4), h->at<uint8_t>(p.rows_sf4), static_cast<int>(c.max_tokens) * K);
+        else if (mx)
             launch(mx_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
                    feat, L, L, h->at<uint8_t>(p.rows8), L, h->at<uint8_t>(p.rows_sf), mx_ld_sf(L));
         else
@@ -762,7 +813,26 @@ int run_experts(lmoe_handle* h, int small, bool need_tc, cudaStream_t s) {
             launch_gemm<256, EPI_BF16>(h->a_rows, h->w1, h->w1, a, h->num_sms, s, &h->o_h);
         }
     }
-    if (mx) {
+    if (c.expert_fmt == LMOE_FMT_NVFP4) {
+        PhaseScope ps(h, PH_UP_STREAM, s, 1);
+        NvArgs a{};
+        a.K = L;
+        a.n_wtiles = m / 128;
+        a.list = small_list;
+        a.count = hdr + HDR_NSMALL;
+        a.w_rows_per_expert = h->g * m;
+        a.up_offset = m;
+        a.w_sf = static_cast<const uint8_t*>(h->w.w1_scales);
+        a.w_g = h->w.w1_gscale;
+        a.n_out = m;
+        a.out4 = h->at<uint8_t>(p.h4);
+        a.out_sf = h->at<uint8_t>(p.h_sf4);
+        a.sf_rows = static_cast<int>(c.max_tokens) * c.top_k;
+        a.err = hdr + HDR_ERR;
+        a.timeout_ns = h->timeout_ns;
+        const int epi = c.act == LMOE_ACT_SWIGLU ? EPI_SWIGLU : (c.act == LMOE_ACT_RELU2 ? EPI_RELU2 : EPI_BF16);
+        launch_nv_phase(true, epi, h->w1n, h->rows4, h->rows_sf4, a, h->num_sms, s);
+    } else if (mx) {
         PhaseScope ps(h, PH_UP_STREAM, s, 1);
         MxArgs a{};
         a.K = L;
@@ -813,7 +883,24 @@ int run_experts(lmoe_handle* h, int small, bool need_tc, cudaStream_t s) {
         a.n_tiles = (L + 255) / 256;
         launch_gemm<256, EPI_BF16>(h->a_h, h->w2, h->w2, a, h->num_sms, s, &h->o_rows);
     }
-    if (mx) {
+    if (c.expert_fmt == LMOE_FMT_NVFP4) {
+        PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
+        NvArgs a{};
+        a.K = m;
+        a.n_wtiles = L / 128;
+        a.list = small_list;
+        a.count = hdr + HDR_NSMALL;
+        a.w_rows_per_expert = L;
+        a.up_offset = 0;
+        a.w_sf = static_cast<const uint8_t*>(h->w.w2_scales);
+        a.w_g = h->w.w2_gscale;
+        a.n_out = L;
+        a.out = rows;
+        a.ld_out = L;
+        a.err = hdr + HDR_ERR;
+        a.timeout_ns = h->timeout_ns;
+        launch_nv_phase(false, EPI_BF16, h->w2n, h->h4, h->h_sf4, a, h->num_sms, s);
+    } else if (mx) {
         PhaseScope ps(h, PH_DOWN_STREAM, s, 1);
         MxArgs a{};
         a.K = m;
@@ -986,9 +1073,11 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     if (c.n_const > 0 && w->const_vecs == nullptr) return LMOE_ERR_INVALID_ARG;
     if (c.shared_m > 0 && (w->w_shared1 == nullptr || w->w_shared2 == nullptr)) return LMOE_ERR_INVALID_ARG;
     const void* ptrs[] = {w->w_router, w->router_bias, w->w_down, w->w_up, w->w1, w->w2, w->const_vecs,
-                          w->w_shared1, w->w_shared2, w->w1_scales, w->w2_scales};
+                          w->w_shared1, w->w_shared2, w->w1_scales, w->w2_scales, w->w1_gscale, w->w2_gscale};
     for (const void* q : ptrs)
         if (!aligned16(q)) return LMOE_ERR_INVALID_ARG;
+    if (c.expert_fmt == LMOE_FMT_NVFP4 && (w->w1_gscale == nullptr || w->w2_gscale == nullptr))
+        return LMOE_ERR_INVALID_ARG;
     if (c.expert_fmt != LMOE_FMT_BF16) {
         if (w->w1_scales == nullptr || w->w2_scales == nullptr) return LMOE_ERR_INVALID_ARG;
         // the packed E2M1 copy reads from 32-byte aligned rows
@@ -1040,6 +1129,14 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
         ok &= make_map(&h->w2, w->w2, w2_rows, m, m, 256);
         ok &= make_map(&h->w1s, w->w1, w1_rows, L, L, 128);
         ok &= make_map(&h->w2s, w->w2, w2_rows, m, m, 128);
+    } else if (c.expert_fmt == LMOE_FMT_NVFP4) {
+        const uint64_t RT = static_cast<uint64_t>(c.max_tokens) * c.top_k;
+        ok &= make_map_u8(&h->w1n, w->w1, w1_rows, L / 2, L / 2, 128, 128, true);
+        ok &= make_map_u8(&h->w2n, w->w2, w2_rows, m / 2, m / 2, 128, 128, true);
+        ok &= make_map_u8(&h->rows4, h->at<void>(p.rows4), RT, L / 2, L / 2, 128, 32, true);
+        ok &= make_map_u8(&h->h4, h->at<void>(p.h4), RT, m / 2, m / 2, 128, 32, true);
+        ok &= make_map_nv_sf(&h->rows_sf4, h->at<void>(p.rows_sf4), RT, L / 64);
+        ok &= make_map_nv_sf(&h->h_sf4, h->at<void>(p.h_sf4), RT, m / 64);
     } else {
         if (c.expert_fmt == LMOE_FMT_MXFP4) {
             ok &= make_map_e2m1(&h->w1q, w->w1, w1_rows, L);
@@ -1377,6 +1474,30 @@ int lmoe_gemm_bf16(const void* A, const void* B, void* C, int32_t M, int32_t N, 
         a.n_tiles = (N + 63) / 64;
         launch_gemm<64, EPI_BF16>(ma, mb, mb, a, std::min<long long>(sms, static_cast<long long>(m_tiles) * a.n_tiles), s);
     }
+    return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+int lmoe_nvfp4_encode_weights(const void* w, int32_t n_mats, int64_t rows_per_mat, int32_t K, void* codes,
+                              void* scales, float* gscale, void* stream) {
+    if (n_mats < 1 || n_mats > 65535 || rows_per_mat < 128 || rows_per_mat % 128 != 0 || K < 64 || K % 64 != 0 ||
+        static_cast<long long>(n_mats) * rows_per_mat * K > (1LL << 40))
+        return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (w == nullptr || codes == nullptr || scales == nullptr || gscale == nullptr || !aligned16(w) ||
+        !aligned16(codes) || !aligned16(scales) || !aligned16(gscale))
+        return LMOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t* gbits = reinterpret_cast<uint32_t*>(gscale);
+    if (cudaMemsetAsync(gbits, 0, static_cast<size_t>(n_mats) * 4, s) != cudaSuccess) return LMOE_ERR_CUDA;
+    const long long per_mat = rows_per_mat * K;
+    const unsigned gx = static_cast<unsigned>(std::min<long long>((per_mat / 8 + 255) / 256, 256));
+    nv_amax_kernel<<<dim3(gx, static_cast<unsigned>(n_mats)), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(w),
+                                                                          per_mat, gbits);
+    nv_tensor_scale_kernel<<<(n_mats + 255) / 256, 256, 0, s>>>(gbits, n_mats);
+    const long long rows = static_cast<long long>(n_mats) * rows_per_mat;
+    const long long blocks = rows * (K / 16);
+    nv_encode_weights_kernel<<<static_cast<unsigned>((blocks + 255) / 256), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(w), rows, rows_per_mat, K, gscale, static_cast<uint8_t*>(codes),
+        static_cast<uint8_t*>(scales));
     return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 

@@ -366,61 +366,40 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + buf * C::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-            uint32_t g[NT], u[NT], g2[NT], u2[NT];
-            tmem_ld_32x32b_x32(taddr, g);
-            tmem_ld_32x32b_x32(taddr + C::NA * NT, g2);
-            if (C::NA == 2) {
-                tmem_ld_32x32b_x32(taddr + NT, u);
-                tmem_ld_32x32b_x32(taddr + 3 * NT, u2);
+            const bool valid = col < args.n_out;
+            uint8_t* dst8 = QOUT ? args.out8 + static_cast<size_t>(e.y) * args.ld_out8 + col : nullptr;
+            uint8_t* sdst = QOUT ? args.out_sf + static_cast<size_t>(e.y) * args.ld_out_sf + (col >> 7) * 16 + ((col >> 5) & 3)
+                                 : nullptr;
+            __nv_bfloat16* dst = QOUT ? nullptr : args.out + static_cast<size_t>(e.y) * args.ld_out + col;
+            // Only the expert's rows in this tile (e.z, the same for the whole warp), one at a time, each row's
+            // accumulator columns (the two chains) read from tensor memory and added.  A small loop keeps the
+            // epilogue's code small, so the other warps do not stall on instruction fetch.
+            for (int j = 0; j < e.z; ++j) {
+                uint32_t c0, c1, c2 = 0u, c3 = 0u;
+                tmem_ld_32x32b_x1(taddr + j, c0);
+                tmem_ld_32x32b_x1(taddr + C::NA * NT + j, c1);
+                if (C::NA == 2) {
+                    tmem_ld_32x32b_x1(taddr + NT + j, c2);
+                    tmem_ld_32x32b_x1(taddr + 3 * NT + j, c3);
+                }
+                tmem_ld_wait();
+                float a = __uint_as_float(c0) + __uint_as_float(c1);
+                if (EPI == EPI_RELU2) a = act_relu2(a);
+                if (EPI == EPI_SWIGLU) a = act_silu_mul(a, __uint_as_float(c2) + __uint_as_float(c3));
+                if (QOUT) {
+                    // the stored (bf16) activation, its block maximum over the warp (the warp's 32 columns are
+                    // one block), the E8M0 scale, the E4M3 codes; lane 0 writes the block scale
+                    const float v = valid ? __bfloat162float(__float2bfloat16_rn(a)) : 0.f;
+                    const int sx = mx_scale_exp(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v))), 8);
+                    if (valid) dst8[static_cast<size_t>(j) * args.ld_out8] = static_cast<uint8_t>(mx_e4m3(v * mx_exp2i(-sx)));
+                    if (lane == 0) sdst[static_cast<size_t>(j) * args.ld_out_sf] = static_cast<uint8_t>(sx + 127);
+                } else if (valid) {
+                    dst[static_cast<size_t>(j) * args.ld_out] = __float2bfloat16_rn(a);
+                }
             }
-            tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);
-            // the two accumulation chains
-#pragma unroll
-            for (int j = 0; j < NT; ++j) {
-                g[j] = __float_as_uint(__uint_as_float(g[j]) + __uint_as_float(g2[j]));
-                if (C::NA == 2) u[j] = __float_as_uint(__uint_as_float(u[j]) + __uint_as_float(u2[j]));
-            }
-            const bool valid = col < args.n_out;
-            if (QOUT) {
-                // the stored (bf16) activation of each token row; then the 32 block maxima (independent warp
-                // reductions, one per row); then the codes.  Lane j writes row j's block scale.
-                float v[NT];
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    float a = __uint_as_float(g[j]);
-                    if (EPI == EPI_RELU2) a = act_relu2(a);
-                    if (EPI == EPI_SWIGLU) a = act_silu_mul(a, __uint_as_float(u[j]));
-                    v[j] = valid ? __bfloat162float(__float2bfloat16_rn(a)) : 0.f;
-                }
-                uint32_t amax[NT];
-#pragma unroll
-                for (int j = 0; j < NT; ++j) amax[j] = __reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v[j])));
-                uint8_t* dst = args.out8 + static_cast<size_t>(e.y) * args.ld_out8 + col;
-                uint32_t my_scale = 0;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    const int sx = mx_scale_exp(amax[j], 8);
-                    if (lane == j) my_scale = static_cast<uint32_t>(sx + 127);
-                    if (j < e.z && valid) dst[static_cast<size_t>(j) * args.ld_out8] = static_cast<uint8_t>(mx_e4m3(v[j] * mx_exp2i(-sx)));
-                }
-                if (lane < e.z)
-                    args.out_sf[static_cast<size_t>(e.y + lane) * args.ld_out_sf + (col >> 7) * 16 + ((col >> 5) & 3)] =
-                        static_cast<uint8_t>(my_scale);
-            } else if (valid) {
-                __nv_bfloat16* dst = args.out + static_cast<size_t>(e.y) * args.ld_out + col;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    if (j < e.z) {
-                        float v = __uint_as_float(g[j]);
-                        if (EPI == EPI_RELU2) v = act_relu2(v);
-                        if (EPI == EPI_SWIGLU) v = act_silu_mul(v, __uint_as_float(u[j]));
-                        dst[static_cast<size_t>(j) * args.ld_out] = __float2bfloat16_rn(v);
-                    }
-                }
-            }
+            if (lane == 0) mbar_arrive(&tempty[buf]);  // this tile's accumulator is free for the MMA warp
         }
     }
 

@@ -101,6 +101,14 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// 3-D tiled load of the box at (c0, c1, c2) (c0 innermost), completion on `bar`.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1, int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // 1-D bulk copy global -> shared (no tensor map), completion on `bar`.  Both
 // addresses 16-byte aligned, `bytes` a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -203,6 +211,28 @@ __device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t adesc, uint64_
         : "memory");
 }
 
+// Instruction descriptor of an NVFP4 MMA (kind::mxf4nvf4 with 16-element blocks: both operands E2M1,
+// packed two per byte, K-major; E4M3 scales; fp32 accumulate; K = 64 per MMA).  Each MMA reads four
+// scales per row: a whole 32-bit TMEM scale column, so the scale-factor ids stay 0.
+__host__ __device__ constexpr uint32_t umma_idesc_nvf4(int M, int N) {
+    return (1u << 7)                                // A element format: E2M1
+           | (1u << 10)                             // B element format: E2M1
+           | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+           | (static_cast<uint32_t>(M >> 4) << 24); // M / 16; scale format bit 23 = 0: E4M3
+}
+
+// D (+)= (A * SFA) (B * SFB)^T with an E4M3 scale per 16 elements along K, read from TMEM at tmem_sfa /
+// tmem_sfb (K = 64 per MMA: four scales per row).
+__device__ __forceinline__ void umma_nv(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t tmem_sfa, uint32_t tmem_sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
+        : "memory");
+}
+
 // Copy 32 rows x 16 bytes of shared memory into 4 TMEM columns of lanes 0-31,
 // repeated in each of the four 32-lane sub-partitions (the layout the MMA
 // reads its scale factors from).  Ordered before the MMAs this thread issues
@@ -236,6 +266,10 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t ncols) {
 }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i gets row (lane base + i).
+// 32 lanes x 1 32-bit column.
+__device__ __forceinline__ void tmem_ld_32x32b_x1(uint32_t taddr, uint32_t& r) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 "

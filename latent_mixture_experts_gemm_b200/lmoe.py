@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblmoe.so")
 
 LMOE_OK = 0
-LMOE_FMT_BF16, LMOE_FMT_MXFP8, LMOE_FMT_MXFP4 = 0, 1, 2
+LMOE_FMT_BF16, LMOE_FMT_MXFP8, LMOE_FMT_MXFP4, LMOE_FMT_NVFP4 = 0, 1, 2, 3
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_ARG", -2: "LMOE_ERR_UNSUPPORTED_SHAPE", -3: "LMOE_ERR_TOO_MANY_TOKENS",
           -4: "LMOE_ERR_CUDA", -5: "LMOE_ERR_TIMEOUT", -6: "LMOE_ERR_BAD_INDEX", -7: "LMOE_ERR_WORKSPACE",
           -8: "LMOE_ERR_BAD_COUNTS"}
@@ -33,7 +33,8 @@ class lmoe_config(ctypes.Structure):
 
 class lmoe_weights(ctypes.Structure):
     _fields_ = [("w_router", P), ("router_bias", P), ("w_down", P), ("w_up", P), ("w1", P), ("w2", P),
-                ("const_vecs", P), ("w_shared1", P), ("w_shared2", P), ("w1_scales", P), ("w2_scales", P)]
+                ("const_vecs", P), ("w_shared1", P), ("w_shared2", P), ("w1_scales", P), ("w2_scales", P),
+                ("w1_gscale", P), ("w2_gscale", P)]
 
 
 class lmoe_debug(ctypes.Structure):
@@ -80,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
         L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
         L.lmoe_mx_encode_weights.argtypes = [P, ctypes.c_int64, I32, I32, P, P, P]
+        L.lmoe_nvfp4_encode_weights.argtypes = [P, I32, ctypes.c_int64, I32, P, P, P, P]
         L.lmoe_ep_dispatch.argtypes = [P, P, I32, P, P, P]
         L.lmoe_ep_experts.argtypes = [P, P, P, I32, I32, P, P]
         L.lmoe_ep_combine.argtypes = [P, P, P, P]
@@ -232,6 +234,23 @@ def lmoe_ep_combine(h: int, ret_rows: torch.Tensor, y: torch.Tensor, stream=None
     _check("lmoe_ep_combine", lib().lmoe_ep_combine(h, ret_rows.data_ptr(), y.data_ptr(), _stream(stream)))
 
 
+def lmoe_nvfp4_encode_weights(w: torch.Tensor, stream=None):
+    """NVFP4 encoding of a device bf16 tensor of matrices ``[n_mats, rows_per_mat, K]``.
+
+    Returns ``(codes, scales, gscale)`` as new device tensors: codes uint8 [n_mats * rows_per_mat, K/2] (element
+    2i in the low nibble of byte i), scales uint8 in the tensor-core atom order ``include/lmoe.h`` describes,
+    gscale fp32 [n_mats].
+    """
+    n_mats, rows_per_mat, K = (int(v) for v in w.shape)
+    codes = torch.empty((n_mats * rows_per_mat, K // 2), dtype=torch.uint8, device=w.device)
+    scales = torch.empty(n_mats * rows_per_mat * K // 16, dtype=torch.uint8, device=w.device)
+    gscale = torch.empty(n_mats, dtype=torch.float32, device=w.device)
+    _check("lmoe_nvfp4_encode_weights", lib().lmoe_nvfp4_encode_weights(
+        w.data_ptr(), n_mats, rows_per_mat, K, codes.data_ptr(), scales.data_ptr(), gscale.data_ptr(),
+        _stream(stream)))
+    return codes, scales, gscale
+
+
 # ------------------------------------------------------------------ convenience owner of a layer
 def make_config(cfg, max_tokens: int, ep_size: int = 0, ep_rank: int = 0) -> lmoe_config:
     return lmoe_config(cfg.d, cfg.latent, cfg.m, cfg.n_ffn, cfg.top_k, int(max_tokens), cfg.act, cfg.n_zero,
@@ -245,7 +264,8 @@ class LatentMoE:
     ``cfg`` is a ``synth.LayerConfig`` (or anything with the same fields),
     ``layer`` the dict of CPU tensors from ``synth.make_layer``.  With a
     block-scaled ``cfg.expert_fmt`` the bf16 W1 / W2 are encoded on the device
-    by ``lmoe_mx_encode_weights`` and only the encodings are kept.  With
+    (``lmoe_mx_encode_weights``, or ``lmoe_nvfp4_encode_weights`` for NVFP4)
+    and only the encodings are kept.  With
     ``ep_size`` > 1 the handle is one rank of an expert-parallel layer:
     ``layer['w1']`` / ``layer['w2']`` must then hold that rank's experts only
     (see ``expert_parallel``).
@@ -259,9 +279,14 @@ class LatentMoE:
         dev = lambda t: None if t is None else t.to(self.device).contiguous()  # noqa: E731
         self.w = {k: dev(layer.get(k)) for k in ("w_router", "bias", "w_down", "w_up", "w1", "w2", "const_vecs",
                                                   "w_shared1", "w_shared2")}
-        self.w["w1_scales"] = self.w["w2_scales"] = None
+        self.w["w1_scales"] = self.w["w2_scales"] = self.w["w1_gscale"] = self.w["w2_gscale"] = None
         fmt = getattr(cfg, "expert_fmt", 0)
-        if fmt != LMOE_FMT_BF16:
+        if fmt == LMOE_FMT_NVFP4:
+            with torch.cuda.device(self.device):
+                for k in ("w1", "w2"):
+                    self.w[k], self.w[k + "_scales"], self.w[k + "_gscale"] = lmoe_nvfp4_encode_weights(self.w[k])
+                torch.cuda.synchronize(self.device)
+        elif fmt != LMOE_FMT_BF16:
             with torch.cuda.device(self.device):
                 for k in ("w1", "w2"):
                     self.w[k], self.w[k + "_scales"] = lmoe_mx_encode_weights(self.w[k], fmt)
@@ -274,7 +299,7 @@ class LatentMoE:
         self.weights = lmoe_weights(_p(self.w["w_router"]), _p(self.w["bias"]), _p(self.w["w_down"]),
                                     _p(self.w["w_up"]), _p(self.w["w1"]), _p(self.w["w2"]), _p(self.w["const_vecs"]),
                                     _p(self.w["w_shared1"]), _p(self.w["w_shared2"]), _p(self.w["w1_scales"]),
-                                    _p(self.w["w2_scales"]))
+                                    _p(self.w["w2_scales"]), _p(self.w["w1_gscale"]), _p(self.w["w2_gscale"]))
         with torch.cuda.device(self.device):
             self.h = lmoe_create(self.c, self.weights, self.workspace.data_ptr(), nbytes)
 

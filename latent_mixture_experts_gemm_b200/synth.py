@@ -111,6 +111,8 @@ WORKLOADS: Dict[str, LayerConfig] = {
                                   top_k=22, act="relu2", expert_fmt=1, seed=7),
     "nemotron_decode_mxfp4": _cfg(name="nemotron_decode_mxfp4", tokens=32, d=4096, latent=1024, m=1024, n_ffn=512,
                                   top_k=22, act="relu2", expert_fmt=2, seed=8),
+    "nemotron_decode_nvfp4": _cfg(name="nemotron_decode_nvfp4", tokens=32, d=4096, latent=1024, m=1024, n_ffn=512,
+                                  top_k=22, act="relu2", expert_fmt=3, seed=6),
 }
 
 

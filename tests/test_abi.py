@@ -101,8 +101,8 @@ def test_block_scaled_config_and_encoder_checks():
     L = lmoe.lib()
     ok = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp4"], 32)
     assert lmoe.lmoe_workspace_bytes(ok) > lmoe.lmoe_workspace_bytes(lmoe.make_config(synth.WORKLOADS["nemotron_decode"], 32))
-    # block-scaled experts: decode batches only, latent and m whole 128-element stages, formats 0..2
-    for b in (dict(max_tokens=33), dict(latent=192), dict(m=320), dict(expert_fmt=3), dict(expert_fmt=-1)):
+    # block-scaled experts: decode batches only, latent and m whole 128-element stages, formats 0..3
+    for b in (dict(max_tokens=33), dict(latent=192), dict(m=320), dict(expert_fmt=4), dict(expert_fmt=-1)):
         c = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp8"], 32)
         for k, v in b.items():
             setattr(c, k, v)
@@ -138,3 +138,29 @@ def test_expert_parallel_config_checks():
     # block-scaled experts are not split; the expert-side capacity must stay below 2^30 rows
     assert lmoe.lmoe_workspace_bytes(lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp8"], 32, ep_size=2)) == 0
     assert lmoe.lmoe_workspace_bytes(lmoe.make_config(wl, 1 << 25, ep_size=8)) == 0
+
+
+def test_nvfp4_config_and_encoder_checks():
+    L = lmoe.lib()
+    ok = lmoe.make_config(synth.WORKLOADS["nemotron_decode_nvfp4"], 32)
+    assert lmoe.lmoe_workspace_bytes(ok) > 0
+    # NVFP4 experts stream in stages of 256 elements; decode batches only; no expert parallelism
+    for b in (dict(latent=384), dict(m=640), dict(max_tokens=33), dict(expert_fmt=4)):
+        c = lmoe.make_config(synth.WORKLOADS["nemotron_decode_nvfp4"], 32)
+        for k, v in b.items():
+            setattr(c, k, v)
+        assert lmoe.lmoe_workspace_bytes(c) == 0, b
+    assert lmoe.lmoe_workspace_bytes(lmoe.make_config(synth.WORKLOADS["nemotron_decode_nvfp4"], 32, ep_size=2)) == 0
+    # a layer without its tensor scales is rejected before any device work
+    cfg = lmoe.make_config(synth.WORKLOADS["nemotron_decode_nvfp4"], 32)
+    big = lmoe.lmoe_workspace_bytes(cfg)
+    h = ctypes.c_void_p()
+    w = lmoe.lmoe_weights(w_router=0x10000, w_down=0x10000, w_up=0x10000, w1=0x10000, w2=0x10000,
+                          w1_scales=0x20000, w2_scales=0x20000)
+    assert L.lmoe_create(ctypes.byref(cfg), ctypes.byref(w), 0x100000, big, ctypes.byref(h)) == -1
+    assert h.value is None
+    # the encoder checks sizes before pointers
+    assert L.lmoe_nvfp4_encode_weights(0x100, 1, 100, 128, 0x100, 0x100, 0x100, None) == -2
+    assert L.lmoe_nvfp4_encode_weights(0x100, 1, 128, 96, 0x100, 0x100, 0x100, None) == -2
+    assert L.lmoe_nvfp4_encode_weights(0x100, 0, 128, 128, 0x100, 0x100, 0x100, None) == -2
+    assert L.lmoe_nvfp4_encode_weights(None, 1, 128, 128, 0x100, 0x100, 0x100, None) == -1
