@@ -244,14 +244,14 @@ __global__ void __launch_bounds__(192, 1)
             if (!ok) break;
             tc_fence_after();
             const uint32_t taddr = tmem_base + buf * C::ACC_COLS + (static_cast<uint32_t>(quad * 32) << 16);
-            uint32_t g[NT], u[NT];
-            tmem_ld_cols<NT>(taddr, g);
-            if (C::NA == 2) tmem_ld_cols<NT>(taddr + NT, u);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tempty[buf]);  // accumulator copied to registers: release it early
             if (args.partial != nullptr) {
+                // dense split-K projections: every token column's fp32 partial sum
+                uint32_t g[NT];
+                tmem_ld_cols<NT>(taddr, g);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);  // accumulator copied to registers: release it early
                 if (col < args.part_rows) {
                     float4* dst = reinterpret_cast<float4*>(
                         args.partial + (static_cast<size_t>(j.split) * args.part_rows + col) * NT);
@@ -260,17 +260,24 @@ __global__ void __launch_bounds__(192, 1)
                         dst[i] = make_float4(__uint_as_float(g[4 * i]), __uint_as_float(g[4 * i + 1]),
                                              __uint_as_float(g[4 * i + 2]), __uint_as_float(g[4 * i + 3]));
                 }
-            } else if (col < args.n_out) {
+            } else {
+                // experts: only the expert's rows in this tile (e.z, the same for the whole warp), one at a time,
+                // each row's accumulator column(s) read from tensor memory.  A small loop keeps the epilogue's
+                // code small, so the TMA and MMA warps do not stall on instruction fetch.
                 __nv_bfloat16* dst = args.out + static_cast<size_t>(e.y) * args.ld_out + col;
-#pragma unroll
-                for (int j = 0; j < NT; ++j) {
-                    if (j < e.z) {
-                        float v = __uint_as_float(g[j]);
-                        if (EPI == EPI_RELU2) v = act_relu2(v);
-                        if (EPI == EPI_SWIGLU) v = act_silu_mul(v, __uint_as_float(u[j]));
-                        dst[static_cast<size_t>(j) * args.ld_out] = __float2bfloat16_rn(v);
-                    }
+                for (int r = 0; r < e.z; ++r) {
+                    uint32_t gv, uv = 0u;
+                    tmem_ld_32x32b_x1(taddr + r, gv);
+                    if (C::NA == 2) tmem_ld_32x32b_x1(taddr + NT + r, uv);
+                    tmem_ld_wait();
+                    float v = __uint_as_float(gv);
+                    if (EPI == EPI_RELU2) v = act_relu2(v);
+                    if (EPI == EPI_SWIGLU) v = act_silu_mul(v, __uint_as_float(uv));
+                    if (col < args.n_out) dst[static_cast<size_t>(r) * args.ld_out] = __float2bfloat16_rn(v);
                 }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);  // this tile's accumulator is free for the MMA warp
             }
         }
     }
