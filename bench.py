@@ -148,10 +148,13 @@ EXPERT_RATE = {0: 1.0, 1: 2.0, 2: 2.0, 3: 4.0}
 
 
 #: DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of that kernel as it is now:
-#: the expert up stream of the Nemotron-like decode read 817.4 / 792.2 MB and wrote 1.4 / 1.3 MB in two
-#: captured launches.  A kernel that changes drops out of this table until it is captured again.
+#: the expert up stream of the Nemotron-like decode read 817.4 / 792.2 MB and wrote 1.4 / 2.0 MB in two captured
+#: launches; the NVFP4 decode's expert streams read 224.3 / 224.2 MB and wrote 4.2 / 4.5 MB (up / down).  A kernel
+#: that changes drops out of this table until it is captured again.
 NCU_TRAFFIC = {
-    ("nemotron_decode", "expert_up_stream"): 806.1e6,
+    ("nemotron_decode", "expert_up_stream"): 806.5e6,
+    ("nemotron_decode_nvfp4", "expert_up_stream"): 228.5e6,
+    ("nemotron_decode_nvfp4", "expert_down_stream"): 228.8e6,
 }
 
 
