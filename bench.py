@@ -325,6 +325,41 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     if status != 0:
         raise RuntimeError(f"device error in the kernel-timed region: {lmoe.lmoe_status_string(status)}")
 
+    # ---------------------------------------------------------------- the same steps replayed from CUDA graphs
+    # one graph per input batch, each holding one whole forward (its launches and the shared expert's stream)
+    graph = None
+    if with_e2e:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            mod.forward(xd[0], yd)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graphs = []
+        for i in range(N_INPUT_BATCHES):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                mod.forward(xd[i], yd)
+            graphs.append(gr)
+        for i in range(warmup):
+            graphs[i % N_INPUT_BATCHES].replay()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(steps):
+            graphs[i % N_INPUT_BATCHES].replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        g_ms = max_over_ranks(ev0.elapsed_time(ev1))
+        status = mod.last_error()
+        if status != 0:
+            raise RuntimeError(f"device error in the graph-replay region: {lmoe.lmoe_status_string(status)}")
+        graph = {"value": world * T * steps / (g_ms / 1e3), "unit": "tokens/s", "ms_per_step": g_ms / steps,
+                 "launch": "one CUDA graph per forward, replayed"}
+        del graphs
+
     # ---------------------------------------------------------------- end to end through host buffers
     e2e = None
     if with_e2e:
@@ -350,7 +385,7 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     mod.close()
     roof["kernel_timed_ms_per_step"] = ms_profiled / steps
     return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
-            "e2e": e2e, "clocks": clk, "stats": stats}
+            "e2e": e2e, "clocks": clk, "stats": stats, "graph": graph}
 
 
 def run_ep(cfg, steps, warmup, rank, world, device, peaks):
@@ -599,6 +634,8 @@ def main():
                 "clocks": res["clocks"],
                 "phases_ms_per_step": {k: v[0] / args.steps for k, v in res["phases"].items()},
                 "routing": res["stats"]}
+        if res.get("graph") is not None:
+            line["graph_replay"] = res["graph"]
         if secondary is not None:
             line["secondary"] = secondary
         if args.ep:
