@@ -384,6 +384,12 @@ struct FewTokenGemm {
     int ld_resid;
     int act = EPI_BF16;     // activation of segment 0 (EPI_RELU2 / EPI_SWIGLU: gate rows first, then up rows)
     int out_cols0 = -1;     // output columns of segment 0 (default rows0; rows0 / 2 when gated)
+    // router: with topk_idx set, segment 1 holds the router logits, and the reduction also selects each
+    // token's top-K' (bias added) and writes ids and renormalised weights
+    const float* bias = nullptr;
+    int topk = 0;
+    int32_t* topk_idx = nullptr;
+    float* topk_w = nullptr;
 };
 
 template <int NT>
@@ -399,6 +405,27 @@ void launch_few_token_reduce(const FewTokenGemm& g, int T, const float* partial,
     else if (g.act == EPI_SWIGLU) LMOE_REDUCE(EPI_SWIGLU);
     else LMOE_REDUCE(EPI_BF16);
 #undef LMOE_REDUCE
+}
+
+// The router's reduction with the top-K' selection: one block per token (segment 1 = the logits, no
+// activation on segment 0).
+template <int NT>
+void launch_router_reduce_topk(const FewTokenGemm& g, int T, const float* partial, int part_rows, int splits, int t0,
+                               cudaStream_t s) {
+    const int n1 = g.rows1, npl = (n1 + 31) / 32;
+    const size_t smem = static_cast<size_t>(n1) * 4;
+    // T routing blocks, then the z columns at one element per thread
+    const unsigned grid = static_cast<unsigned>(T + (static_cast<long>(g.rows0) * T + 511) / 512);
+#define LMOE_RTOPK(N)                                                                                             \
+    launch(router_reduce_topk_kernel<NT, N>, grid, 512, smem, s, partial, part_rows, splits, T, g.rows0, n1,      \
+           t0 * 128, g.out0, g.ld0, g.out1, g.ld1, g.bias, g.topk, g.topk_idx, g.topk_w)
+    if (npl <= 1) LMOE_RTOPK(1);
+    else if (npl <= 2) LMOE_RTOPK(2);
+    else if (npl <= 4) LMOE_RTOPK(4);
+    else if (npl <= 8) LMOE_RTOPK(8);
+    else if (npl <= 16) LMOE_RTOPK(16);
+    else LMOE_RTOPK(32);
+#undef LMOE_RTOPK
 }
 
 int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_splits, int num_sms, int* err,
@@ -421,10 +448,12 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
     const int grid = std::min(num_sms, (t0 + t1) * splits);
     if (T <= 16) {
         launch_swap<16, EPI_BF16>(*g.w, *g.x16, *g.w2, a, grid, s);
-        launch_few_token_reduce<16>(g, T, partial, a.part_rows, splits, t0, s);
+        if (g.topk_idx != nullptr) launch_router_reduce_topk<16>(g, T, partial, a.part_rows, splits, t0, s);
+        else launch_few_token_reduce<16>(g, T, partial, a.part_rows, splits, t0, s);
     } else {
         launch_swap<32, EPI_BF16>(*g.w, *g.x32, *g.w2, a, grid, s);
-        launch_few_token_reduce<32>(g, T, partial, a.part_rows, splits, t0, s);
+        if (g.topk_idx != nullptr) launch_router_reduce_topk<32>(g, T, partial, a.part_rows, splits, t0, s);
+        else launch_few_token_reduce<32>(g, T, partial, a.part_rows, splits, t0, s);
     }
     return 2;
 }
@@ -663,24 +692,34 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
 
     // ---------------------------------------------------------------- router (+ W_down)
     if (T <= kFewTokenRows) {
-        // few tokens: split-K weight streaming (weights as the 128-row operand) + in-order reduction
+        // few tokens: split-K weight streaming (weights as the 128-row operand), then the in-order reduction,
+        // which also takes each token's top-K' and softmax from its logits (router_reduce_topk_kernel)
         CUtensorMap x16, x32;
         if (!make_map(&x16, x, T, d, d, 16) || !make_map(&x32, x, T, d, d, 32)) return LMOE_ERR_CUDA;
         float* part = h->at<float>(p.partial);
         const bool fused = proj && !c.latent_router;
         const int n_launch = (proj && c.latent_router) ? 4 : 2;
         PhaseScope ps(h, PH_ROUTER, s, n_launch);
+        auto with_topk = [&](FewTokenGemm& r) {
+            r.bias = bias;
+            r.topk = K;
+            r.topk_idx = idx;
+            r.topk_w = wts;
+        };
         if (proj && c.latent_router) {
             FewTokenGemm g{&h->wdown128, &h->wdown128, &x16, &x32, L, 0, d, z, L, nullptr, 0, nullptr, 0};
             launch_few_token(g, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
             FewTokenGemm r{&h->wr128, &h->wr128, &h->z16, &h->z32, 0, nt, L, nullptr, 0, logits, p.ld_logits,
                            nullptr, 0};
+            with_topk(r);
             launch_few_token(r, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
         } else if (fused) {
             FewTokenGemm g{&h->wdown128, &h->wr128, &x16, &x32, L, nt, d, z, L, logits, p.ld_logits, nullptr, 0};
+            with_topk(g);
             launch_few_token(g, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
         } else {
             FewTokenGemm r{&h->wr128, &h->wr128, &x16, &x32, 0, nt, d, nullptr, 0, logits, p.ld_logits, nullptr, 0};
+            with_topk(r);
             launch_few_token(r, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
         }
     } else {
@@ -728,8 +767,8 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
             }
         }
     }
-    // ---------------------------------------------------------------- top-K' + softmax
-    {
+    // ---------------------------------------------------------------- top-K' + softmax (T > 32: its own kernel)
+    if (T > kFewTokenRows) {
         PhaseScope ps(h, PH_TOPK, s, 1);
         const dim3 grid((T + 3) / 4), block(128);  // one warp per token, 4 per block (few tokens: more SMs)
 #define LMOE_TOPK(N) launch(topk_softmax_kernel<N>, grid, block, 0, s, logits, p.ld_logits, bias, T, nt, K, idx, wts)

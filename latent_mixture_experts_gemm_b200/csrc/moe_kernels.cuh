@@ -72,8 +72,10 @@ __device__ __forceinline__ void bitonic_step(uint32_t& k, uint32_t& i, int e, in
 // K'-th largest key (it is the K'-th largest of a subset), so every selected
 // key is among the keys at or above it.  When at most 64 keys qualify, they are
 // sorted outright (64-element warp bitonic sort) and the first K' are taken.
-// Otherwise the exact radix selection below runs.
-template <int NPL>
+// Otherwise the exact radix selection below runs.  SMEM_ROW: the logit row is
+// in shared memory (plain loads) rather than in global memory written by an
+// earlier kernel (read-only-cache loads).
+template <int NPL, bool SMEM_ROW = false>
 __device__ __forceinline__ void topk_one_token(const float* __restrict__ row, const float* __restrict__ bias,
                                                int n_tot, int K, uint32_t* s_key, uint32_t* s_id,
                                                int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
@@ -84,7 +86,7 @@ __device__ __forceinline__ void topk_one_token(const float* __restrict__ row, co
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
         const int e = lane + 32 * i;
-        lv[i] = e < n_tot ? __ldg(row + e) : 0.0f;
+        lv[i] = e < n_tot ? (SMEM_ROW ? row[e] : __ldg(row + e)) : 0.0f;
         bv[i] = (bias != nullptr && e < n_tot) ? __ldg(bias + e) : 0.0f;
     }
     uint32_t key[NPL];
@@ -210,6 +212,56 @@ __global__ void __launch_bounds__(128) topk_softmax_kernel(const float* __restri
     if (t >= T) return;
     topk_one_token<NPL>(logits + static_cast<size_t>(t) * ld, bias, n_tot, K, s_key[warp], s_id[warp],
                         idx_out + static_cast<size_t>(t) * K, w_out + static_cast<size_t>(t) * K);
+}
+
+// Few-token router: the in-order sum of the split-K partials, as
+// swap_reduce_kernel takes it, with the top-K' selection folded in.  Blocks
+// 0 .. T-1 take one token each: its router logits (fp32, also stored), then
+// its top-K' and renormalised softmax by one warp on the logits kept in shared
+// memory.  The blocks after them take the z columns (bf16), one element per
+// thread.  Router GEMM, selection and softmax end in this kernel, with no
+// separate top-K' launch.
+//   z[t][n] = bf16(sum of partial row n), n < n0
+//   logits[t][c] = sum of partial row p1 + c, c < n1
+template <int NT, int NPL>
+__global__ void __launch_bounds__(512) router_reduce_topk_kernel(const float* __restrict__ partial, int part_rows,
+                                                                 int splits, int T, int n0, int n1, int p1,
+                                                                 __nv_bfloat16* __restrict__ out0, int ld0,
+                                                                 float* __restrict__ logits, int ld1,
+                                                                 const float* __restrict__ bias, int K,
+                                                                 int32_t* __restrict__ idx_out,
+                                                                 float* __restrict__ w_out) {
+    pdl_begin();
+    extern __shared__ float s_logit[];  // n1 values
+    __shared__ uint32_t s_key[64], s_id[64];
+    auto reduce = [&](int prow, int t) {  // all split loads in flight together; the sum runs in split order
+        float pv[16];
+#pragma unroll
+        for (int sp = 0; sp < 16; ++sp)
+            pv[sp] = sp < splits ? partial[(static_cast<size_t>(sp) * part_rows + prow) * NT + t] : 0.f;
+        float v = 0.f;
+#pragma unroll
+        for (int sp = 0; sp < 16; ++sp)
+            if (sp < splits) v += pv[sp];
+        return v;
+    };
+    if (static_cast<int>(blockIdx.x) < T) {
+        const int t = blockIdx.x;
+        for (int c = threadIdx.x; c < n1; c += blockDim.x) {
+            const float v = reduce(p1 + c, t);
+            logits[static_cast<size_t>(t) * ld1 + c] = v;
+            s_logit[c] = v;
+        }
+        __syncthreads();
+        if (threadIdx.x < 32)
+            topk_one_token<NPL, true>(s_logit, bias, n1, K, s_key, s_id, idx_out + static_cast<size_t>(t) * K,
+                                      w_out + static_cast<size_t>(t) * K);
+    } else {
+        const long i = static_cast<long>(blockIdx.x - T) * blockDim.x + threadIdx.x;
+        if (i >= static_cast<long>(n0) * T) return;
+        const int n = static_cast<int>(i % n0), t = static_cast<int>(i / n0);
+        out0[static_cast<size_t>(t) * ld0 + n] = __float2bfloat16_rn(reduce(n, t));
+    }
 }
 
 // ============================================================================ dispatch
