@@ -86,8 +86,10 @@ extern "C" {
  * n_total = n_experts + n_zero + n_copy + n_const <= 1024; n_experts >= 1;
  * max_tokens >= 1; has_proj == 0 requires latent == d; shared_m is 0 or a
  * multiple of 64 up to 16384.  A block-scaled expert_fmt also requires
- * latent and m to be multiples of 128 (256 for NVFP4) and max_tokens <= 32
- * (the decode regime, where every expert streams its weights).
+ * latent and m to be multiples of 128 (256 for NVFP4).  Block-scaled experts
+ * always take the weight-streaming GEMM: an expert that received more than 32
+ * rows streams its weights once per 32 rows, so they suit decode batches (at
+ * T <= 32 each touched expert streams once).
  * Expert parallelism (see lmoe_ep_dispatch): ep_size 0 or 1 means none;
  * otherwise 2 <= ep_size <= n_experts, n_experts a multiple of ep_size,
  * 0 <= ep_rank < ep_size, expert_fmt == LMOE_FMT_BF16, and
@@ -222,7 +224,9 @@ LMOE_API const char *lmoe_phase_name(int phase);
  * M-tiles, [3] experts on the weight-streaming path, [4] rows on that path,
  * [5] experts on the grouped tensor-core path, [6] rows on that path, [7] the
  * row threshold the forward used (see lmoe_set_small_rows).  Used to compute
- * the algorithmic work of a forward.
+ * the algorithmic work of a forward.  With block-scaled experts [3] counts the
+ * entries of the weight-streaming list, 32 rows at most each: an expert with
+ * more rows takes several, each streaming its weights.
  */
 LMOE_API int lmoe_routing_stats(lmoe_handle *h, int32_t *out8);
 

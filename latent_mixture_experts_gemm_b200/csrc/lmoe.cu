@@ -122,8 +122,7 @@ bool config_ok(const lmoe_config& c) {
     if (c.expert_fmt < LMOE_FMT_BF16 || c.expert_fmt > LMOE_FMT_NVFP4) return false;
     // block-scaled experts stream their weights (decode batches) in stages of 128 (MX) or 256 (NVFP4) elements
     const int stage = c.expert_fmt == LMOE_FMT_NVFP4 ? 256 : 128;
-    if (c.expert_fmt != LMOE_FMT_BF16 && (c.latent % stage != 0 || c.m % stage != 0 || c.max_tokens > SMALL_MAX))
-        return false;
+    if (c.expert_fmt != LMOE_FMT_BF16 && (c.latent % stage != 0 || c.m % stage != 0)) return false;
     if (c.ep_size < 0 || c.ep_size > 1024) return false;
     if (c.ep_size > 1) {  // expert parallelism: whole local expert sets, bf16 experts
         if (c.n_experts % c.ep_size != 0 || c.ep_rank < 0 || c.ep_rank >= c.ep_size) return false;
@@ -190,7 +189,8 @@ Plan make_plan(const lmoe_config& c) {
     p.perm = take(R * 4);
     p.inv = take(R * 4);
     p.mt_list = take(static_cast<size_t>(p.mt_max) * 16);
-    p.small_list = take(static_cast<size_t>(c.n_experts) * 16);
+    // weight-streaming list: one entry per expert, or (block-scaled experts) one per 32 rows of an expert
+    p.small_list = take((static_cast<size_t>(c.n_experts) + RC / SMALL_MAX + 1) * 16);
     p.rows = take(RC * L * 2);  // gathered expert inputs, then (reused) expert outputs
     p.hbuf = take(RC * m * 2);
     p.yl = c.has_proj ? take(T * L * 2) : 0;
@@ -796,14 +796,21 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
             launch(dispatch_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K,
                    c.n_experts, feat, L, L, rows_dst, L);
     } else {
-        PhaseScope ps(h, PH_DISPATCH, s, 4);
+        PhaseScope ps(h, PH_DISPATCH, s, mx ? 5 : 4);
         uint32_t* bitmap = h->at<uint32_t>(p.bitmap);
         uint32_t* prefix = h->at<uint32_t>(p.prefix);
         launch(dispatch_bitmap_kernel, (nwords + 7) / 8, 256, 8 * nt * 4, s, idx, T, K, nt, bitmap, hdr);
         launch(dispatch_expert_scan_kernel, (nt + 7) / 8, 256, 0, s, bitmap, T, nt, prefix, counts);
         launch(dispatch_offsets_kernel, 1, 1024, 0, s, counts, nt, c.n_experts, small, offsets, mt_list, small_list, hdr);
+        // block-scaled experts: the scatter only places the slots (no bf16 row copy); the gather encodes the rows
         launch(dispatch_scatter_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, T, K, nt, c.n_experts,
-               bitmap, prefix, offsets, feat, L, L, rows_dst, L, perm, inv);
+               bitmap, prefix, offsets, feat, L, mx ? 0 : L, rows_dst, L, perm, inv);
+        if (c.expert_fmt == LMOE_FMT_NVFP4)
+            launch(nv_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
+                   feat, L, L, h->at<uint8_t>(p.rows4), h->at<uint8_t>(p.rows_sf4), static_cast<int>(c.max_tokens) * K);
+        else if (mx)
+            launch(mx_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
+                   feat, L, L, h->at<uint8_t>(p.rows8), L, h->at<uint8_t>(p.rows_sf), mx_ld_sf(L));
     }
     return LMOE_OK;
 }
@@ -1046,9 +1053,13 @@ int run_back(lmoe_handle* h, const __nv_bfloat16* O, const void* x, void* y, int
 int choose_small(const lmoe_handle* h, long rows_bound) {
     int small = h->small_max;
     if (small > 0 && rows_bound <= SMALL_MAX) small = rows_bound <= 16 ? 16 : SMALL_MAX;
-    if (h->c.expert_fmt != LMOE_FMT_BF16) small = SMALL_MAX;  // block-scaled experts always stream (T <= 32)
+    if (h->c.expert_fmt != LMOE_FMT_BF16) small = SMALL_MAX;  // block-scaled experts always stream
     return small;
 }
+
+// The `small_max` the dispatch builds its lists with: block-scaled experts stream whatever their rows, in
+// list entries of at most 32 rows (chunk mode, a negative value); others split by `small`.
+int list_small(const lmoe_handle* h, int small) { return h->c.expert_fmt != LMOE_FMT_BF16 ? -SMALL_MAX : small; }
 
 int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, const lmoe_debug* dbg) {
     const lmoe_config& c = h->c;
@@ -1059,9 +1070,9 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     h->last_small = small;
     h->stats_ep = false;
     __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
-    int st = run_front(h, x, T, s, rows, small);
+    int st = run_front(h, x, T, s, rows, list_small(h, small));
     if (st != LMOE_OK) return st;
-    st = run_experts(h, small, T > small, s);
+    st = run_experts(h, small, c.expert_fmt == LMOE_FMT_BF16 && T > small, s);
     if (st != LMOE_OK) return st;
     st = run_back(h, rows, x, y, T, s);
     if (st != LMOE_OK) return st;
@@ -1437,10 +1448,11 @@ int lmoe_routing_stats(lmoe_handle* h, int32_t* out8) {
                    cudaMemcpyDeviceToHost) != cudaSuccess)
         return LMOE_ERR_CUDA;
     int touched = 0, st_experts = 0, st_rows = 0, tc_experts = 0, tc_rows = 0;
+    const bool all_stream = h->c.expert_fmt != LMOE_FMT_BF16;
     for (int e = 0; e < n_ffn; ++e) {
         const int n = counts[e];
         touched += n > 0;
-        if (n > 0 && n <= h->last_small) {
+        if (n > 0 && (all_stream || n <= h->last_small)) {
             ++st_experts;
             st_rows += n;
         } else if (n > h->last_small) {

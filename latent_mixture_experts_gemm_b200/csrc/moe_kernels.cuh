@@ -356,9 +356,24 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 
 // Offsets (exclusive scan of counts), the tensor-core M-tile list (experts
 // with more than `small_max` rows, split in 128-row tiles) and the
-// weight-streaming list (experts with 1..small_max rows).  Body for a single
-// block of 1024 threads, thread e holding expert e's row count c (0 for
-// e >= n_tot); returns offsets[e].
+// weight-streaming list (experts with 1..small_max rows).  A negative
+// small_max selects chunk mode instead (block-scaled experts, which only
+// stream): every FFN expert with rows enters the weight-streaming list as
+// entries of at most -small_max rows each, and the M-tile list stays empty.
+// Body for a single block of 1024 threads, thread e holding expert e's row
+// count c (0 for e >= n_tot); returns offsets[e].
+
+// Weight-streaming list entries of expert e with c rows starting at sorted row off.
+__device__ __forceinline__ int stream_entries(bool ffn, int c, int small_max) {
+    if (!ffn || c <= 0) return 0;
+    if (small_max < 0) return (c - small_max - 1) / (-small_max);
+    return c <= small_max ? 1 : 0;
+}
+__device__ __forceinline__ void write_stream_entries(int4* __restrict__ small_list, int pos, int n, int e, int off,
+                                                     int c, int small_max) {
+    const int chunk = small_max < 0 ? -small_max : c;
+    for (int i = 0; i < n; ++i) small_list[pos + i] = make_int4(e, off + chunk * i, min(chunk, c - chunk * i), 0);
+}
 __device__ __forceinline__ int offsets_and_tiles(int c, int n_tot, int n_ffn, int small_max, int* __restrict__ offsets,
                                                  int4* __restrict__ mt_list, int4* __restrict__ small_list,
                                                  int* __restrict__ hdr, int* scratch) {
@@ -368,13 +383,13 @@ __device__ __forceinline__ int offsets_and_tiles(int c, int n_tot, int n_ffn, in
     if (e < n_tot) offsets[e] = off;
     if (e == 0) offsets[n_tot] = total;
     const bool ffn = e < n_ffn;
-    const int ntile = (ffn && c > small_max) ? (c + 127) / 128 : 0;
-    const int small = (ffn && c > 0 && c <= small_max) ? 1 : 0;
+    const int ntile = (ffn && small_max >= 0 && c > small_max) ? (c + 127) / 128 : 0;
+    const int small = stream_entries(ffn, c, small_max);
     int mt_total, small_total;
     const int mt_pos = block_exclusive_scan(ntile, scratch, &mt_total);
     const int sm_pos = block_exclusive_scan(small, scratch, &small_total);
     for (int i = 0; i < ntile; ++i) mt_list[mt_pos + i] = make_int4(e, off + 128 * i, min(128, c - 128 * i), 0);
-    if (small) small_list[sm_pos] = make_int4(e, off, c, 0);
+    write_stream_entries(small_list, sm_pos, small, e, off, c, small_max);
     // R = rows of FFN experts = offsets[n_ffn] (FFN ids come first)
     const int ffn_rows_part = ffn ? c : 0;
     int rows_total;
@@ -445,14 +460,14 @@ __device__ __forceinline__ void dispatch_small_body(const int32_t* __restrict__ 
     }
     if (e == 0) offsets[n_tot] = total;
     const bool ffn = e < n_ffn;
-    const int ntile = (ffn && c > small_max) ? (c + 127) / 128 : 0;
-    const int small = (ffn && c > 0 && c <= small_max) ? 1 : 0;
+    const int ntile = (ffn && small_max >= 0 && c > small_max) ? (c + 127) / 128 : 0;
+    const int small = stream_entries(ffn, c, small_max);
     int mt_total, small_total, rows_total;
     const int mt_pos = block_exclusive_scan(ntile, scratch, &mt_total);
     const int sm_pos = block_exclusive_scan(small, scratch, &small_total);
     block_exclusive_scan(ffn ? c : 0, scratch, &rows_total);
     for (int i = 0; i < ntile; ++i) mt_list[mt_pos + i] = make_int4(e, off + 128 * i, min(128, c - 128 * i), 0);
-    if (small) small_list[sm_pos] = make_int4(e, off, c, 0);
+    write_stream_entries(small_list, sm_pos, small, e, off, c, small_max);
     if (e == 0) {
         hdr[HDR_ROWS] = rows_total;
         hdr[HDR_MT] = mt_total;

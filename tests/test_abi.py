@@ -101,8 +101,10 @@ def test_block_scaled_config_and_encoder_checks():
     L = lmoe.lib()
     ok = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp4"], 32)
     assert lmoe.lmoe_workspace_bytes(ok) > lmoe.lmoe_workspace_bytes(lmoe.make_config(synth.WORKLOADS["nemotron_decode"], 32))
-    # block-scaled experts: decode batches only, latent and m whole 128-element stages, formats 0..3
-    for b in (dict(max_tokens=33), dict(latent=192), dict(m=320), dict(expert_fmt=4), dict(expert_fmt=-1)):
+    # block-scaled experts: latent and m whole 128-element stages, formats 0..3; any batch size
+    big_batch = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp8"], 4096)
+    assert lmoe.lmoe_workspace_bytes(big_batch) > 0
+    for b in (dict(latent=192), dict(m=320), dict(expert_fmt=4), dict(expert_fmt=-1)):
         c = lmoe.make_config(synth.WORKLOADS["nemotron_decode_mxfp8"], 32)
         for k, v in b.items():
             setattr(c, k, v)
@@ -144,8 +146,8 @@ def test_nvfp4_config_and_encoder_checks():
     L = lmoe.lib()
     ok = lmoe.make_config(synth.WORKLOADS["nemotron_decode_nvfp4"], 32)
     assert lmoe.lmoe_workspace_bytes(ok) > 0
-    # NVFP4 experts stream in stages of 256 elements; decode batches only; no expert parallelism
-    for b in (dict(latent=384), dict(m=640), dict(max_tokens=33), dict(expert_fmt=4)):
+    # NVFP4 experts stream in stages of 256 elements; no expert parallelism
+    for b in (dict(latent=384), dict(m=640), dict(expert_fmt=4)):
         c = lmoe.make_config(synth.WORKLOADS["nemotron_decode_nvfp4"], 32)
         for k, v in b.items():
             setattr(c, k, v)

@@ -6,8 +6,9 @@
 * The layer with MXFP8 and MXFP4 experts against the oracle's MX layer.  The
   oracle encodes the weights itself: no code or scale crosses from the GPU.
   The contract tolerances apply.  Every case is a decode batch (T <= 32, the
-  regime block-scaled experts serve), and every case covers several K stages
-  and a ragged tail of token-scale blocks.
+  regime block-scaled experts serve) or a larger batch whose experts stream
+  in several 32-row entries; every case covers several K stages and a ragged
+  tail of token-scale blocks.
 """
 import numpy as np
 import pytest
@@ -37,6 +38,10 @@ CASES = {
     "mxfp4_ragged_scale_chunks_swiglu": MX_BASE.with_(expert_fmt=2, d=512, latent=640, m=384, n_ffn=24, top_k=6,
                                                       act="swiglu", tokens=23, seed=59),
     "mxfp8_shared_latent_router": MX_BASE.with_(expert_fmt=1, shared_m=128, latent_router=1, seed=60),
+    # more than 32 rows per expert: each expert streams in several 32-row entries (up to 5 with the skew)
+    "mxfp8_150_tokens": MX_BASE.with_(expert_fmt=1, tokens=150, seed=62),
+    "mxfp4_300_tokens_swiglu_skew": MX_BASE.with_(expert_fmt=2, act="swiglu", zipf=1.1, n_zero=1, tokens=300,
+                                                  seed=63),
     "nemotron_decode_mxfp8": synth.WORKLOADS["nemotron_decode_mxfp8"],
     "nemotron_decode_mxfp4": synth.WORKLOADS["nemotron_decode_mxfp4"],
 }

@@ -5,9 +5,10 @@
   they are taken out of the tensor-core atom order.
 * The layer with NVFP4 experts against the oracle's NVFP4 layer.  The oracle
   encodes the weights itself: no code or scale crosses from the GPU.  The
-  contract tolerances apply.  Every case is a decode batch (T <= 32, the
-  regime block-scaled experts serve).  The cases span one to three K stages of
-  256 elements.
+  contract tolerances apply.  Most cases are decode batches (T <= 32, the
+  regime block-scaled experts serve); two are larger, so that experts stream
+  in several 32-row entries.  The cases span one to three K stages of 256
+  elements.
 """
 import numpy as np
 import pytest
@@ -32,6 +33,9 @@ CASES = {
     # K = 768 for the up GEMM (three stages), 512 for the down GEMM (two)
     "nvfp4_three_stages": NV_BASE.with_(latent=768, m=512, n_ffn=24, top_k=6, tokens=31, seed=66),
     "nvfp4_shared_latent_router": NV_BASE.with_(shared_m=128, latent_router=1, seed=67),
+    # more than 32 rows per expert: several 32-row entries per expert
+    "nvfp4_200_tokens": NV_BASE.with_(tokens=200, seed=68),
+    "nvfp4_260_tokens_swiglu_skew": NV_BASE.with_(act="swiglu", zipf=1.1, n_copy=1, tokens=260, seed=69),
     "nemotron_decode_nvfp4": synth.WORKLOADS["nemotron_decode_nvfp4"],
 }
 
