@@ -13,11 +13,14 @@ Tolerances (fixed for the layer's output):
 The CUDA path stores z, the expert hidden rows H, the expert outputs O, the
 combined latent yl and y in bf16 (H, yl and z feed bf16 tensor-core GEMMs).  On
 a few degenerate shapes (top-1 routing, where nothing averages the expert
-output) those roundings alone exceed the max-error bound.  ``emulate_bf16``
-evaluates the layer with exactly those storage roundings (fp64 otherwise); a
-max-error miss is accepted only when that emulation alone reaches at least 75%
-of the bound, the GPU stays within 1.5x of the emulation's error, and the mean
-relative error still meets 5e-3.
+output, or outputs of a few times RMS(y_ref), where one bf16 rounding of y is
+already worth most of the bound) those roundings alone exceed the max-error
+bound.  ``emulate_bf16`` evaluates the layer with exactly those storage
+roundings (fp64 otherwise), and with block-scaled experts with the oracle's
+encodings of their weights and inputs on top; a max-error miss is accepted only
+when that emulation alone reaches at least 75% of the bound, the GPU stays
+within 1.5x of the emulation's error, and the mean relative error still meets
+5e-3.
 """
 from __future__ import annotations
 
@@ -52,28 +55,69 @@ def _bf(a: np.ndarray) -> np.ndarray:
     return torch.from_numpy(np.ascontiguousarray(a, np.float64)).to(torch.float32).to(torch.bfloat16).double().numpy()
 
 
+def _expert_weights(cfg, layer):
+    """Each expert's W1_e, W2_e at the values the layer computes with: as stored (bf16), or the oracle's
+    block-scaled encoding of them decoded (MXFP8 / MXFP4 per matrix row blocks, NVFP4 per expert matrix)."""
+    fmt = getattr(cfg, "expert_fmt", 0)
+    W1, W2 = layer["w1"], layer["w2"]
+    if fmt == 0:
+        return [w.double().numpy() for w in W1], [w.double().numpy() for w in W2]
+    out = []
+    for W in (W1, W2):
+        mats = []
+        for e in range(W.shape[0]):
+            if fmt == oracle.FMT_NVFP4:
+                g = oracle.nv_tensor_scale(W[e])
+                c, sc = oracle.nv_quantize(W[e], g)
+                mats.append(oracle.nv_dequantize(c, sc, g))
+            else:
+                c, sc = oracle.mx_quantize(W[e], fmt)
+                mats.append(oracle.mx_dequantize(c, sc, fmt))
+        out.append(mats)
+    return out[0], out[1]
+
+
+def _expert_input(cfg, v: np.ndarray) -> np.ndarray:
+    """An expert GEMM's input as the layer feeds it: bf16, then (block-scaled experts) its encoding decoded:
+    MXFP8 for the MX formats, NVFP4 with tensor scale 1 for NVFP4."""
+    fmt = getattr(cfg, "expert_fmt", 0)
+    b = _bf(v)
+    if fmt == 0:
+        return b
+    t = torch.from_numpy(b.reshape(1, -1)).to(torch.bfloat16)
+    if fmt == oracle.FMT_NVFP4:
+        c, sc = oracle.nv_quantize(t, 1.0)
+        return oracle.nv_dequantize(c, sc, 1.0).reshape(-1)
+    c, sc = oracle.mx_quantize(t, oracle.FMT_MXFP8)
+    return oracle.mx_dequantize(c, sc, oracle.FMT_MXFP8).reshape(-1)
+
+
 def emulate_bf16(cfg, layer, x: torch.Tensor, idx: np.ndarray, w: np.ndarray) -> np.ndarray:
     """y with the GPU path's bf16 storage points (z, H, O, yl, the shared expert's hidden rows and
-    x + its output, y) on the given routes."""
+    x + its output, y) on the given routes.  With block-scaled experts the expert weights and inputs take
+    the oracle's encodings (the layer's definition) on top of those storage points."""
     f = lambda t: None if t is None else t.double().numpy()  # noqa: E731
     X = f(x)
-    W1, W2 = layer["w1"], layer["w2"]
+    W1, W2 = _expert_weights(cfg, layer)
     z = _bf(X @ f(layer["w_down"]).T) if cfg.has_proj else X
     m = cfg.m
     yl = np.zeros_like(z)
     for t in range(X.shape[0]):
         acc = np.zeros(z.shape[1])
+        zin = None
         for k in range(cfg.top_k):
             e = int(idx[t, k])
             if e < cfg.n_ffn:
-                u = W1[e].double().numpy() @ z[t]
+                if zin is None:
+                    zin = _expert_input(cfg, z[t])
+                u = W1[e] @ zin
                 if cfg.act == 0:
                     h = np.maximum(u, 0) ** 2
                 elif cfg.act == 1:
                     h = u[:m] / (1 + np.exp(-u[:m])) * u[m:]
                 else:
                     h = u
-                o = _bf(W2[e].double().numpy() @ _bf(h))
+                o = _bf(W2[e] @ _expert_input(cfg, h))
             elif e < cfg.n_ffn + cfg.n_zero:
                 o = np.zeros_like(z[t])
             elif e < cfg.n_ffn + cfg.n_zero + cfg.n_copy:
