@@ -432,7 +432,10 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
                      unsigned long long timeout_ns, cudaStream_t s) {
     const int t0 = (g.rows0 + 127) / 128, t1 = (g.rows1 + 127) / 128;
     const int nkb = g.K / 64;
-    int splits = (num_sms + t0 + t1 - 1) / (t0 + t1);
+    // Each (weight tile, K split) unit streams a 512-deep slice of K, 128 KB of weights, and there is at
+    // most one unit per SM.  Longer units beat one unit per SM: each split costs a CTA's fixed set-up and
+    // adds a block of partial sums to the in-order reduction.
+    int splits = std::min((num_sms + t0 + t1 - 1) / (t0 + t1), (nkb + 7) / 8);
     splits = std::max(1, std::min(splits, std::min(max_splits, nkb)));
     SwapArgs a{};
     a.K = g.K;
