@@ -53,6 +53,18 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------- clocks
+# Untimed steps run right before the timed region, about this many seconds of them, while the clock
+# sampler runs: a decode step is ~0.3 ms, so the K timed steps alone are far shorter than nvidia-smi's
+# 200 ms sampling period.  The samples cover these steps and the timed region, the GPU under one load.
+SOAK_S = 1.0
+
+
+def soak_count(step_ms: float, max_over_ranks) -> int:
+    """Steps of the clock soak for a step of `step_ms` ms; the same count on every rank."""
+    n = SOAK_S * 1e3 / max(step_ms, 1e-3)
+    return int(min(max(max_over_ranks(n), 1.0), 100000.0))
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
 
@@ -276,12 +288,16 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     barrier = lambda: dist_barrier(world)  # noqa: E731
     max_over_ranks = lambda v: dist_max(v, world, dev)  # noqa: E731
 
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
     for i in range(warmup):
         mod.forward(xd[i % N_INPUT_BATCHES], yd)
+    w1.record(stream)
     torch.cuda.synchronize()
     status = mod.last_error()
     if status != 0:
         raise RuntimeError(f"device error during warm-up: {lmoe.lmoe_status_string(status)}")
+    n_soak = soak_count(w0.elapsed_time(w1) / max(warmup, 1), max_over_ranks) if with_clocks else 0
 
     # ---------------------------------------------------------------- device-timed region (the headline)
     # No per-phase events here: an event between two kernels costs ~2 us of GPU time and breaks the
@@ -289,7 +305,8 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     clocks = ClockSampler(_smi_id(device)) if with_clocks else None
     if clocks:
         clocks.start()
-        time.sleep(0.3)
+    for i in range(n_soak):  # untimed: the clock samples cover these steps and the timed region
+        mod.forward(xd[i % N_INPUT_BATCHES], yd)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -422,14 +439,19 @@ def run_ep(cfg, steps, warmup, rank, world, device, peaks):
         sc = rk.send_counts.cpu().view(world, nl).sum(1)
         sent_away += float(sc.sum() - sc[rank]) / len(xd)
     stats = acc
+    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    w0.record(stream)
     for i in range(warmup):
         rk.forward(xd[i % N_INPUT_BATCHES], yd)
+    w1.record(stream)
     torch.cuda.synchronize()
     check("during warm-up")
+    n_soak = soak_count(w0.elapsed_time(w1) / max(warmup, 1), max_over_ranks)
 
     clocks = ClockSampler(_smi_id(device))
     clocks.start()
-    time.sleep(0.3)
+    for i in range(n_soak):  # untimed, the same count on every rank: the clock samples cover these steps too
+        rk.forward(xd[i % N_INPUT_BATCHES], yd)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()
