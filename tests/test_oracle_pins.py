@@ -236,6 +236,29 @@ def test_shared_expert_alone_is_a_plain_ffn_on_x():
     np.testing.assert_allclose(b["y"] - x, 2 * (a["y"] - x), rtol=1e-12, atol=1e-13)
 
 
+@pytest.mark.parametrize("act", ["relu2", "swiglu"])
+@pytest.mark.parametrize("has_proj", [1, 0])
+def test_one_expert_top1_is_a_plain_ffn(act, has_proj):
+    """N' = K' = 1 (no bypass experts): the only expert gets weight 1 for every token, so the layer is
+    x + W_up W2 act(W1 W_down x), or x + W2 act(W1 x) without projections, here in numpy fp64 matmuls."""
+    cfg = SMALL.with_(n_ffn=1, n_zero=0, n_copy=0, n_const=0, top_k=1, act=act, has_proj=has_proj,
+                      latent=SMALL.latent if has_proj else SMALL.d)
+    layer = synth.make_layer(cfg, tokens=9)
+    x = _np(layer["x"])
+    z = x @ _np(layer["w_down"]).T if has_proj else x
+    u = z @ _np(layer["w1"][0]).T
+    if act == "swiglu":
+        g, up = u[:, :cfg.m], u[:, cfg.m:]
+        h = g / (1.0 + np.exp(-g)) * up
+    else:
+        h = np.maximum(u, 0.0) ** 2
+    o = h @ _np(layer["w2"][0]).T
+    y = x + (o @ _np(layer["w_up"]).T if has_proj else o)
+    ref = oracle.forward(cfg, layer, want=("y", "idx", "w"))
+    assert np.all(ref["idx"] == 0) and np.all(ref["w"] == 1.0)
+    np.testing.assert_allclose(ref["y"], y, rtol=1e-12, atol=1e-12)
+
+
 def test_latent_router_matches_dense_bruteforce():
     cfg = SMALL.with_(latent_router=1)
     layer = synth.make_layer(cfg)
