@@ -178,6 +178,13 @@ LMOE_API int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *wo
  * by the caller (same stream).  Device-side faults (a bounded wait that gave
  * up, a bad expert id) are reported by lmoe_last_error after the stream is
  * synchronised.  Output is bit-identical from run to run.  `dbg` may be NULL.
+ * By default, for a layer without a shared expert, the forward's launches
+ * reach the GPU as one CUDA graph: they are captured on a stream of the
+ * handle's own and the handle's executable graph is updated and launched on
+ * `stream` (see lmoe_set_graph_launch).  No device memory is allocated and the
+ * host does not wait on the device.  With a shared expert (two streams), while
+ * `stream` is itself being captured, with phase timing on, or with `dbg` set,
+ * the launches go onto `stream` one by one; the results are the same bits.
  */
 LMOE_API int lmoe_forward(lmoe_handle *h, const void *x, void *y, int32_t T, void *stream, const lmoe_debug *dbg);
 
@@ -240,6 +247,16 @@ LMOE_API int lmoe_routing_stats(lmoe_handle *h, int32_t *out8);
  * to the grouped GEMM.
  */
 LMOE_API int lmoe_set_small_rows(lmoe_handle *h, int32_t rows);
+
+/*
+ * enable = 1 (default): lmoe_forward and lmoe_forward_host launch each forward
+ * of a layer without a shared expert as one CUDA graph (captured per call on
+ * the handle's own stream, replayed from one executable graph that is updated
+ * in place); 0: the kernels are launched on the caller's stream one by one.
+ * Outputs are bit-identical.
+ * Errors: LMOE_ERR_INVALID_ARG for a NULL handle or enable not 0 or 1.
+ */
+LMOE_API int lmoe_set_graph_launch(lmoe_handle *h, int enable);
 
 /* Bound of every in-kernel wait, nanoseconds (default 1e9). */
 LMOE_API int lmoe_set_wait_timeout(lmoe_handle *h, uint64_t ns);

@@ -77,6 +77,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_routing_stats.argtypes = [P, ctypes.POINTER(I32)]
         L.lmoe_set_small_rows.argtypes = [P, I32]
         L.lmoe_set_wait_timeout.argtypes = [P, ctypes.c_uint64]
+        L.lmoe_set_graph_launch.argtypes = [P, ctypes.c_int]
         L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
         L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
         L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
@@ -176,6 +177,11 @@ def lmoe_set_small_rows(h: int, rows: int) -> None:
 
 def lmoe_set_wait_timeout(h: int, ns: int) -> None:
     _check("lmoe_set_wait_timeout", lib().lmoe_set_wait_timeout(h, ns))
+
+
+def lmoe_set_graph_launch(h: int, enable: bool) -> None:
+    """Launch each forward as one CUDA graph (default) or its kernels one by one."""
+    _check("lmoe_set_graph_launch", lib().lmoe_set_graph_launch(h, 1 if enable else 0))
 
 
 def lmoe_selftest_wait(h: int, timeout_ns: int, stream=None) -> None:

@@ -85,6 +85,7 @@ def test_null_handle_calls_are_rejected():
     assert L.lmoe_ep_dispatch(None, None, 1, None, None, None) == -1
     assert L.lmoe_ep_experts(None, None, None, 1, 1, None, None) == -1
     assert L.lmoe_ep_combine(None, None, None, None) == -1
+    assert L.lmoe_set_graph_launch(None, 1) == -1
     assert lmoe.lmoe_num_phases() == 11
     assert lmoe.lmoe_phase_name(10) == "ep_regroup"
     assert [lmoe.lmoe_phase_name(i) for i in range(3)] == ["router_proj_gemm", "topk_softmax", "dispatch"]

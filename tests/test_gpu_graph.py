@@ -1,4 +1,5 @@
-"""The layer forward captured in a CUDA graph and replayed, through the C ABI.
+"""CUDA graphs, through the C ABI: the layer forward captured by the caller and replayed, and the
+library's own graph launch of each forward.
 
 lmoe_forward enqueues kernels only: no allocation, no host synchronisation,
 with the shared expert's second stream forked and joined by events.  A graph
@@ -54,5 +55,51 @@ def test_graph_replay_matches_the_eager_forward(name):
             assert torch.equal(static_y, ref)
         assert mod.last_error() == 0
         del g
+    finally:
+        mod.close()
+
+
+# lmoe_forward launches each forward as a CUDA graph of its own by default (captured on the handle's stream,
+# replayed from one executable graph).  These cases check it against the kernels launched one by one.
+LIB_GRAPH_CASES = dict(CASES, std_moe_medium=MEDIUM.with_(has_proj=0, latent=512, seed=124),
+                       medium_latent_router=MEDIUM.with_(latent_router=1, seed=125))
+
+
+@pytest.mark.parametrize("name", list(LIB_GRAPH_CASES))
+def test_library_graph_launch_matches_direct_launches(name):
+    cfg = LIB_GRAPH_CASES[name]
+    T = cfg.tokens
+    layer = synth.make_layer(cfg)
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=T)
+    try:
+        # token counts that keep the launch sequence (graph updated in place) and change it (rebuilt)
+        sizes = [T, T, max(1, T // 2), min(T, 24), T]
+        xs = [synth.make_tokens(cfg, n, seed=700 + i).cuda() for i, n in enumerate(sizes)]
+        lmoe.lmoe_set_graph_launch(mod.h, False)
+        direct = [mod.forward(x) for x in xs]
+        torch.cuda.synchronize()
+        lmoe.lmoe_set_graph_launch(mod.h, True)
+        graphed = [mod.forward(x) for x in xs]
+        torch.cuda.synchronize()
+        assert mod.last_error() == 0
+        for a, b in zip(direct, graphed):
+            assert torch.equal(a, b)
+        # the host-buffer entry point takes the same graph path
+        xh = xs[0].cpu().pin_memory()
+        yh = torch.empty_like(xh).pin_memory()
+        mod.forward_host(xh, yh)
+        torch.cuda.synchronize()
+        assert torch.equal(yh, direct[0].cpu())
+    finally:
+        mod.close()
+
+
+def test_graph_launch_switch_rejects_bad_values():
+    cfg = MEDIUM.with_(tokens=8)
+    mod = lmoe.LatentMoE(cfg, synth.make_layer(cfg), max_tokens=8)
+    try:
+        assert lmoe.lib().lmoe_set_graph_launch(mod.h, 2) == -1
+        lmoe.lmoe_set_graph_launch(mod.h, False)
+        lmoe.lmoe_set_graph_launch(mod.h, True)
     finally:
         mod.close()
