@@ -53,34 +53,59 @@ def load_peaks():
 
 
 # ----------------------------------------------------------------------------- clocks
-# Untimed steps run right before the timed region, about this many seconds of them, while the clock
-# sampler runs: a decode step is ~0.3 ms, so the K timed steps alone are far shorter than nvidia-smi's
-# 200 ms sampling period.  The samples cover these steps and the timed region, the GPU under one load.
-SOAK_S = 1.0
+# Throttle reasons reported in the clock record, with the NVML constant of each.
+CLOCK_REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+                 ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+                 ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+                 ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
 
-def soak_count(step_ms: float, max_over_ranks) -> int:
-    """Steps of the clock soak for a step of `step_ms` ms; the same count on every rank."""
-    n = SOAK_S * 1e3 / max(step_ms, 1e-3)
-    return int(min(max(max_over_ranks(n), 1.0), 100000.0))
+def clock_summary(samples, max_mhz, nvml):
+    """The clock record from (SM MHz, reason bits) samples: the median clock, the maximum clock and the names
+    of the reasons any sample had active."""
+    reasons = sorted(name for name, const in CLOCK_REASONS
+                     if any(bits & getattr(nvml, const) for _, bits in samples))
+    sm = [mhz for mhz, _ in samples]
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max_mhz, "reasons": reasons,
+            "samples": len(sm)}
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """SM clock and throttle reasons sampled while the timed region runs (read-only queries).
+
+    NVML, the library nvidia-smi reads, is polled every 2 ms from a thread, so even the ~15 ms of K decode
+    steps get several samples.  Without NVML, nvidia-smi runs every 200 ms instead.
+    """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.002
 
-    def __init__(self, device_index: int):
-        self.idx = device_index
+    def __init__(self, device_uuid: str):
+        self.uuid = device_uuid
         self.proc = None
         self.lines = []
         self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.samples = []
+        self.done = threading.Event()
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+            import pynvml
+            pynvml.nvmlInit()
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.nvml = pynvml
+        except Exception:
+            self.nvml = None
+        if self.nvml is not None:
+            self.thread = threading.Thread(target=self._poll, daemon=True)
+            self.thread.start()
+            return
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.uuid}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
                                          stderr=subprocess.DEVNULL, text=True)
         except Exception:
@@ -89,11 +114,33 @@ class ClockSampler:
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
 
+    def _poll(self):
+        n = self.nvml
+        while not self.done.is_set():
+            try:
+                mhz = float(n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM))
+                bits = int(n.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+                self.samples.append((mhz, bits))
+            except Exception:
+                return
+            time.sleep(self.PERIOD_S)
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append(line.strip())
 
     def stop(self):
+        if self.nvml is not None:
+            self.done.set()
+            if self.thread:
+                self.thread.join(timeout=2)
+            try:
+                max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
+            except Exception:
+                max_mhz = None
+            out = clock_summary(self.samples, max_mhz, self.nvml)
+            out["source"] = "nvml, every 2 ms"
+            return out
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -118,7 +165,7 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(n)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "source": "nvidia-smi, every 200 ms"}
 
 
 def _smi_id(device: int) -> str:
@@ -288,16 +335,12 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     barrier = lambda: dist_barrier(world)  # noqa: E731
     max_over_ranks = lambda v: dist_max(v, world, dev)  # noqa: E731
 
-    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    w0.record(stream)
     for i in range(warmup):
         mod.forward(xd[i % N_INPUT_BATCHES], yd)
-    w1.record(stream)
     torch.cuda.synchronize()
     status = mod.last_error()
     if status != 0:
         raise RuntimeError(f"device error during warm-up: {lmoe.lmoe_status_string(status)}")
-    n_soak = soak_count(w0.elapsed_time(w1) / max(warmup, 1), max_over_ranks) if with_clocks else 0
 
     # ---------------------------------------------------------------- device-timed region (the headline)
     # No per-phase events here: an event between two kernels costs ~2 us of GPU time and breaks the
@@ -305,8 +348,6 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
     clocks = ClockSampler(_smi_id(device)) if with_clocks else None
     if clocks:
         clocks.start()
-    for i in range(n_soak):  # untimed: the clock samples cover these steps and the timed region
-        mod.forward(xd[i % N_INPUT_BATCHES], yd)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()
@@ -439,19 +480,13 @@ def run_ep(cfg, steps, warmup, rank, world, device, peaks):
         sc = rk.send_counts.cpu().view(world, nl).sum(1)
         sent_away += float(sc.sum() - sc[rank]) / len(xd)
     stats = acc
-    w0, w1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    w0.record(stream)
     for i in range(warmup):
         rk.forward(xd[i % N_INPUT_BATCHES], yd)
-    w1.record(stream)
     torch.cuda.synchronize()
     check("during warm-up")
-    n_soak = soak_count(w0.elapsed_time(w1) / max(warmup, 1), max_over_ranks)
 
     clocks = ClockSampler(_smi_id(device))
     clocks.start()
-    for i in range(n_soak):  # untimed, the same count on every rank: the clock samples cover these steps too
-        rk.forward(xd[i % N_INPUT_BATCHES], yd)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     barrier()

@@ -2,9 +2,8 @@
 
 Each rank is an independent replica of the layer (tokens shard with no exchange
 step), so the only cross-rank operations are the barrier and the maximum of the
-per-rank device time; the reference arm runs on rank 0 alone.  The untimed
-steps under the clock sampler are sized from each rank's own step time, and
-every rank must run the same number (an expert-parallel step has collectives).
+per-rank device time; the reference arm runs on rank 0 alone.  The clock
+record's summary of NVML samples is checked against a fake NVML here.
 """
 import os
 import socket
@@ -33,8 +32,7 @@ def _rank_main(rank, world, port, out):
         got = bench.dist_max(mine, world, torch.device("cpu"))
         # the reference arm: only rank 0 does any work or prints
         ref = bench.run_reference(type("A", (), {"steps": 1, "warmup": 0})(), None, rank, world) if rank else "rank0"
-        soak = bench.soak_count(0.3 if rank == 0 else 0.5, lambda v: bench.dist_max(v, world, torch.device("cpu")))
-        out.put((rank, got, ref, soak))
+        out.put((rank, got, ref))
         bench.dist_barrier(world)
     finally:
         tdist.destroy_process_group()
@@ -50,21 +48,25 @@ def test_two_gloo_ranks_take_the_max_time_and_only_rank0_reports():
     for p in procs:
         p.join(timeout=120)
     assert all(p.exitcode == 0 for p in procs)
-    res = dict((r, (g, ref, soak)) for r, g, ref, soak in [q.get(timeout=5) for _ in range(2)])
+    res = dict((r, (g, ref)) for r, g, ref in [q.get(timeout=5) for _ in range(2)])
     assert res[0][0] == res[1][0] == 15.0
     assert res[1][1] is None and res[0][1] == "rank0"
-    # about 1 s of the faster rank's 0.3 ms steps, on both ranks
-    assert res[0][2] == res[1][2] == int(bench_soak_s() * 1e3 / 0.3)
 
 
-def bench_soak_s():
+class _FakeNvml:
+    """The NVML reason constants the clock record decodes (their values in NVML's header)."""
+    nvmlClocksEventReasonSwPowerCap = 0x4
+    nvmlClocksEventReasonHwSlowdown = 0x8
+    nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nvmlClocksEventReasonHwThermalSlowdown = 0x40
+
+
+def test_clock_record_from_samples():
     import bench
-    return bench.SOAK_S
-
-
-def test_soak_count_is_bounded():
-    import bench
-    same = lambda v: v  # noqa: E731  (one rank)
-    assert bench.soak_count(1.0, same) == int(bench.SOAK_S * 1e3)
-    assert bench.soak_count(0.0, same) == 100000  # a step time of 0 is clamped, not divided by
-    assert bench.soak_count(1e9, same) == 1
+    idle_bit = 0x1  # GPU idle: not a reason the record reports
+    samples = [(1965.0, 0), (1830.0, 0x4), (1965.0, idle_bit), (1890.0, 0x4)]
+    rec = bench.clock_summary(samples, 1965.0, _FakeNvml)
+    assert rec == {"sm_mhz": 1927.5, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 4}
+    rec = bench.clock_summary([(1500.0, 0x8 | 0x40)], 1965.0, _FakeNvml)
+    assert rec["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+    assert bench.clock_summary([], None, _FakeNvml)["sm_mhz"] is None
