@@ -39,7 +39,10 @@
  *     device; "host" pointers are ordinary (preferably pinned) host memory;
  *   - every device pointer must be 16-byte aligned;
  *   - the caller owns every buffer; the library never allocates device memory
- *     and borrows the weights and the workspace for the handle's lifetime;
+ *     for data and borrows the weights and the workspace for the handle's
+ *     lifetime (the executable CUDA graph of lmoe_forward is a driver object
+ *     that the handle creates on its first forward and again when the launch
+ *     sequence changes shape; lmoe_destroy releases it);
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream); work is
  *     enqueued asynchronously, nothing in lmoe_forward synchronises the host;
  *   - return values: LMOE_OK (0) or a negative LMOE_ERR_* status; a rejected
