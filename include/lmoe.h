@@ -40,9 +40,9 @@
  *   - every device pointer must be 16-byte aligned;
  *   - the caller owns every buffer; the library never allocates device memory
  *     for data and borrows the weights and the workspace for the handle's
- *     lifetime (the executable CUDA graph of lmoe_forward is a driver object
- *     that the handle creates on its first forward and again when the launch
- *     sequence changes shape; lmoe_destroy releases it);
+ *     lifetime (the executable CUDA graphs of lmoe_forward are driver objects
+ *     that the handle creates on the first forward of each launch sequence,
+ *     at most 8; lmoe_destroy releases them);
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream); work is
  *     enqueued asynchronously, nothing in lmoe_forward synchronises the host;
  *   - return values: LMOE_OK (0) or a negative LMOE_ERR_* status; a rejected
@@ -183,8 +183,8 @@ LMOE_API int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *wo
  * synchronised.  Output is bit-identical from run to run.  `dbg` may be NULL.
  * By default, for a layer without a shared expert, the forward's launches
  * reach the GPU as one CUDA graph: they are captured on a stream of the
- * handle's own and the handle's executable graph is updated and launched on
- * `stream` (see lmoe_set_graph_launch).  No device memory is allocated and the
+ * handle's own, and the handle's executable graph for that launch sequence is
+ * updated and launched on `stream` (see lmoe_set_graph_launch).  No device memory is allocated and the
  * host does not wait on the device.  With a shared expert (two streams), while
  * `stream` is itself being captured, with phase timing on, or with `dbg` set,
  * the launches go onto `stream` one by one; the results are the same bits.
@@ -254,9 +254,10 @@ LMOE_API int lmoe_set_small_rows(lmoe_handle *h, int32_t rows);
 /*
  * enable = 1 (default): lmoe_forward and lmoe_forward_host launch each forward
  * of a layer without a shared expert as one CUDA graph (captured per call on
- * the handle's own stream, replayed from one executable graph that is updated
- * in place); 0: the kernels are launched on the caller's stream one by one.
- * Outputs are bit-identical.
+ * the handle's own stream, replayed from an executable graph updated in place;
+ * the handle keeps up to 8, one per launch sequence, since token counts can
+ * change which kernels run); 0: the kernels are launched on the caller's
+ * stream one by one.  Outputs are bit-identical.
  * Errors: LMOE_ERR_INVALID_ARG for a NULL handle or enable not 0 or 1.
  */
 LMOE_API int lmoe_set_graph_launch(lmoe_handle *h, int enable);

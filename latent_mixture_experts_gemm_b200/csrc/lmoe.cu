@@ -553,9 +553,16 @@ struct lmoe_handle {
     CUtensorMap o_h{}, o_rows{}, o_z{};
     cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
     // Forwards launched as a CUDA graph: each call captures its launches on `cap` and replays them on the
-    // caller's stream from `gexec`, which is updated in place while the launch sequence keeps its shape.
+    // caller's stream from an executable graph, updated in place.  A few executable graphs are kept, one per
+    // launch sequence (token counts that change the kernels used), least recently used first out.
+    struct GraphExec {
+        std::vector<const void*> sig;  // node kinds and kernel functions, in the capture's order
+        cudaGraphExec_t exec = nullptr;
+        uint64_t used = 0;
+    };
     cudaStream_t cap = nullptr;
-    cudaGraphExec_t gexec = nullptr;
+    std::vector<GraphExec> graphs;
+    uint64_t graph_tick = 0;
     int use_graph = 1;
     cudaEvent_t ev_fork = nullptr, ev_join = nullptr;
     // profiling
@@ -1107,10 +1114,32 @@ int run_forward(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s, c
     return LMOE_OK;
 }
 
+constexpr size_t kGraphCache = 8;
+
+// The launch sequence of a captured graph: each node's kind and, for kernels, the function.
+bool graph_signature(cudaGraph_t g, std::vector<const void*>& sig) {
+    size_t n = 0;
+    if (cudaGraphGetNodes(g, nullptr, &n) != cudaSuccess) return false;
+    std::vector<cudaGraphNode_t> nodes(n);
+    if (n > 0 && cudaGraphGetNodes(g, nodes.data(), &n) != cudaSuccess) return false;
+    sig.clear();
+    for (size_t i = 0; i < n; ++i) {
+        cudaGraphNodeType t;
+        if (cudaGraphNodeGetType(nodes[i], &t) != cudaSuccess) return false;
+        sig.push_back(reinterpret_cast<const void*>(static_cast<uintptr_t>(t) + 1));
+        if (t == cudaGraphNodeTypeKernel) {
+            cudaKernelNodeParams kp{};
+            if (cudaGraphKernelNodeGetParams(nodes[i], &kp) != cudaSuccess) return false;
+            sig.push_back(kp.func);
+        }
+    }
+    return true;
+}
+
 // One forward as a CUDA graph.  The launches of run_forward are captured on the handle's own stream and
-// replayed on `s` from one executable graph, updated in place when only launch parameters changed (pointers,
-// grid sizes) and instantiated again when the sequence changed shape.  A graph launch costs the GPU less per
-// kernel than the same launches issued one by one, and the capture costs host time only.
+// replayed on `s` from the executable graph kept for the same launch sequence, updated in place (pointers,
+// grid sizes), or from a new one.  A graph launch costs the GPU less per kernel than the same launches issued
+// one by one, and the capture costs host time only.
 int forward_graph(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s) {
     if (cudaStreamBeginCapture(h->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) return LMOE_ERR_CUDA;
     const int st = run_forward(h, x, y, T, h->cap, nullptr);
@@ -1121,23 +1150,43 @@ int forward_graph(lmoe_handle* h, const void* x, void* y, int T, cudaStream_t s)
         cudaGetLastError();  // the capture's own error state; the handle stays usable
         return st != LMOE_OK ? st : LMOE_ERR_CUDA;
     }
-    bool ready = false;
-    if (h->gexec != nullptr) {
+    std::vector<const void*> sig;
+    const bool have_sig = graph_signature(g, sig);
+    cudaGetLastError();
+    int idx = -1;
+    for (size_t i = 0; have_sig && i < h->graphs.size(); ++i)
+        if (h->graphs[i].sig == sig) idx = static_cast<int>(i);
+    if (idx >= 0) {
         cudaGraphExecUpdateResultInfo info;
-        ready = cudaGraphExecUpdate(h->gexec, g, &info) == cudaSuccess;
-        if (!ready) {
+        if (cudaGraphExecUpdate(h->graphs[idx].exec, g, &info) != cudaSuccess) {
             cudaGetLastError();  // an update refused for a changed shape is not an error of the forward
-            cudaGraphExecDestroy(h->gexec);
-            h->gexec = nullptr;
+            cudaGraphExecDestroy(h->graphs[idx].exec);
+            h->graphs.erase(h->graphs.begin() + idx);
+            idx = -1;
         }
     }
-    if (!ready) {
-        ready = cudaGraphInstantiate(&h->gexec, g, 0) == cudaSuccess;
-        if (!ready) h->gexec = nullptr;
+    if (idx < 0) {
+        cudaGraphExec_t e = nullptr;
+        if (cudaGraphInstantiate(&e, g, 0) != cudaSuccess) {
+            cudaGraphDestroy(g);
+            return LMOE_ERR_CUDA;
+        }
+        if (h->graphs.size() >= kGraphCache) {
+            size_t lru = 0;
+            for (size_t i = 1; i < h->graphs.size(); ++i)
+                if (h->graphs[i].used < h->graphs[lru].used) lru = i;
+            cudaGraphExecDestroy(h->graphs[lru].exec);  // freed when a launch still in flight completes
+            h->graphs.erase(h->graphs.begin() + lru);
+        }
+        lmoe_handle::GraphExec ge;
+        ge.sig = have_sig ? sig : std::vector<const void*>{};
+        ge.exec = e;
+        h->graphs.push_back(ge);
+        idx = static_cast<int>(h->graphs.size()) - 1;
     }
     cudaGraphDestroy(g);
-    if (!ready) return LMOE_ERR_CUDA;
-    return cudaGraphLaunch(h->gexec, s) == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+    h->graphs[idx].used = ++h->graph_tick;
+    return cudaGraphLaunch(h->graphs[idx].exec, s) == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
 // The graph form is taken for layers whose forward runs on one stream.  A layer with a shared expert forks it
@@ -1433,7 +1482,8 @@ void lmoe_destroy(lmoe_handle* h) {
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
     if (h->side) cudaStreamDestroy(h->side);
-    if (h->gexec) cudaGraphExecDestroy(h->gexec);
+    for (auto& ge : h->graphs)
+        if (ge.exec) cudaGraphExecDestroy(ge.exec);  // one still in flight is freed when it completes
     if (h->cap) cudaStreamDestroy(h->cap);
     delete h;
 }

@@ -84,6 +84,12 @@ def test_library_graph_launch_matches_direct_launches(name):
         assert mod.last_error() == 0
         for a, b in zip(direct, graphed):
             assert torch.equal(a, b)
+        # alternating between two launch sequences replays each one's kept graph
+        for _ in range(3):
+            for i in (0, 3):
+                assert torch.equal(mod.forward(xs[i]), direct[i])
+        torch.cuda.synchronize()
+        assert mod.last_error() == 0
         # the host-buffer entry point takes the same graph path
         xh = xs[0].cpu().pin_memory()
         yh = torch.empty_like(xh).pin_memory()
