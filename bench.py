@@ -13,6 +13,11 @@ With --ep the ranks instead split the FFN experts (expert parallelism): each
 rank routes its own tokens and the latent rows cross ranks by NCCL all-to-all
 before and after the experts; with one rank nothing moves and the step times
 the three stages of that forward alone.
+
+The timed steps are plain lmoe_forward calls (each forward reaches the GPU as
+the library's own CUDA graph); `graph_replay` adds the same steps replayed from
+graphs captured by the caller.  SM clocks and throttle reasons are sampled
+through NVML while the timed steps run.
 """
 from __future__ import annotations
 
