@@ -2,12 +2,17 @@
 // workspace plan, TMA descriptors and the launch sequence.  The C ABI is
 // declared in include/lmoe.h.
 //
-// Launch sequence of one forward (all on the caller's stream):
+// Launch sequence of one forward:
 //   router/projection GEMM (tcgen05) -> top-K' + softmax -> counting sort
 //   (bitmap, per-expert prefix, offsets + tile lists, scatter/gather) ->
 //   up GEMM + activation (tcgen05 grouped; weight streaming for experts with
 //   few rows) -> down GEMM (same split) -> combine in the latent width ->
 //   up-projection GEMM with the residual add (tcgen05).
+// At T <= 32 the projections are split-K weight streams with in-order
+// reductions, the router's reduction taking the top-K' too.  The shared
+// expert, when present, runs on a second stream of the handle's own.  The
+// sequence is captured into a CUDA graph that is launched on the caller's
+// stream (forward_graph), or launched there kernel by kernel.
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
