@@ -167,3 +167,15 @@ def test_nvfp4_config_and_encoder_checks():
     assert L.lmoe_nvfp4_encode_weights(0x100, 1, 128, 96, 0x100, 0x100, 0x100, None) == -2
     assert L.lmoe_nvfp4_encode_weights(0x100, 0, 128, 128, 0x100, 0x100, 0x100, None) == -2
     assert L.lmoe_nvfp4_encode_weights(None, 1, 128, 128, 0x100, 0x100, 0x100, None) == -1
+
+
+def test_missing_library_fails_loudly():
+    """Without the built CUDA library the binding raises: there is no CPU or library fallback."""
+    saved_path, saved_lib = lmoe.LIB_PATH, lmoe._lib
+    try:
+        lmoe.LIB_PATH = os.path.join(os.path.dirname(saved_path), "no_such_liblmoe.so")
+        lmoe._lib = None
+        with pytest.raises(RuntimeError, match="not built"):
+            lmoe.lib()
+    finally:
+        lmoe.LIB_PATH, lmoe._lib = saved_path, saved_lib
