@@ -18,9 +18,10 @@
 // the few-token projections: the weight rows of `tmW` come first, those of
 // `tmW2` after them, and K may be split `k_splits` ways so that more CTAs
 // stream the weights (the host takes 512-deep slices, 128 KB of weights per
-// (tile, split) unit, at most one unit per SM).  With `partial` set, each (tile, split) writes its fp32
-// partial sums to partial[split][weight row][NT]; swap_reduce_kernel then adds
-// the splits in order (deterministic) and applies the epilogue.
+// (tile, split) unit, at most one unit per SM).  With `partial` set, each
+// (tile, split) writes its fp32 partial sums to partial[split][weight row][NT];
+// swap_reduce_kernel then adds the splits in order (deterministic) and applies
+// the epilogue.
 #pragma once
 #include "tc_gemm.cuh"
 
