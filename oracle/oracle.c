@@ -12,11 +12,10 @@
  *        f = x (the gate stays at the full width d: "LatentMoE: How MoE Made
  *        a Key Paradigm Leap in 2026", section 2 closing note; Kimi K3 /
  *        Nemotron 3 Super article, "LatentMoE 具体怎么做", closing note), or
- *        f = bf16(z) when the latent-router reading is selected ("routing
- *        happens in the latent", the same sections' second bullet).  The
- *        latent is stored in bf16 before the gate reads it, so the top-K'
- *        decision (an integer decided by floating point) is taken on the same
- *        bf16 input on both sides; everything else stays in fp64.
+ *        f = z (the fp64 latent of step 4) when the latent-router reading is
+ *        selected ("routing happens in the latent", the same sections'
+ *        second bullet).  The pages say nothing about the latent's precision,
+ *        so the gate reads it exactly, like every other step here.
  *   2. top-K' selection: the K' largest logits, ties to the lower expert id,
  *      slots ordered by (logit descending, id ascending).
  *   3. renormalised softmax over the selected logits
@@ -95,9 +94,8 @@ static int n_total(const oracle_cfg *c) { return c->n_ffn + c->n_zero + c->n_cop
 
 /* Round to the nearest bfloat16 (ties to even) through binary32, the way a
  * value accumulated in fp32 is stored as bf16.  Used only where the layer
- * stores a value before an integer decision is taken on it: the latent the
- * latent-router reading feeds to the gate (step 1), and the expert inputs
- * that are MX-encoded (step 9). */
+ * stores a value before an integer decision is taken on it: the expert inputs
+ * that are block-scale encoded (step 9). */
 static double round_bf16(double v)
 {
     float f = (float)v;
@@ -547,7 +545,6 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
     {
         double *xt = (double *)malloc(sizeof(double) * (size_t)d);
         double *z = (double *)malloc(sizeof(double) * (size_t)L);
-        double *zr = (double *)malloc(sizeof(double) * (size_t)L);
         double *lg = (double *)malloc(sizeof(double) * (size_t)Nt);
         double *u = (double *)malloc(sizeof(double) * (size_t)up_rows);
         double *h = (double *)malloc(sizeof(double) * (size_t)m);
@@ -561,7 +558,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
         double *so = (double *)malloc(sizeof(double) * (size_t)d);
         double *zq = (double *)malloc(sizeof(double) * (size_t)L);
         double *hq = (double *)malloc(sizeof(double) * (size_t)m);
-        if (!xt || !z || !zr || !lg || !u || !h || !o || !yl || !up || !w || !sel || !su || !sh || !so || !zq || !hq)
+        if (!xt || !z || !lg || !u || !h || !o || !yl || !up || !w || !sel || !su || !sh || !so || !zq || !hq)
             bad = 1;
 
 #pragma omp for schedule(dynamic, 1)
@@ -571,13 +568,8 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             /* step 4: latent projection (identity for the standard MoE) */
             if (c->has_proj) matvec(L, d, w_down, xt, z);
             else memcpy(z, xt, sizeof(double) * (size_t)d);
-            /* step 1: router logits at the full width (or on the bf16 latent) */
-            if (c->latent_router) {
-                for (int j = 0; j < L; ++j) zr[j] = round_bf16(z[j]);
-                matvec(Nt, fdim, w_router, zr, lg);
-            } else {
-                matvec(Nt, fdim, w_router, xt, lg);
-            }
+            /* step 1: router logits at the full width (or on the latent) */
+            matvec(Nt, fdim, w_router, c->latent_router ? z : xt, lg);
             if (bias)
                 for (int e = 0; e < Nt; ++e) lg[e] += (double)bias[e];
             /* steps 2-3 */
@@ -656,7 +648,7 @@ int oracle_forward(const oracle_cfg *c, int T, const uint16_t *x, const uint16_t
             if (logits_out) memcpy(logits_out + (size_t)t * Nt, lg, sizeof(double) * (size_t)Nt);
         }
         free(su); free(sh); free(so); free(zq); free(hq);
-        free(xt); free(z); free(zr); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
+        free(xt); free(z); free(lg); free(u); free(h); free(o); free(yl); free(up); free(w); free(sel);
     }
     free(c1); free(s1); free(c2); free(s2); free(g1); free(g2);
     return bad ? -1 : 0;

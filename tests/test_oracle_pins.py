@@ -150,9 +150,7 @@ def _dense_bruteforce(cfg, layer):
     W1, W2 = _np(layer["w1"]), _np(layer["w2"])
     T, m = x.shape[0], cfg.m
     z = x @ Wd.T if cfg.has_proj else x.copy()
-    # the latent router reads the latent stored in bf16 (round to nearest even through fp32)
-    z_gate = torch.from_numpy(z).to(torch.float32).to(torch.bfloat16).double().numpy()
-    lg = (z_gate if cfg.latent_router else x) @ Wr.T
+    lg = (z if cfg.latent_router else x) @ Wr.T
     if layer.get("bias") is not None:
         lg = lg + layer["bias"].double().numpy()
     U = np.einsum("eol,tl->teo", W1, z)
@@ -264,6 +262,40 @@ def test_latent_router_matches_dense_bruteforce():
     layer = synth.make_layer(cfg)
     out = oracle.forward(cfg, layer)
     np.testing.assert_allclose(out["y"], _dense_bruteforce(cfg, layer), rtol=1e-11, atol=1e-11)
+
+
+def test_latent_router_gate_reads_the_unrounded_latent():
+    """The gate takes the latent at full precision ("How LatentMoE Works" step 2 says nothing of a rounding).
+
+    z_0 = x_0 + 2^-10 x_1 = 1 + 2^-10 has no bf16 value (bf16 rounds it to 1).  Expert 0's logit is z_0,
+    expert 1's is the constant bias 1 + 2^-11.  On the exact latent expert 0 wins top-1; a gate that read
+    a bf16-rounded latent would pick expert 1.  The two experts differ (W2 of expert 1 is doubled), so
+    the layer output tells which one ran."""
+    cfg = synth.LayerConfig(d=8, latent=8, m=4, n_ffn=2, top_k=1, tokens=1, seed=12, latent_router=1)
+    layer = synth.make_layer(cfg)
+    x = torch.zeros(1, 8, dtype=torch.bfloat16)
+    x[0, 0] = 1.0
+    x[0, 1] = 1.0
+    wd = torch.eye(8, dtype=torch.bfloat16)
+    wd[0, 1] = 2.0 ** -10
+    wr = torch.zeros(2, 8, dtype=torch.bfloat16)
+    wr[0, 0] = 1.0
+    bias = torch.tensor([0.0, 1.0 + 2.0 ** -11], dtype=torch.float32)
+    w2 = layer["w2"].clone()
+    w2[1] = layer["w2"][0] * 2
+    w1 = layer["w1"].clone()
+    w1[1] = layer["w1"][0]
+    lay = dict(layer, x=x, w_down=wd, w_router=wr, bias=bias, w1=w1, w2=w2)
+    out = oracle.forward(cfg, lay, want=("y", "idx", "w", "z", "logits"))
+    assert out["z"][0, 0] == 1.0 + 2.0 ** -10
+    assert float(torch.tensor(out["z"][0, 0]).to(torch.bfloat16)) == 1.0
+    assert out["idx"][0, 0] == 0 and out["w"][0, 0] == 1.0
+    assert out["logits"][0, 0] == 1.0 + 2.0 ** -10 and out["logits"][0, 1] == np.float32(1.0 + 2.0 ** -11)
+    # expert 0's output on the exact latent (numpy fp64): y = x + W_up W2_0 relu(W1_0 z)^2
+    z = _np(x) @ _np(wd).T
+    h = np.maximum(z @ _np(w1[0]).T, 0) ** 2
+    y = _np(x) + (h @ _np(w2[0]).T) @ _np(lay["w_up"]).T
+    np.testing.assert_allclose(out["y"], y, rtol=1e-12, atol=1e-12)
 
 
 def test_identity_projections_reproduce_standard_moe():
