@@ -155,7 +155,7 @@ int ep_ranks(const lmoe_config& c) { return c.ep_size > 1 ? c.ep_size : 1; }
 int n_local_experts(const lmoe_config& c) { return c.n_experts / ep_ranks(c); }
 
 struct Plan {
-    size_t hdr, logits, z, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
+    size_t hdr, logits, z, zlo, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
         partial, hs, s2, partial2, rows4, rows_sf4, h4, h_sf4, rows8, rows_sf, h8, h_sf, xin, yout, ep_map, ep_src,
         ep_dst, ep_counts,
         ep_offsets, total;
@@ -185,6 +185,8 @@ Plan make_plan(const lmoe_config& c) {
     p.hdr = take(HDR_WORDS * 4);
     p.logits = take(T * p.ld_logits * 4);
     p.z = c.has_proj ? take(T * L * 2) : 0;
+    // latent router: the low bf16 part of the fp32 latent, so the gate reads z at ~16 significant bits
+    p.zlo = (c.has_proj && c.latent_router) ? take(T * L * 2) : 0;
     p.idx = take(T * K * 4);
     p.w = take(T * K * 4);
     p.bitmap = take(static_cast<size_t>(p.nwords) * nt * 4);
@@ -352,10 +354,12 @@ bool set_all_smem_attrs() {
     return ok;
 }
 
+// `x2`: the token operand of the k-blocks past args.k_wrap (nullptr: none, x stands in).
 template <int NT, int EPI>
 void launch_swap(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& w2, const SwapArgs& args, int grid,
-                 cudaStream_t s) {
-    launch(tc_swap_kernel<NT, EPI>, grid, 192, SwapCfg<NT, EPI>::SMEM_BYTES, s, w, x, w2, args);
+                 cudaStream_t s, const CUtensorMap* x2 = nullptr) {
+    launch(tc_swap_kernel<NT, EPI>, grid, 192, SwapCfg<NT, EPI>::SMEM_BYTES, s, w, x, w2, x2 != nullptr ? *x2 : x,
+           args);
 }
 
 // Weight-streaming launch for the experts of the small list, dispatched on the token tile and epilogue.
@@ -389,6 +393,11 @@ struct FewTokenGemm {
     int ld_resid;
     int act = EPI_BF16;     // activation of segment 0 (EPI_RELU2 / EPI_SWIGLU: gate rows first, then up rows)
     int out_cols0 = -1;     // output columns of segment 0 (default rows0; rows0 / 2 when gated)
+    __nv_bfloat16* out0_lo = nullptr;  // segment 0 without activation: also the low part bf16(v - bf16(v))
+    // two-part token operand: K = 2 * k_wrap, the k-blocks past k_wrap read x16b / x32b and the weights again
+    int k_wrap = 0;
+    const CUtensorMap* x16b = nullptr;
+    const CUtensorMap* x32b = nullptr;
     // router: with topk_idx set, segment 1 holds the router logits, and the reduction also selects each
     // token's top-K' (bias added) and writes ids and renormalised weights
     const float* bias = nullptr;
@@ -405,7 +414,7 @@ void launch_few_token_reduce(const FewTokenGemm& g, int T, const float* partial,
     const unsigned rgrid = static_cast<unsigned>((outs + 255) / 256);
 #define LMOE_REDUCE(A)                                                                                           \
     launch(swap_reduce_kernel<NT, A>, rgrid, 256, 0, s, partial, part_rows, splits, T, n0, g.rows1, t0 * 128, n0, \
-           g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid)
+           g.out0, g.ld0, g.out1, g.ld1, g.resid, g.ld_resid, A == EPI_BF16 ? g.out0_lo : nullptr)
     if (g.act == EPI_RELU2) LMOE_REDUCE(EPI_RELU2);
     else if (g.act == EPI_SWIGLU) LMOE_REDUCE(EPI_SWIGLU);
     else LMOE_REDUCE(EPI_BF16);
@@ -453,13 +462,14 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
     a.part_rows = (t0 + t1) * 128;
     a.err = err;
     a.timeout_ns = timeout_ns;
+    a.k_wrap = g.k_wrap;
     const int grid = std::min(num_sms, (t0 + t1) * splits);
     if (T <= 16) {
-        launch_swap<16, EPI_BF16>(*g.w, *g.x16, *g.w2, a, grid, s);
+        launch_swap<16, EPI_BF16>(*g.w, *g.x16, *g.w2, a, grid, s, g.k_wrap > 0 ? g.x16b : nullptr);
         if (g.topk_idx != nullptr) launch_router_reduce_topk<16>(g, T, partial, a.part_rows, splits, t0, s);
         else launch_few_token_reduce<16>(g, T, partial, a.part_rows, splits, t0, s);
     } else {
-        launch_swap<32, EPI_BF16>(*g.w, *g.x32, *g.w2, a, grid, s);
+        launch_swap<32, EPI_BF16>(*g.w, *g.x32, *g.w2, a, grid, s, g.k_wrap > 0 ? g.x32b : nullptr);
         if (g.topk_idx != nullptr) launch_router_reduce_topk<32>(g, T, partial, a.part_rows, splits, t0, s);
         else launch_few_token_reduce<32>(g, T, partial, a.part_rows, splits, t0, s);
     }
@@ -468,23 +478,26 @@ int launch_few_token(const FewTokenGemm& g, int T, float* partial, int max_split
 
 // `out` (optional): TMA map of the bf16 output (box 32 rows x 64 columns, 128-byte swizzle); the epilogue
 // then stores whole 32-row blocks with TMA (BN = 256).  Without it every thread stores its own row.
+// `a2` (optional): the A operand of the k-blocks past args.k_wrap.
 template <int BN, int EPI>
 void launch_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args, int grid,
-                 cudaStream_t s, const CUtensorMap* out = nullptr) {
+                 cudaStream_t s, const CUtensorMap* out = nullptr, const CUtensorMap* a2 = nullptr) {
     GemmArgs g = args;
     g.tma_store = (out != nullptr && BN == 256) ? 1 : 0;
-    launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, out != nullptr ? *out : a, g);
+    launch(tc_gemm_kernel<BN, EPI>, grid, 192, GemmCfg<BN>::SMEM_BYTES, s, a, b, b2, out != nullptr ? *out : a,
+           a2 != nullptr ? *a2 : a, g);
 }
 
 // CTA-pair GEMM: `pair_tiles` (or, for a device-built list, an upper bound) pair tiles on up to num_sms / 2 pairs.
 template <int EPI>
 void launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const GemmArgs& args,
-                      int pair_tiles, int num_sms, cudaStream_t s, const CUtensorMap* out = nullptr) {
+                      int pair_tiles, int num_sms, cudaStream_t s, const CUtensorMap* out = nullptr,
+                      const CUtensorMap* a2 = nullptr) {
     const int pairs = std::max(1, std::min(num_sms / 2, pair_tiles));
     GemmArgs g = args;
     g.tma_store = out != nullptr ? 1 : 0;
     launch_pairs(tc_gemm_pair_kernel<EPI>, 2 * pairs, 192, GemmPairCfg::SMEM_BYTES, s, a, b, b2,
-                 out != nullptr ? *out : a, g);
+                 out != nullptr ? *out : a, a2 != nullptr ? *a2 : a, g);
 }
 
 template <int EPI, bool W4, bool QOUT>
@@ -546,6 +559,8 @@ struct lmoe_handle {
     CUtensorMap w1s{}, w2s{}, rows16{}, rows32{}, h16{}, h32{};
     // few-token projections: 128-row weight tiles and 16/32-row token tiles of z and yl
     CUtensorMap wdown128{}, wr128{}, wup128{}, z16{}, z32{}, yl16{}, yl32{};
+    // latent router: the latent's low part as the second A operand (128-row tiles) and token operand (16/32)
+    CUtensorMap a_zlo{}, zlo16{}, zlo32{};
     // shared expert: weights for 64/256-column tiles (gated: half-tile boxes), 128-row weight tiles,
     // its hidden rows as the A operand (128-row tiles) and as 16/32-row token tiles
     CUtensorMap ws1_64{}, ws1_256{}, ws2_64{}, ws2_256{}, ws1_128{}, ws2_128{}, a_hs{}, hs16{}, hs32{};
@@ -727,10 +742,16 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
             r.topk_w = wts;
         };
         if (proj && c.latent_router) {
+            // z = hi + lo from the fp32 sum; the gate multiplies both parts (K = 2L, its weights streamed
+            // twice), so it reads the latent at ~16 significant bits instead of bf16's 8
             FewTokenGemm g{&h->wdown128, &h->wdown128, &x16, &x32, L, 0, d, z, L, nullptr, 0, nullptr, 0};
+            g.out0_lo = h->at<__nv_bfloat16>(p.zlo);
             launch_few_token(g, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
-            FewTokenGemm r{&h->wr128, &h->wr128, &h->z16, &h->z32, 0, nt, L, nullptr, 0, logits, p.ld_logits,
+            FewTokenGemm r{&h->wr128, &h->wr128, &h->z16, &h->z32, 0, nt, 2 * L, nullptr, 0, logits, p.ld_logits,
                            nullptr, 0};
+            r.k_wrap = L;
+            r.x16b = &h->zlo16;
+            r.x32b = &h->zlo32;
             with_topk(r);
             launch_few_token(r, T, part, kFewTokenMaxSplits, h->num_sms, hdr + HDR_ERR, h->timeout_ns, s);
         } else if (fused) {
@@ -750,12 +771,14 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
             const int n_gemm = (proj && c.latent_router) ? 2 : 1;
             PhaseScope ps(h, PH_ROUTER, s, n_gemm);
             if (proj && c.latent_router) {
+                // z (bf16) and its low part zlo = bf16(z32 - z) from the fp32 accumulator
                 GemmArgs a = base;
                 a.M = T;
                 a.K = d;
                 a.N0 = L;
                 a.out0 = z;
                 a.ld0 = L;
+                a.out_lo = h->at<__nv_bfloat16>(p.zlo);
                 if (big) {
                     a.n_tiles = (L + 255) / 256;
                     launch_gemm<256, EPI_BF16>(a_x, h->wdown256, h->wdown256, a, std::min(h->num_sms, m_tiles * a.n_tiles), s);
@@ -767,6 +790,10 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
             GemmArgs a = base;
             a.M = T;
             a.K = c.latent_router ? L : d;
+            if (proj && c.latent_router) {  // the gate reads z + zlo: K = 2L, the router weights read twice
+                a.K = 2 * L;
+                a.k_wrap = L;
+            }
             a.N0 = fused ? L : 0;
             a.N1 = nt;
             a.out0 = z;
@@ -778,12 +805,14 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
                 a.n_tiles0 = fused ? (L + 255) / 256 : 0;
                 a.n_tiles = a.n_tiles0 + (nt + 255) / 256;
                 launch_gemm_pair<EPI_PROJ_ROUTER>(A, fused ? h->wdown128 : h->wr128, h->wr128, a,
-                                                  (T + 255) / 256 * a.n_tiles, h->num_sms, s, fused ? &h->o_z : nullptr);
+                                                  (T + 255) / 256 * a.n_tiles, h->num_sms, s, fused ? &h->o_z : nullptr,
+                                                  a.k_wrap > 0 ? &h->a_zlo : nullptr);
             } else {
                 a.n_tiles0 = fused ? (L + 63) / 64 : 0;
                 a.n_tiles = a.n_tiles0 + (nt + 63) / 64;
                 launch_gemm<64, EPI_PROJ_ROUTER>(A, fused ? h->wdown64 : h->wr64, h->wr64, a,
-                                                 std::min(h->num_sms, m_tiles * a.n_tiles), s);
+                                                 std::min(h->num_sms, m_tiles * a.n_tiles), s, nullptr,
+                                                 a.k_wrap > 0 ? &h->a_zlo : nullptr);
             }
         }
     }
@@ -1282,6 +1311,11 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
         ok &= make_map(&h->z32, h->at<void>(p.z), c.max_tokens, L, L, 32);
         ok &= make_map(&h->yl16, h->at<void>(p.yl), c.max_tokens, L, L, 16);
         ok &= make_map(&h->yl32, h->at<void>(p.yl), c.max_tokens, L, L, 32);
+        if (c.latent_router) {
+            ok &= make_map(&h->a_zlo, h->at<void>(p.zlo), c.max_tokens, L, L, 128);
+            ok &= make_map(&h->zlo16, h->at<void>(p.zlo), c.max_tokens, L, L, 16);
+            ok &= make_map(&h->zlo32, h->at<void>(p.zlo), c.max_tokens, L, L, 32);
+        }
     }
     const uint64_t w1_rows = static_cast<uint64_t>(h->n_local) * h->g * m, w2_rows = static_cast<uint64_t>(h->n_local) * L;
     if (c.expert_fmt == LMOE_FMT_BF16) {
@@ -1476,7 +1510,7 @@ int lmoe_last_error(lmoe_handle* h) {
     if (cudaMemcpy(&err, dev, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return LMOE_ERR_CUDA;
     if (err != 0 && cudaMemset(dev, 0, 4) != cudaSuccess) return LMOE_ERR_CUDA;
     if (err & DEVERR_TIMEOUT) return LMOE_ERR_TIMEOUT;
-    if (err & DEVERR_BAD_INDEX) return LMOE_ERR_BAD_INDEX;
+    if (err & (DEVERR_BAD_INDEX | DEVERR_REPEATED_INDEX)) return LMOE_ERR_BAD_INDEX;
     if (err & DEVERR_BAD_COUNTS) return LMOE_ERR_BAD_COUNTS;
     return LMOE_OK;
 }

@@ -47,6 +47,13 @@ struct GemmArgs {
     const __nv_bfloat16* resid;
     int ld_resid;
     int tma_store;         // 1: bf16 out0 rows leave through shared-memory staging and TMA stores (BN = 256)
+    // Two-part A: with k_wrap > 0 the reduction runs over K = 2 * k_wrap; k-blocks at or past k_wrap take
+    // their A tile from tmA2 and their B tile from k - k_wrap, so the product is (A + A2) * B^T with B read
+    // twice.  A bf16 split A = hi + lo of an fp32 operand then multiplies at ~16 significant bits.
+    int k_wrap;
+    // EPI_BF16 without TMA stores: also write out_lo = bf16(acc - bf16(acc)), the low part of the fp32
+    // accumulator (ld0 is its row pitch too)
+    __nv_bfloat16* out_lo;
     int* err;
     unsigned long long timeout_ns;
 };
@@ -250,11 +257,21 @@ __device__ __forceinline__ void gemm_epilogue_store(const GemmArgs& args, const 
             }
             if (col >= args.N0) continue;
             uint4 q[8];
+            const bool lo_out = EPI == EPI_BF16 && args.out_lo != nullptr && !tma_rows;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 float f[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v2[h][i]);
+                if (lo_out) {
+                    // the rounding error of each bf16 output, exact in fp32, itself stored in bf16
+                    float r[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = f[i] - __bfloat162float(__float2bfloat16_rn(f[i]));
+                    uint4* dlo = reinterpret_cast<uint4*>(args.out_lo + row * args.ld0 + col + 32 * h);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dlo[i] = pack8(r + 8 * i);
+                }
                 if (EPI == EPI_RELU2) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) f[i] = act_relu2(f[i]);
@@ -295,7 +312,7 @@ template <int BN, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
-                   const GemmArgs args) {
+                   const __grid_constant__ CUtensorMap tmA2, const GemmArgs args) {
     pdl_begin();
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
@@ -333,6 +350,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         if (EPI == EPI_PROJ_ROUTER) tma_prefetch_desc(&tmB2);
+        if (args.k_wrap > 0) tma_prefetch_desc(&tmA2);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
     tc_fence_before();
@@ -360,13 +378,15 @@ __global__ void __launch_bounds__(192, 1)
                         ok = false;
                         break;
                     }
+                    const bool a2 = args.k_wrap > 0 && kb * C::BK >= args.k_wrap;
+                    const int kx = a2 ? kb * C::BK - args.k_wrap : kb * C::BK;
                     mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
-                    tma_load_2d(sA + s * C::A_BYTES, &tmA, &full[s], kb * C::BK, j.a_row0);
+                    tma_load_2d(sA + s * C::A_BYTES, a2 ? &tmA2 : &tmA, &full[s], kx, j.a_row0);
                     if (EPI == EPI_SWIGLU) {
-                        tma_load_2d(sB + s * C::B_BYTES, bmap, &full[s], kb * C::BK, j.b_row0);
-                        tma_load_2d(sB + s * C::B_BYTES + C::B_BYTES / 2, bmap, &full[s], kb * C::BK, j.b_row1);
+                        tma_load_2d(sB + s * C::B_BYTES, bmap, &full[s], kx, j.b_row0);
+                        tma_load_2d(sB + s * C::B_BYTES + C::B_BYTES / 2, bmap, &full[s], kx, j.b_row1);
                     } else {
-                        tma_load_2d(sB + s * C::B_BYTES, bmap, &full[s], kb * C::BK, j.b_row0);
+                        tma_load_2d(sB + s * C::B_BYTES, bmap, &full[s], kx, j.b_row0);
                     }
                     issued[s] = true;
                     last_parity[s] = ph;
@@ -536,7 +556,7 @@ template <int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
-                        const GemmArgs args) {
+                        const __grid_constant__ CUtensorMap tmA2, const GemmArgs args) {
     pdl_begin();
     using C = GemmPairCfg;
     constexpr int BN = C::BN;
@@ -577,6 +597,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmA);
         tma_prefetch_desc(&tmB);
         if (EPI == EPI_PROJ_ROUTER) tma_prefetch_desc(&tmB2);
+        if (args.k_wrap > 0) tma_prefetch_desc(&tmA2);
     }
     if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
     tc_fence_before();
@@ -607,8 +628,10 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * (C::A_BYTES + C::B_BYTES));
                     const uint32_t fb = mapa_shared(&full[s], 0);
-                    tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, fb, kb * C::BK, j.a_row0);
-                    tma_load_2d_pair(sB + s * C::B_BYTES, bmap, fb, kb * C::BK, j.b_row0);
+                    const bool a2 = args.k_wrap > 0 && kb * C::BK >= args.k_wrap;
+                    const int kx = a2 ? kb * C::BK - args.k_wrap : kb * C::BK;
+                    tma_load_2d_pair(sA + s * C::A_BYTES, a2 ? &tmA2 : &tmA, fb, kx, j.a_row0);
+                    tma_load_2d_pair(sB + s * C::B_BYTES, bmap, fb, kx, j.b_row0);
                     issued[s] = true;
                     last_parity[s] = ph;
                 }

@@ -44,6 +44,10 @@ struct SwapArgs {
     int ld_out;
     int* err;
     unsigned long long timeout_ns;
+    // Two-part token operand (dense mode): with k_wrap > 0, K = 2 * k_wrap and k-blocks at or past k_wrap
+    // read their token tile from tmX2 and their weight tile at k - k_wrap: W * (X + X2)^T, the weights
+    // streamed twice.
+    int k_wrap;
 };
 
 template <int NT, int EPI>
@@ -109,7 +113,8 @@ __device__ __forceinline__ void swap_job(const SwapArgs& a, int t, int nkb, Swap
 template <int NT, int EPI>
 __global__ void __launch_bounds__(192, 1)
     tc_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
-                   const __grid_constant__ CUtensorMap tmW2, const SwapArgs args) {
+                   const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmX2,
+                   const SwapArgs args) {
     pdl_begin();
     using C = SwapCfg<NT, EPI>;
     extern __shared__ uint8_t smem_raw[];
@@ -144,6 +149,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_prefetch_desc(&tmW);
         tma_prefetch_desc(&tmX);
         if (args.list == nullptr) tma_prefetch_desc(&tmW2);
+        if (args.k_wrap > 0) tma_prefetch_desc(&tmX2);
     }
     if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
     tc_fence_before();
@@ -172,10 +178,12 @@ __global__ void __launch_bounds__(192, 1)
                         break;
                     }
                     uint8_t* st = smem + s * C::STAGE_BYTES;
+                    const bool x2 = args.k_wrap > 0 && kb * C::BK >= args.k_wrap;
+                    const int kx = x2 ? kb * C::BK - args.k_wrap : kb * C::BK;
                     mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d(st, wmap, &full[s], kb * C::BK, j.wrow);
-                    if (C::NA == 2) tma_load_2d(st + C::A_BYTES, wmap, &full[s], kb * C::BK, j.wrow + args.up_offset);
-                    tma_load_2d(st + C::NA * C::A_BYTES, &tmX, &full[s], kb * C::BK, j.e.y);
+                    tma_load_2d(st, wmap, &full[s], kx, j.wrow);
+                    if (C::NA == 2) tma_load_2d(st + C::A_BYTES, wmap, &full[s], kx, j.wrow + args.up_offset);
+                    tma_load_2d(st + C::NA * C::A_BYTES, x2 ? &tmX2 : &tmX, &full[s], kx, j.e.y);
                     issued[s] = true;
                     last_parity[s] = ph;
                 }
@@ -298,13 +306,15 @@ __global__ void __launch_bounds__(192, 1)
 //   n < n0:             out0[t][n] = bf16(act(sum) (+ resid[t][n] when resid is set)), partial row n
 //   n0 <= n < n0 + n1:  out1[t][n - n0] = sum (fp32 router logits), partial row p1 + (n - n0)
 // ACT: EPI_BF16 (none), EPI_RELU2, or EPI_SWIGLU (gate = partial row n, up =
-// partial row up_row0 + n).
+// partial row up_row0 + n).  out0_lo (optional, ACT = EPI_BF16 without resid):
+// out0_lo[t][n] = bf16(sum - bf16(sum)), the low part of the fp32 sum.
 template <int NT, int ACT>
 __global__ void __launch_bounds__(256) swap_reduce_kernel(const float* __restrict__ partial, int part_rows, int splits,
                                                           int T, int n0, int n1, int p1, int up_row0,
                                                           __nv_bfloat16* __restrict__ out0, int ld0,
                                                           float* __restrict__ out1, int ld1,
-                                                          const __nv_bfloat16* __restrict__ resid, int ld_resid) {
+                                                          const __nv_bfloat16* __restrict__ resid, int ld_resid,
+                                                          __nv_bfloat16* __restrict__ out0_lo) {
     pdl_begin();
     const long i = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int cols = n0 + n1;
@@ -327,7 +337,9 @@ __global__ void __launch_bounds__(256) swap_reduce_kernel(const float* __restric
     }
     if (n < n0) {
         if (resid != nullptr) v += __bfloat162float(resid[static_cast<size_t>(t) * ld_resid + n]);
-        out0[static_cast<size_t>(t) * ld0 + n] = __float2bfloat16_rn(v);
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        out0[static_cast<size_t>(t) * ld0 + n] = hi;
+        if (out0_lo != nullptr) out0_lo[static_cast<size_t>(t) * ld0 + n] = __float2bfloat16_rn(v - __bfloat162float(hi));
     } else {
         out1[static_cast<size_t>(t) * ld1 + (n - n0)] = v;
     }

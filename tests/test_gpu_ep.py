@@ -13,6 +13,8 @@
 * Counts that do not match the rows are reported as LMOE_ERR_BAD_COUNTS, and
   the stage then computes nothing; bad calls are rejected.
 """
+import warnings
+
 import numpy as np
 import pytest
 import torch
@@ -111,7 +113,7 @@ def test_emulated_ranks_match_the_oracle(name):
             torch.cuda.synchronize()
             gidx, gw = dbg["idx"].cpu().numpy(), dbg["w"].cpu().numpy()
             ref = oracle.forward(cfg, layer, x=x, want=("y", "idx", "w", "logits"))
-            differ = P.check_routing(gidx, gw, ref, cfg.top_k, w_atol=1e-3 if cfg.latent_router else 2e-5)
+            differ = P.check_routing(gidx, gw, ref, cfg.top_k, w_atol=2e-5)
             if differ.any():
                 ref2 = oracle.forward(cfg, layer, x=x, idx=gidx, want=("y",))
                 ref["y"] = np.where(differ[:, None], ref2["y"], ref["y"])
@@ -120,7 +122,10 @@ def test_emulated_ranks_match_the_oracle(name):
             emulated = None
             if m["max_err"] > P.MAX_ERR_VS_RMS * m["rms_ref"]:
                 emulated = P.emulate_bf16(cfg, layer, x, gidx, gw)
-            P.assert_layer_close(got, ref["y"], emulated, f"rank {r} y")
+            m = P.assert_layer_close(got, ref["y"], emulated, f"rank {r} y")
+            if "bf16_storage_max_err" in m:
+                warnings.warn(f"bf16-storage allowance used by {name} rank {r}: max_err {m['max_err']:.4g}; "
+                              f"bf16 storage alone {m['bf16_storage_max_err']:.4g}")
     finally:
         _close(ranks + [single])
 

@@ -6,6 +6,8 @@ benchmark times) and are compared on a seeded sample of tokens (tokens are
 independent: no capacity, no dropping), plus properties that hold at any size
 (dispatch bit-exact, weights sum to one, determinism).
 """
+import warnings
+
 import numpy as np
 import pytest
 import torch
@@ -45,6 +47,11 @@ CASES = {
     "std_decode": synth.WORKLOADS["std_decode"],
 }
 
+# The layer configurations the contract names (tiny, the Nemotron-like decode and prefill batches, the
+# standard MoE at both sizes, the Kimi-like skewed layer): these meet the plain tolerances, with no
+# bf16-storage allowance.
+CONTRACT = {"tiny", "nemotron_decode", "nemotron_prefill", "std_decode", "std_prefill", "kimi_skew"}
+
 _layers = {}
 
 
@@ -54,7 +61,11 @@ def _layer(name, cfg):
     return _layers[name]
 
 
-def _run_and_check(cfg, layer, small_rows=None, sample=None):
+def _run_and_check(cfg, layer, small_rows=None, sample=None, label=None):
+    """Forward through the C ABI and compare with the oracle.  ``label`` names the case: a name in
+    CONTRACT is held to the plain tolerances; any other case may use the bf16-storage allowance, and a
+    warning records each case that does, with both errors."""
+    label = label or cfg.name
     T = int(layer["x"].shape[0])
     mod = lmoe.LatentMoE(cfg, layer, max_tokens=max(T, 1))
     try:
@@ -72,11 +83,9 @@ def _run_and_check(cfg, layer, small_rows=None, sample=None):
         rows = np.arange(T) if sample is None else sample
         xs = layer["x"][rows]
         ref = oracle.forward(cfg, layer, x=xs, want=("y", "idx", "w", "logits", "z", "yl"))
-        # With the latent router the gate reads the bf16 latent: where the GPU's fp32-accumulated z and the
-        # oracle's fp64 z round to neighbouring bf16 values, a logit moves by ~W_r * ulp(z) ~ 1e-4..1e-3,
-        # and the renormalised weights by as much; elsewhere the weights are fp32 softmaxes of fp32 logits.
-        w_atol = 1e-3 if cfg.latent_router else 2e-5
-        differ = P.check_routing(gidx[rows], gw[rows], ref, cfg.top_k, w_atol=w_atol)
+        # The weights are fp32 softmaxes of fp32 logits; with the latent router the gate reads the latent
+        # as a bf16 hi + lo pair of the fp32 latent (~16 significant bits), against the oracle's fp64 latent.
+        differ = P.check_routing(gidx[rows], gw[rows], ref, cfg.top_k, w_atol=2e-5)
         # logits (the GPU debug copy excludes the bias)
         lg_ref = ref["logits"] - (0 if layer["bias"] is None else layer["bias"].double().numpy())
         P.assert_close(P.to_np(dbg["logits"])[rows], lg_ref, "logits", max_vs_rms=2e-3, mean_rel=1e-3)
@@ -89,11 +98,17 @@ def _run_and_check(cfg, layer, small_rows=None, sample=None):
             # yl carries four bf16 storage roundings (z, H, O, yl): a diagnostic bound, not the contract
             P.assert_close(P.to_np(dbg["yl"])[rows], ref["yl"], "yl", max_vs_rms=6e-2, mean_rel=1e-2)
         got = P.to_np(y)[rows]
+        if label in CONTRACT:
+            return P.assert_close(got, ref["y"], f"{label} y"), y, dbg
         m = P.metrics(got, ref["y"])
         emulated = None
         if m["max_err"] > P.MAX_ERR_VS_RMS * m["rms_ref"]:
             emulated = P.emulate_bf16(cfg, layer, xs, gidx[rows], gw[rows])
-        m = P.assert_layer_close(got, ref["y"], emulated, "y")
+        m = P.assert_layer_close(got, ref["y"], emulated, f"{label} y")
+        if "bf16_storage_max_err" in m:
+            warnings.warn(f"bf16-storage allowance used by {label}: max_err {m['max_err']:.4g} > "
+                          f"{P.MAX_ERR_VS_RMS * m['rms_ref']:.4g} (2e-2 RMS); bf16 storage alone "
+                          f"{m['bf16_storage_max_err']:.4g}; mean_rel {m['mean_rel']:.3g}")
         return m, y, dbg
     finally:
         mod.close()
@@ -103,7 +118,7 @@ def _run_and_check(cfg, layer, small_rows=None, sample=None):
 @pytest.mark.parametrize("name", list(CASES))
 def test_layer_parity(name, small_rows):
     cfg = CASES[name]
-    _run_and_check(cfg, _layer(name, cfg), small_rows=small_rows)
+    _run_and_check(cfg, _layer(name, cfg), small_rows=small_rows, label=name)
 
 
 @pytest.mark.parametrize("name", ["nemotron_prefill", "std_prefill", "kimi_skew"])
@@ -113,7 +128,7 @@ def test_full_size_parity_on_sampled_tokens(name):
     rng = np.random.default_rng(1234)
     sample = np.sort(rng.choice(cfg.tokens, size=48, replace=False))
     sample[-1] = cfg.tokens - 1  # include the ragged end of the last tile
-    _run_and_check(cfg, layer, sample=sample)
+    _run_and_check(cfg, layer, sample=sample, label=name)
 
 
 def test_deterministic_and_host_entry_point_agree():

@@ -50,7 +50,7 @@ CASES = {
 @pytest.mark.parametrize("name", list(CASES))
 def test_mx_layer_parity(name):
     cfg = CASES[name]
-    _run_and_check(cfg, synth.make_layer(cfg))
+    _run_and_check(cfg, synth.make_layer(cfg), label=name)
 
 
 def _detile_scales(s: np.ndarray, rows: int, K: int) -> np.ndarray:

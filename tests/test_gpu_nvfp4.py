@@ -43,7 +43,7 @@ CASES = {
 @pytest.mark.parametrize("name", list(CASES))
 def test_nvfp4_layer_parity(name):
     cfg = CASES[name]
-    _run_and_check(cfg, synth.make_layer(cfg))
+    _run_and_check(cfg, synth.make_layer(cfg), label=name)
 
 
 def _detile_scales(s: np.ndarray, rows: int, K: int) -> np.ndarray:
