@@ -293,7 +293,8 @@ static __global__ void __launch_bounds__(256) dispatch_bitmap_kernel(const int32
                 atomicOr(&hdr[HDR_ERR], DEVERR_BAD_INDEX);
                 continue;
             }
-            atomicOr(&mine[e], 1u << lane);
+            // only this lane sets its bit: finding it set means this token named e before
+            if (atomicOr(&mine[e], 1u << lane) & (1u << lane)) atomicOr(&hdr[HDR_ERR], DEVERR_REPEATED_INDEX);
         }
     }
     __syncwarp();
@@ -441,7 +442,8 @@ __device__ __forceinline__ void dispatch_small_body(const int32_t* __restrict__ 
             atomicOr(&hdr[HDR_ERR], DEVERR_BAD_INDEX);
             continue;
         }
-        atomicOr(&bits[(t >> 5) * n_tot + e], 1u << (t & 31));
+        const uint32_t bit = 1u << (t & 31);  // set by token t's slots only: found set, t named e twice
+        if (atomicOr(&bits[(t >> 5) * n_tot + e], bit) & bit) atomicOr(&hdr[HDR_ERR], DEVERR_REPEATED_INDEX);
     }
     __syncthreads();
     const int e = threadIdx.x;

@@ -12,6 +12,7 @@ enum : int {
     DEVERR_TIMEOUT = 1,    // a bounded wait gave up
     DEVERR_BAD_INDEX = 2,  // an expert id outside [0, n_total)
     DEVERR_BAD_COUNTS = 4, // received row counts of the expert-parallel experts stage are inconsistent
+    DEVERR_REPEATED_INDEX = 8,  // one token's row names the same expert twice
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -16,6 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "liblmoe.so")
 
 LMOE_OK = 0
+#: device error bits of lmoe_dispatch_noalloc's error word
+LMOE_DEVERR_BAD_INDEX = 2
+LMOE_DEVERR_REPEATED_INDEX = 8
 LMOE_FMT_BF16, LMOE_FMT_MXFP8, LMOE_FMT_MXFP4, LMOE_FMT_NVFP4 = 0, 1, 2, 3
 STATUS = {0: "LMOE_OK", -1: "LMOE_ERR_INVALID_ARG", -2: "LMOE_ERR_UNSUPPORTED_SHAPE", -3: "LMOE_ERR_TOO_MANY_TOKENS",
           -4: "LMOE_ERR_CUDA", -5: "LMOE_ERR_TIMEOUT", -6: "LMOE_ERR_BAD_INDEX", -7: "LMOE_ERR_WORKSPACE",
@@ -79,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_set_wait_timeout.argtypes = [P, ctypes.c_uint64]
         L.lmoe_set_graph_launch.argtypes = [P, ctypes.c_int]
         L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
-        L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P]
+        L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P, P]
         L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
         L.lmoe_mx_encode_weights.argtypes = [P, ctypes.c_int64, I32, I32, P, P, P]
         L.lmoe_nvfp4_encode_weights.argtypes = [P, I32, ctypes.c_int64, I32, P, P, P, P]
@@ -196,13 +199,32 @@ def lmoe_gemm_bf16(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor, err: torch
                                                   err.data_ptr()))
 
 
+def _int32_buffer(name: str, t: torch.Tensor, device: torch.device, numel: int) -> None:
+    """Raise ValueError unless ``t`` is a contiguous int32 tensor on ``device`` with at least ``numel`` elements."""
+    if not isinstance(t, torch.Tensor) or t.dtype != torch.int32 or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name}: a contiguous int32 tensor on {device} is required")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: {t.numel()} elements, at least {numel} required")
+
+
 def lmoe_dispatch_noalloc(idx: torch.Tensor, n_total: int, counts: torch.Tensor, offsets: torch.Tensor,
-                          perm: torch.Tensor, inv: torch.Tensor, stream=None) -> None:
+                          perm: torch.Tensor, inv: torch.Tensor, err: Optional[torch.Tensor] = None,
+                          stream=None) -> None:
     """Expert counting sort of ``idx`` [T, top_k] (int32, device) into caller buffers, with no device
-    allocation: the library's fixed scratch array serves as workspace (see ``include/lmoe.h``)."""
+    allocation: the library's fixed scratch array serves as workspace (see ``include/lmoe.h``).  ``err``
+    (optional, one int32 on the device) receives the call's device error bits (``LMOE_DEVERR_*``)."""
+    if idx.dim() != 2 or idx.device.type != "cuda":
+        raise ValueError("idx: a [T, top_k] tensor on a CUDA device is required")
     T, K = idx.shape
+    _int32_buffer("idx", idx, idx.device, T * K)
+    _int32_buffer("counts", counts, idx.device, n_total)
+    _int32_buffer("offsets", offsets, idx.device, n_total + 1)
+    _int32_buffer("perm", perm, idx.device, T * K)
+    _int32_buffer("inv", inv, idx.device, T * K)
+    if err is not None:
+        _int32_buffer("err", err, idx.device, 1)
     _check("lmoe_dispatch_noalloc", lib().lmoe_dispatch_noalloc(
-        _p(idx), T, K, n_total, _p(counts), _p(offsets), _p(perm), _p(inv), _stream(stream)))
+        _p(idx), T, K, n_total, _p(counts), _p(offsets), _p(perm), _p(inv), _p(err), _stream(stream)))
 
 
 def lmoe_mx_encode_weights(w: torch.Tensor, fmt: int, stream=None):

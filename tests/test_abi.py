@@ -179,3 +179,30 @@ def test_missing_library_fails_loudly():
             lmoe.lib()
     finally:
         lmoe.LIB_PATH, lmoe._lib = saved_path, saved_lib
+
+
+def test_noalloc_binding_checks_its_buffers_before_any_call():
+    """The binding rejects host tensors, wrong dtypes, non-contiguous or short buffers with ValueError
+    before it reaches the library (a short perm or inv would let the scatter write past its end)."""
+    import torch
+
+    idx = torch.zeros((4, 2), dtype=torch.int32)
+    buf = torch.zeros(16, dtype=torch.int32)
+    with pytest.raises(ValueError):
+        lmoe.lmoe_dispatch_noalloc(idx, 8, buf, buf, buf, buf)       # host tensors
+    with pytest.raises(ValueError):
+        lmoe.lmoe_dispatch_noalloc(idx.reshape(-1), 8, buf, buf, buf, buf)  # idx not [T, top_k]
+    meta = dict(dtype=torch.int32, device="meta")
+    idm, ok = torch.empty((4, 2), **meta), torch.empty(16, **meta)
+    # the device check runs first for anything that is not a CUDA tensor
+    with pytest.raises(ValueError):
+        lmoe.lmoe_dispatch_noalloc(idm, 8, ok, ok, ok, ok)
+    e = lmoe._int32_buffer
+    dev = torch.device("meta")
+    with pytest.raises(ValueError):
+        e("perm", torch.empty(7, **meta), dev, 8)                    # short
+    with pytest.raises(ValueError):
+        e("perm", torch.empty(8, dtype=torch.int64, device="meta"), dev, 8)  # dtype
+    with pytest.raises(ValueError):
+        e("perm", torch.empty((4, 4), **meta).t(), dev, 8)           # not contiguous
+    e("perm", torch.empty(8, **meta), dev, 8)                         # accepted
