@@ -40,7 +40,11 @@ from latent_mixture_experts_gemm_b200 import lmoe, synth  # noqa: E402
 
 METRIC = "LatentMoE layer tokens/s at 1 B200 (prefill & decode); % of BF16/HBM roofline"
 DEFAULT_WORKLOAD = "nemotron_decode"
-SECONDARY_WORKLOAD = "nemotron_prefill"
+#: the other layer configurations, each measured in the same run and reported under `secondary`: the
+#: Nemotron-like prefill, the standard MoE at equal budget (prefill and decode), the Kimi-like skewed layer
+#: with MoE++ experts, and the Nemotron-like decode batch with NVFP4 and MXFP4 expert weights
+SECONDARY_WORKLOADS = ("nemotron_prefill", "std_prefill", "std_decode", "kimi_skew", "nemotron_decode_nvfp4",
+                       "nemotron_decode_mxfp4")
 N_INPUT_BATCHES = 4  # distinct token batches cycled through the steps
 
 
@@ -78,14 +82,14 @@ def clock_summary(samples, max_mhz, nvml):
 class ClockSampler:
     """SM clock and throttle reasons sampled while the timed region runs (read-only queries).
 
-    NVML, the library nvidia-smi reads, is polled every 2 ms from a thread, so even the ~15 ms of K decode
-    steps get several samples.  Without NVML, nvidia-smi runs every 200 ms instead.
+    NVML, the library nvidia-smi reads, is polled every 0.5 ms from a thread, so even the ~6 ms of 20 decode
+    steps get a dozen samples.  Without NVML, nvidia-smi runs every 200 ms instead.
     """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    PERIOD_S = 0.002
+    PERIOD_S = 0.0005
 
     def __init__(self, device_uuid: str):
         self.uuid = device_uuid
@@ -144,7 +148,7 @@ class ClockSampler:
             except Exception:
                 max_mhz = None
             out = clock_summary(self.samples, max_mhz, self.nvml)
-            out["source"] = "nvml, every 2 ms"
+            out["source"] = "nvml, every 0.5 ms"
             return out
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
@@ -246,7 +250,12 @@ def layer_work(cfg, stats, T):
 
 
 def phase_units(cfg, stats, T, phase):
-    """Algorithmic (flops, bytes) of one launch of a phase's kernel."""
+    """Algorithmic (flops, bytes) of one launch of a phase's kernel.
+
+    The expert phases count the weights of the experts they touch as their bytes: the gathered rows they read
+    and the hidden rows / expert outputs they write are the layer's intermediates, implementation traffic like
+    the ncu `traffic` figure, not algorithmic bytes.  So a grouped GEMM on a prefill batch is tensor-bound
+    (thousands of FLOPs per weight byte), and a weight stream on a decode batch HBM-bound."""
     g = 2 if cfg.gated else 1
     d, L, m, nt = cfg.d, cfg.latent, cfg.m, cfg.n_total
     fmt = getattr(cfg, "expert_fmt", 0)
@@ -257,13 +266,13 @@ def phase_units(cfg, stats, T, phase):
     e_tc = stats.get("tc_experts", 0)
     e_st = stats.get("stream_experts", 0)
     if phase == "expert_up_gemm":
-        return 2.0 * rows_tc * fin * g * m, 2.0 * (g * m * fin * e_tc + rows_tc * fin + rows_tc * m)
+        return 2.0 * rows_tc * fin * g * m, 2.0 * g * m * fin * e_tc
     if phase == "expert_down_gemm":
-        return 2.0 * rows_tc * m * fin, 2.0 * (fin * m * e_tc + rows_tc * m + rows_tc * fin)
-    if phase == "expert_up_stream":  # block-scaled: MXFP8 rows in, MXFP8 hidden rows out
-        return 2.0 * rows_st * fin * g * m, wb * g * m * fin * e_st + ab * (rows_st * fin + rows_st * m)
-    if phase == "expert_down_stream":  # bf16 rows out
-        return 2.0 * rows_st * m * fin, wb * fin * m * e_st + ab * rows_st * m + 2.0 * rows_st * fin
+        return 2.0 * rows_tc * m * fin, 2.0 * fin * m * e_tc
+    if phase == "expert_up_stream":
+        return 2.0 * rows_st * fin * g * m, wb * g * m * fin * e_st
+    if phase == "expert_down_stream":
+        return 2.0 * rows_st * m * fin, wb * fin * m * e_st
     if phase == "router_proj_gemm":
         n_out = (L if cfg.has_proj else 0) + nt
         return 2.0 * T * d * n_out, 2.0 * (n_out * d + T * d) + T * (L * 2 if cfg.has_proj else 0) + 4.0 * T * nt
@@ -289,9 +298,13 @@ def rooflines(cfg, stats, T, phases, peaks, step_ms):
     per_launch_ms = dom_ms / max(dom_n, 1)
     intensity = flops / max(nbytes, 1.0)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if "gemm" in dom and intensity >= ridge:
-        roof = {"bound": "tensor", "achieved": flops / (per_launch_ms / 1e3) / 1e12, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
+    fmt = getattr(cfg, "expert_fmt", 0)
+    rate = EXPERT_RATE[fmt] if dom.startswith("expert_") else 1.0
+    if intensity >= ridge * rate:
+        # a contraction takes the peak of its own dtype: block-scaled expert GEMMs run at the nominal
+        # fp8 / fp4 : bf16 ratio times the measured bf16 peak
+        roof = {"bound": "tensor", "achieved": flops / (per_launch_ms / 1e3) / 1e12,
+                "peak": peaks["bf16_tflops"] * rate, "unit": "TFLOP/s"}
     else:
         roof = {"bound": "hbm", "achieved": nbytes / (per_launch_ms / 1e3) / 1e9, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s"}
@@ -300,7 +313,8 @@ def rooflines(cfg, stats, T, phases, peaks, step_ms):
     roof["launch_ms"] = per_launch_ms
     roof["algorithmic_per_launch"] = {"flops": flops, "bytes": nbytes}
     roof["traffic"] = NCU_TRAFFIC.get((cfg.name, dom))
-    roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "")
+    roof["peak_source"] = peaks["source"] + (" (burst)" if roof["bound"] == "tensor" else "") + (
+        f", bf16 x {rate:g} (nominal ratio of the expert dtype)" if roof["bound"] == "tensor" and rate != 1.0 else "")
 
     F, B, F_eff = layer_work(cfg, stats, T)
     t_f, t_b = F_eff / (peaks["bf16_tflops"] * 1e12), B / (peaks["hbm_gbs"] * 1e9)
@@ -642,7 +656,9 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling runs)")
     ap.add_argument("--impl", default="lmoe", choices=["lmoe", "reference"])
-    ap.add_argument("--no-secondary", action="store_true", help="skip the prefill side measurement")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the other workloads' measurements")
+    ap.add_argument("--secondary", default=",".join(SECONDARY_WORKLOADS),
+                    help="comma-separated workloads measured beside the main one (reported under `secondary`)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
     args = ap.parse_args()
@@ -675,14 +691,20 @@ def main():
         else:
             res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks)
         secondary = None
-        if not args.ep and not args.no_secondary and args.workload != SECONDARY_WORKLOAD:
-            sc = synth.WORKLOADS[SECONDARY_WORKLOAD]
-            s_steps = max(3, min(args.steps, 20))
-            r2 = run_gpu(sc, s_steps, args.warmup, rank, world, local, peaks, with_e2e=False, with_clocks=False)
-            secondary = {"workload": sc.name, "tokens_per_s": world * sc.tokens * s_steps / (r2["ms"] / 1e3),
-                         "ms_per_step": r2["ms"] / s_steps, "roofline": r2["roofline"],
-                         "layer_roofline": r2["layer_roofline"],
-                         "phases_ms_per_step": {k: v[0] / s_steps for k, v in r2["phases"].items()}}
+        if not args.ep and not args.no_secondary:
+            secondary = []
+            for name in [w for w in args.secondary.split(",") if w and w != args.workload]:
+                sc = synth.WORKLOADS[name]
+                # at least 20 steps for every workload: decode batches take well under a millisecond each
+                s_steps = max(20, min(args.steps, 50)) if sc.tokens <= 32 else max(3, min(args.steps, 20))
+                r2 = run_gpu(sc, s_steps, args.warmup, rank, world, local, peaks, with_e2e=False)
+                secondary.append({"workload": sc.name, "config": workload_config(sc), "dtype": compute_dtype(sc),
+                                  "steps": s_steps,
+                                  "tokens_per_s": world * sc.tokens * s_steps / (r2["ms"] / 1e3),
+                                  "ms_per_step": r2["ms"] / s_steps, "roofline": r2["roofline"],
+                                  "layer_roofline": r2["layer_roofline"], "clocks": r2["clocks"],
+                                  "phases_ms_per_step": {k: v[0] / s_steps for k, v in r2["phases"].items()},
+                                  "gpu_launches": r2["launches"], "routing": r2["stats"]})
     finally:
         pass
     if rank == 0:

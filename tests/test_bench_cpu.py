@@ -37,3 +37,39 @@ def test_decode_is_hbm_bound_and_prefill_tensor_bound():
         F, B, F_eff = bench.layer_work(cfg, {"ffn_rows": rows, "experts_touched": touched}, cfg.tokens)
         t_f, t_b = F_eff / 1646e12, B / 6540e9
         assert (t_b > t_f) == name.endswith("decode"), name
+
+
+def test_grouped_expert_gemm_roofline_is_tensor_framed():
+    """A prefill grouped GEMM's bytes are its touched experts' weights (the gathered and hidden rows are
+    intermediates), so it is tensor-bound: 377.96 GFLOP in 0.3843 ms is 0.598 of a 1645.9 TFLOP/s peak."""
+    cfg = synth.WORKLOADS["nemotron_prefill"]
+    stats = {"ffn_rows": 8192 * 22, "experts_touched": 512, "tc_rows": 8192 * 22, "tc_experts": 512,
+             "stream_rows": 0, "stream_experts": 0}
+    peaks = {"hbm_gbs": 6540.2, "bf16_tflops": 1645.9, "source": "measured"}
+    phases = {"expert_up_gemm": (0.3843, 1), "expert_down_gemm": (0.3809, 1), "combine": (0.07, 1)}
+    roof, layer, launches = bench.rooflines(cfg, stats, cfg.tokens, phases, peaks, 1.09)
+    assert roof["kernel"] == "expert_up_gemm" and roof["bound"] == "tensor"
+    assert roof["algorithmic_per_launch"]["bytes"] == 2 * 1024 * 1024 * 512  # W1: bf16 m x latent per expert
+    assert roof["frac"] == pytest.approx(377.96e9 / 0.3843e-3 / 1645.9e12, rel=1e-3)
+    assert launches == 3
+
+
+def test_decode_weight_stream_roofline_is_hbm_framed():
+    """A decode weight stream's bytes are the touched experts' weights: 380 experts x 2 MiB in 0.1246 ms."""
+    cfg = synth.WORKLOADS["nemotron_decode"]
+    stats = {"ffn_rows": 704, "experts_touched": 380, "tc_rows": 0, "tc_experts": 0, "stream_rows": 704,
+             "stream_experts": 380}
+    peaks = {"hbm_gbs": 6540.2, "bf16_tflops": 1645.9, "source": "measured"}
+    roof, _, _ = bench.rooflines(cfg, stats, 32, {"expert_up_stream": (0.1246, 1)}, peaks, 0.286)
+    assert roof["bound"] == "hbm"
+    assert roof["achieved"] == pytest.approx(380 * 2 * 1024 * 1024 / 0.1246e-3 / 1e9, rel=1e-9)
+
+
+def test_block_scaled_expert_gemm_takes_its_own_dtype_peak():
+    """An NVFP4 expert contraction that is compute-bound is framed against 4x the bf16 peak (fp4 : bf16)."""
+    cfg = synth.WORKLOADS["nemotron_decode_nvfp4"].with_(tokens=8192, name="nvfp4_big")
+    stats = {"ffn_rows": 8192 * 22, "experts_touched": 512, "tc_rows": 0, "tc_experts": 0,
+             "stream_rows": 8192 * 22, "stream_experts": 512}
+    peaks = {"hbm_gbs": 6540.2, "bf16_tflops": 1645.9, "source": "measured"}
+    roof, _, _ = bench.rooflines(cfg, stats, cfg.tokens, {"expert_up_stream": (0.2, 1)}, peaks, 1.0)
+    assert roof["bound"] == "tensor" and roof["peak"] == pytest.approx(4 * 1645.9)
