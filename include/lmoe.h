@@ -70,7 +70,7 @@ extern "C" {
 #define LMOE_ERR_TOO_MANY_TOKENS (-3)   /* T > max_tokens, or T < 0 */
 #define LMOE_ERR_CUDA (-4)              /* a CUDA runtime / driver call failed */
 #define LMOE_ERR_TIMEOUT (-5)           /* device: a bounded wait inside a kernel gave up */
-#define LMOE_ERR_BAD_INDEX (-6)         /* device: an expert id outside [0, n_total) */
+#define LMOE_ERR_BAD_INDEX (-6)         /* device: an expert id outside [0, n_total), or twice in one row */
 #define LMOE_ERR_WORKSPACE (-7)         /* workspace missing or smaller than lmoe_workspace_bytes */
 #define LMOE_ERR_BAD_COUNTS (-8)        /* device: received row counts of lmoe_ep_experts inconsistent */
 
@@ -184,8 +184,13 @@ LMOE_API int lmoe_create(const lmoe_config *cfg, const lmoe_weights *w, void *wo
  * By default, for a layer without a shared expert, the forward's launches
  * reach the GPU as one CUDA graph: they are captured on a stream of the
  * handle's own, and the handle's executable graph for that launch sequence is
- * updated and launched on `stream` (see lmoe_set_graph_launch).  No device memory is allocated and the
- * host does not wait on the device.  With a shared expert (two streams), while
+ * updated and launched on `stream` (see lmoe_set_graph_launch).  The library
+ * allocates no device memory and the host does not wait on the device.  The
+ * executable graph is a driver object: its first instantiation (the first
+ * graph-launched forward of a handle, or the first after a change of launch
+ * sequence) left the free device memory that cudaMemGetInfo reports
+ * unchanged on B200, for a decode-size and a prefill-path layer (measured to
+ * its 2 MiB granularity), and replays of a kept graph take none.  With a shared expert (two streams), while
  * `stream` is itself being captured, with phase timing on, or with `dbg` set,
  * the launches go onto `stream` one by one; the results are the same bits.
  */
@@ -299,26 +304,41 @@ LMOE_API int lmoe_gemm_bf16(const void *A, const void *B, void *C, int32_t M, in
  * the process exits.  It allocates nothing (no cudaMalloc, no cudaFree, no
  * allocating library call).
  *
- *   idx      device int32 [T, top_k]: expert ids in [0, n_total) (out-of-range
- *            ids are skipped and their slots left unset)
+ *   idx      device int32 [T, top_k]: expert ids in [0, n_total); the ids of
+ *            one row (one token) must be distinct, as a top-K' selection's are
  *   counts   device int32 [n_total]: rows per expert
  *   offsets  device int32 [n_total + 1]: exclusive scan of counts
  *   perm     device int32 [T * top_k]: the slot index t*top_k+k at each sorted
  *            position
  *   inv      device int32 [T * top_k]: the sorted position of each slot
+ *   err_word optional device int32 (NULL: not reported).  The call writes its
+ *            device error bits there, 0 when the ids were valid:
+ *              LMOE_DEVERR_BAD_INDEX       an id outside [0, n_total) was
+ *                                          skipped: its slot's inv entry is not
+ *                                          written, counts leave it out, and
+ *                                          perm is filled only up to
+ *                                          offsets[n_total] < T * top_k;
+ *              LMOE_DEVERR_REPEATED_INDEX  a row named one expert twice: counts,
+ *                                          perm and inv are then not a valid
+ *                                          sort (every write still stays inside
+ *                                          the buffers above).
  *
  * Limits: 0 <= T <= 8192 (else LMOE_ERR_TOO_MANY_TOKENS); 1 <= top_k <= 32,
  * top_k <= n_total <= 1024 (else LMOE_ERR_UNSUPPORTED_SHAPE).  A rejected call
- * enqueues no work.
- * The first call on a device looks up the device address of the scratch array
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  Every call on a device shares the one scratch array, so
+ * enqueues no work.  T = 0 zeroes counts, offsets and *err_word.
+ * The scratch array's device address is looked up (cudaGetSymbolAddress) by
+ * the first call on a device, with that device current, and again whenever the
+ * current context of that device has changed since (after cudaDeviceReset, for
+ * instance); make that first call before any stream capture.  Every call on a
+ * device shares the one scratch array, which keeps the last call's contents, so
  * calls whose work overlaps on the GPU (different streams, no ordering between
  * them) race and corrupt each other's results; order them on one stream.
  * Asynchronous on `stream`.
  */
+#define LMOE_DEVERR_BAD_INDEX 2
+#define LMOE_DEVERR_REPEATED_INDEX 8
 LMOE_API int lmoe_dispatch_noalloc(const int32_t *idx, int32_t T, int32_t top_k, int32_t n_total, int32_t *counts,
-                                   int32_t *offsets, int32_t *perm, int32_t *inv, void *stream);
+                                   int32_t *offsets, int32_t *perm, int32_t *inv, int32_t *err_word, void *stream);
 
 /*
  * Block-scaled (MX) encoding of a bf16 weight matrix, for lmoe_weights.w1 /

@@ -9,6 +9,8 @@ holds at replay time.  The cases cover the decode paths (split-K projections,
 weight streaming, NVFP4 experts), the prefill paths (tensor-core GEMMs) and the
 shared expert on its own stream.
 """
+import warnings
+
 import pytest
 import torch
 
@@ -107,5 +109,41 @@ def test_graph_launch_switch_rejects_bad_values():
         assert lmoe.lib().lmoe_set_graph_launch(mod.h, 2) == -1
         lmoe.lmoe_set_graph_launch(mod.h, False)
         lmoe.lmoe_set_graph_launch(mod.h, True)
+    finally:
+        mod.close()
+
+
+@pytest.mark.parametrize("name", ["nemotron_decode", "medium_prefill_path"])
+def test_graph_launch_device_memory(name):
+    """How much device memory the library's graph launch takes: the free memory the driver reports
+    (cudaMemGetInfo) before and after the first graph-launched forward of a handle, after a direct-launch
+    forward has loaded every kernel's module, with no other allocation in between.  Replays of the kept
+    executable graph must take nothing more."""
+    cfg = CASES["nemotron_decode"] if name == "nemotron_decode" else MEDIUM.with_(tokens=300, seed=124)
+    layer = synth.make_layer(cfg)
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=cfg.tokens)
+    try:
+        x = layer["x"].cuda()
+        y = torch.empty_like(x)
+        lmoe.lmoe_set_graph_launch(mod.h, False)
+        mod.forward(x, y)          # direct launches: loads the modules of every kernel the forward uses
+        ref = y.clone()
+        torch.cuda.synchronize()
+        lmoe.lmoe_set_graph_launch(mod.h, True)
+        free0, _ = torch.cuda.mem_get_info()
+        mod.forward(x, y)          # captures, instantiates and launches the handle's first executable graph
+        torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info()
+        for _ in range(5):
+            mod.forward(x, y)      # updates the kept graph in place and launches it
+        torch.cuda.synchronize()
+        free2, _ = torch.cuda.mem_get_info()
+        assert torch.equal(y, ref)
+        assert mod.last_error() == 0
+        took = free0 - free1
+        warnings.warn(f"graph launch, {name}: first graph-launched forward took {took} bytes of device memory "
+                      f"(free {free0} -> {free1}); five more forwards took {free1 - free2}")
+        assert free2 == free1, "replays of the kept executable graph took device memory"
+        assert took <= 32 << 20, f"graph instantiation took {took} bytes"
     finally:
         mod.close()
