@@ -275,9 +275,9 @@ def phase_units(cfg, stats, T, phase):
         return 2.0 * rows_st * m * fin, wb * fin * m * e_st
     if phase == "router_proj_gemm":
         n_out = (L if cfg.has_proj else 0) + nt
-        return 2.0 * T * d * n_out, 2.0 * (n_out * d + T * d) + T * (L * 2 if cfg.has_proj else 0) + 4.0 * T * nt
-    if phase == "up_proj_gemm":
-        return 2.0 * T * L * d, 2.0 * (d * L + T * L + 2 * T * d)
+        return 2.0 * T * d * n_out, 2.0 * (n_out * d + T * d)
+    if phase == "up_proj_gemm":  # W_up and the residual x in, y out
+        return 2.0 * T * L * d, 2.0 * (d * L + 2 * T * d)
     if phase == "shared_expert":
         ms = getattr(cfg, "shared_m", 0)
         return 2.0 * T * (g + 1) * d * ms, 2.0 * ((g + 1) * d * ms + T * (d + ms) + T * (ms + 2 * d))

@@ -267,6 +267,21 @@ LMOE_API int lmoe_set_small_rows(lmoe_handle *h, int32_t rows);
  */
 LMOE_API int lmoe_set_graph_launch(lmoe_handle *h, int enable);
 
+/*
+ * Kernel of the grouped (tensor-core) expert GEMMs, for the experts that get
+ * more rows than the weight-streaming threshold.  kind = 0 (default):
+ * single-CTA 128 x 256 tiles over 128-row slices of each expert's rows.
+ * kind = 1: CTA pairs computing each expert's GEMM transposed, weight rows as
+ * the 256-row operand split over the pair and the expert's token rows as
+ * N <= 256 (taken when latent is a multiple of 256 and m of 256, or of 128
+ * with SwiGLU, for bf16 experts; other shapes keep kind 0).  Kind 1 moves a
+ * quarter fewer operand bytes from L2 and was faster on the Kimi-like skewed
+ * layer, kind 0 on the Nemotron-like one (about 350 rows per expert); both
+ * are deterministic and agree with each other to rounding.
+ * Errors: LMOE_ERR_INVALID_ARG for a NULL handle or kind not 0 or 1.
+ */
+LMOE_API int lmoe_set_grouped_gemm(lmoe_handle *h, int kind);
+
 /* Bound of every in-kernel wait, nanoseconds (default 1e9). */
 LMOE_API int lmoe_set_wait_timeout(lmoe_handle *h, uint64_t ns);
 

@@ -26,6 +26,7 @@ static __global__ void __launch_bounds__(1024) ep_prep_kernel(const int32_t* __r
                                                               int n_local, int n_recv, int rows_bound, int small_max,
                                                               int* __restrict__ counts, int* __restrict__ offsets,
                                                               int4* __restrict__ mt_list, int4* __restrict__ small_list,
+                                                              int4* __restrict__ pt_list,
                                                               int* __restrict__ src_off, int* __restrict__ dst_base,
                                                               int* __restrict__ hdr) {
     pdl_begin();
@@ -61,7 +62,8 @@ static __global__ void __launch_bounds__(1024) ep_prep_kernel(const int32_t* __r
     }
     const int c = static_cast<int>(c64);
     if (j < n_local) counts[j] = c;
-    const int off = offsets_and_tiles(c, n_local, n_local, small_max, offsets, mt_list, small_list, hdr, scratch);
+    const int off =
+        offsets_and_tiles(c, n_local, n_local, small_max, offsets, mt_list, small_list, pt_list, hdr, scratch);
     s_off[j] = off;
     int total;
     const int so = block_exclusive_scan(cj, scratch, &total);  // synchronises: s_off and s_cnt are visible

@@ -29,6 +29,7 @@
 #include "nv.cuh"
 #include "ep.cuh"
 #include "tc_gemm.cuh"
+#include "tc_group.cuh"
 #include "tc_swap.cuh"
 
 using namespace lmoe;
@@ -59,6 +60,36 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, ui
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
                                 estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// bf16 matrix [rows, cols] (row pitch `ld` elements) with an unswizzled box of box_rows x box_cols: the output
+// blocks the transposed grouped GEMM stages in shared memory row-major.
+bool make_map_plain(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld, uint32_t box_cols,
+                    uint32_t box_rows) {
+    if (!load_encode() || rows == 0) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {ld * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+                                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Gated expert weights W1 [n_experts][2m][K] bf16 (gate rows, then up rows) as a 5-D tensor
+// (K, 16 rows, {gate, up}, m / 16 groups, expert), 128-byte swizzle.  A box of 64 x 16 x 2 x 4 x 1 lands
+// as 16 gate rows, their 16 up rows, the next 16 gate rows, ...: 128 rows of 128 bytes.
+bool make_map_gated(CUtensorMap* map, const void* base, uint64_t n_experts, uint64_t m, uint64_t K) {
+    if (!load_encode() || n_experts == 0 || m % 16 != 0) return false;
+    cuuint64_t dims[5] = {K, 16, 2, m / 16, n_experts};
+    cuuint64_t strides[4] = {K * 2, m * K * 2, 16 * K * 2, 2 * m * K * 2};
+    cuuint32_t box[5] = {64, 16, 2, 4, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides,
+                                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -155,7 +186,8 @@ int ep_ranks(const lmoe_config& c) { return c.ep_size > 1 ? c.ep_size : 1; }
 int n_local_experts(const lmoe_config& c) { return c.n_experts / ep_ranks(c); }
 
 struct Plan {
-    size_t hdr, logits, z, zlo, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, small_list, rows, hbuf, yl,
+    size_t hdr, logits, z, zlo, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, pt_list, small_list, rows,
+        hbuf, yl,
         partial, hs, s2, partial2, rows4, rows_sf4, h4, h_sf4, rows8, rows_sf, h8, h_sf, xin, yout, ep_map, ep_src,
         ep_dst, ep_counts,
         ep_offsets, total;
@@ -196,6 +228,7 @@ Plan make_plan(const lmoe_config& c) {
     p.perm = take(R * 4);
     p.inv = take(R * 4);
     p.mt_list = take(static_cast<size_t>(p.mt_max) * 16);
+    p.pt_list = take(((RC + 255) / 256 + c.n_experts) * 16);  // CTA-pair tiles: entries of up to 256 rows
     // weight-streaming list: one entry per expert, or (block-scaled experts) one per 32 rows of an expert
     p.small_list = take((static_cast<size_t>(c.n_experts) + RC / SMALL_MAX + 1) * 16);
     p.rows = take(RC * L * 2);  // gathered expert inputs, then (reused) expert outputs
@@ -243,6 +276,12 @@ enum Phase : int { PH_ROUTER = 0, PH_TOPK, PH_DISPATCH, PH_UP_TC, PH_UP_STREAM, 
 const char* kPhaseNames[PH_COUNT] = {"router_proj_gemm", "topk_softmax", "dispatch", "expert_up_gemm",
                                      "expert_up_stream", "expert_down_gemm", "expert_down_stream", "combine",
                                      "up_proj_gemm", "shared_expert", "ep_regroup"};
+
+template <int EPI>
+bool set_group_attr() {
+    return cudaFuncSetAttribute(tc_group_pair_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GroupCfg::SMEM_BYTES) == cudaSuccess;
+}
 
 template <int EPI>
 bool set_pair_attr() {
@@ -320,6 +359,9 @@ bool set_all_smem_attrs() {
     ok &= set_nv_attr<EPI_RELU2, true>();
     ok &= set_nv_attr<EPI_SWIGLU, true>();
     ok &= set_nv_attr<EPI_BF16, false>();
+    ok &= set_group_attr<EPI_BF16>();
+    ok &= set_group_attr<EPI_RELU2>();
+    ok &= set_group_attr<EPI_SWIGLU>();
     ok &= set_pair_attr<EPI_BF16>();
     ok &= set_pair_attr<EPI_RELU2>();
     ok &= set_pair_attr<EPI_SWIGLU>();
@@ -500,6 +542,15 @@ void launch_gemm_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensor
                  out != nullptr ? *out : a, a2 != nullptr ? *a2 : a, g);
 }
 
+// Grouped expert GEMM on CTA pairs (computed transposed): one pair per two SMs, persistent.
+// x32 / x64 / x128: the token rows (K-major, 128-byte swizzle) in boxes of 32, 64 and 128 rows.
+template <int EPI>
+void launch_group(const CUtensorMap& w, const CUtensorMap& x32, const CUtensorMap& x64, const CUtensorMap& x128,
+                  const CUtensorMap& out, const GroupArgs& a, int num_sms, cudaStream_t s) {
+    launch_pairs(tc_group_pair_kernel<EPI>, 2 * (num_sms / 2), GroupCfg::THREADS, GroupCfg::SMEM_BYTES, s, w, x32, x64,
+                 x128, out, a);
+}
+
 template <int EPI, bool W4, bool QOUT>
 void launch_mx(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf, const MxArgs& a, int grid,
                cudaStream_t s) {
@@ -571,6 +622,11 @@ struct lmoe_handle {
     CUtensorMap w1n{}, w2n{}, rows4{}, rows_sf4{}, h4{}, h_sf4{};
     // TMA store maps of bf16 GEMM outputs (32-row x 64-column boxes): hidden rows, expert outputs, z
     CUtensorMap o_h{}, o_rows{}, o_z{};
+    // grouped expert GEMMs on CTA pairs (transposed): gated W1 as 16-row gate / up groups, unswizzled output blocks of
+    // 32 rows x 32 (x 16 for gated) columns of the hidden rows and of the expert outputs
+    CUtensorMap w1g16{}, og_h{}, og_rows{}, rows64{}, h64{};
+    bool group_pair_ok = false;  // the shapes allow it: m (gated: m / 2 per pair tile) and latent in 256-row tiles
+    int group_pair = 0;          // 1: grouped expert GEMMs on CTA pairs; 0 (default): single-CTA 128-row tiles
     cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
     // Forwards launched as a CUDA graph: each call captures its launches on `cap` and replays them on the
     // caller's stream from an executable graph, updated in place.  A few executable graphs are kept, one per
@@ -834,7 +890,7 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
         PhaseScope ps(h, PH_DISPATCH, s, 2);
         const size_t sm = (static_cast<size_t>(2 * nwords) * nt + nt) * 4;
         launch(dispatch_small_kernel, 1, 1024, sm, s, idx, T, K, nt, c.n_experts, small, counts, offsets, mt_list,
-               small_list, perm, inv, hdr);
+               small_list, h->at<int4>(p.pt_list), perm, inv, hdr);
         if (c.expert_fmt == LMOE_FMT_NVFP4)
             launch(nv_gather_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, inv, T, K, c.n_experts,
                    feat, L, L, h->at<uint8_t>(p.rows4), h->at<uint8_t>(p.rows_sf4), static_cast<int>(c.max_tokens) * K);
@@ -850,7 +906,8 @@ int run_front(lmoe_handle* h, const void* x, int T, cudaStream_t s, __nv_bfloat1
         uint32_t* prefix = h->at<uint32_t>(p.prefix);
         launch(dispatch_bitmap_kernel, (nwords + 7) / 8, 256, 8 * nt * 4, s, idx, T, K, nt, bitmap, hdr);
         launch(dispatch_expert_scan_kernel, (nt + 7) / 8, 256, 0, s, bitmap, T, nt, prefix, counts);
-        launch(dispatch_offsets_kernel, 1, 1024, 0, s, counts, nt, c.n_experts, small, offsets, mt_list, small_list, hdr);
+        launch(dispatch_offsets_kernel, 1, 1024, 0, s, counts, nt, c.n_experts, small, offsets, mt_list, small_list,
+               h->at<int4>(p.pt_list), hdr);
         // block-scaled experts: the scatter only places the slots (no bf16 row copy); the gather encodes the rows
         launch(dispatch_scatter_kernel, static_cast<unsigned>((slots + 7) / 8), 256, 0, s, idx, T, K, nt, c.n_experts,
                bitmap, prefix, offsets, feat, L, mx ? 0 : L, rows_dst, L, perm, inv);
@@ -882,11 +939,29 @@ int run_experts(lmoe_handle* h, int small, bool need_tc, cudaStream_t s) {
     base.err = hdr + HDR_ERR;
     base.timeout_ns = h->timeout_ns;
 
+    const bool pair = need_tc && h->group_pair && h->group_pair_ok;
+    GroupArgs ga{};
+    ga.list = h->at<int4>(p.pt_list);
+    ga.count = hdr + HDR_PT;
+    ga.err = hdr + HDR_ERR;
+    ga.timeout_ns = h->timeout_ns;
     // ---------------------------------------------------------------- expert up (+ activation)
-    if (need_tc) {
-        // Grouped GEMMs stay on single-CTA 128-row tiles: with a few hundred rows per expert, 256-row pair
-        // tiles would need a second launch for each expert's remainder, which reads the expert's weights
-        // from HBM a second time.
+    if (pair) {
+        // CTA pairs, weight rows as the 256-row operand: each expert's rows in N <= 256 token tiles
+        PhaseScope ps(h, PH_UP_TC, s, 1);
+        GroupArgs a = ga;
+        a.K = L;
+        a.n_mt = c.act == LMOE_ACT_SWIGLU ? m / 128 : m / 256;
+        a.w_rows_per_expert = h->g * m;
+        a.up_offset = m;
+        a.out = hbuf;
+        a.ld_out = m;
+        if (c.act == LMOE_ACT_SWIGLU)
+            launch_group<EPI_SWIGLU>(h->w1g16, h->rows32, h->rows64, h->a_rows, h->og_h, a, h->num_sms, s);
+        else if (c.act == LMOE_ACT_RELU2)
+            launch_group<EPI_RELU2>(h->w1s, h->rows32, h->rows64, h->a_rows, h->og_h, a, h->num_sms, s);
+        else launch_group<EPI_BF16>(h->w1s, h->rows32, h->rows64, h->a_rows, h->og_h, a, h->num_sms, s);
+    } else if (need_tc) {
         PhaseScope ps(h, PH_UP_TC, s, 1);
         GemmArgs a = base;
         a.K = L;
@@ -965,7 +1040,16 @@ int run_experts(lmoe_handle* h, int small, bool need_tc, cudaStream_t s) {
         launch_stream(small, epi, h->w1s, h->rows16, h->rows32, a, h->num_sms, s);
     }
     // ---------------------------------------------------------------- expert down (output reuses the gathered rows)
-    if (need_tc) {
+    if (pair) {
+        PhaseScope ps(h, PH_DOWN_TC, s, 1);
+        GroupArgs a = ga;
+        a.K = m;
+        a.n_mt = L / 256;
+        a.w_rows_per_expert = L;
+        a.out = rows;
+        a.ld_out = L;
+        launch_group<EPI_BF16>(h->w2s, h->h32, h->h64, h->a_h, h->og_rows, a, h->num_sms, s);
+    } else if (need_tc) {
         PhaseScope ps(h, PH_DOWN_TC, s, 1);
         GemmArgs a = base;
         a.K = m;
@@ -1348,6 +1432,14 @@ int lmoe_create(const lmoe_config* cfg, const lmoe_weights* w, void* workspace, 
     ok &= make_map(&h->a_h, h->at<void>(p.hbuf), RC, m, m, 128);
     ok &= make_map(&h->o_h, h->at<void>(p.hbuf), RC, m, m, 32);
     ok &= make_map(&h->o_rows, h->at<void>(p.rows), RC, L, L, 32);
+    h->group_pair_ok = c.expert_fmt == LMOE_FMT_BF16 && L % 256 == 0 && m % (h->g == 2 ? 128 : 256) == 0;
+    if (h->group_pair_ok) {
+        if (h->g == 2) ok &= make_map_gated(&h->w1g16, w->w1, h->n_local, m, L);
+        ok &= make_map_plain(&h->og_h, h->at<void>(p.hbuf), RC, m, m, h->g == 2 ? 16 : 32, 32);
+        ok &= make_map_plain(&h->og_rows, h->at<void>(p.rows), RC, L, L, 32, 32);
+        ok &= make_map(&h->rows64, h->at<void>(p.rows), RC, L, L, 64);
+        ok &= make_map(&h->h64, h->at<void>(p.hbuf), RC, m, m, 64);
+    }
     if (c.has_proj) ok &= make_map(&h->o_z, h->at<void>(p.z), c.max_tokens, L, L, 32);
     ok &= make_map(&h->rows16, h->at<void>(p.rows), RC, L, L, 16);
     ok &= make_map(&h->rows32, h->at<void>(p.rows), RC, L, L, 32);
@@ -1469,7 +1561,7 @@ int lmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const int32_t* recv_c
         PhaseScope ps(h, PH_EP_REGROUP, s, 2);
         launch(ep_prep_kernel, 1, 1024, 0, s, recv_counts, ep, nl, static_cast<int>(n_recv),
                static_cast<int>(rows_bound), small, h->at<int>(p.ep_counts), h->at<int>(p.ep_offsets),
-               h->at<int4>(p.mt_list), h->at<int4>(p.small_list), src_off, dst_base, hdr);
+               h->at<int4>(p.mt_list), h->at<int4>(p.small_list), h->at<int4>(p.pt_list), src_off, dst_base, hdr);
         launch(ep_regroup_kernel, grid, 32 * EP_ROWS_PER_PASS, static_cast<size_t>(2 * n_seg + 1) * 4, s,
                static_cast<const __nv_bfloat16*>(recv_rows), static_cast<int>(n_recv), L,
                static_cast<const int*>(src_off), static_cast<const int*>(dst_base), n_seg,
@@ -1630,6 +1722,12 @@ int lmoe_set_small_rows(lmoe_handle* h, int32_t rows) {
 int lmoe_set_graph_launch(lmoe_handle* h, int enable) {
     if (h == nullptr || (enable != 0 && enable != 1)) return LMOE_ERR_INVALID_ARG;
     h->use_graph = enable;
+    return LMOE_OK;
+}
+
+int lmoe_set_grouped_gemm(lmoe_handle* h, int kind) {
+    if (h == nullptr || (kind != 0 && kind != 1)) return LMOE_ERR_INVALID_ARG;
+    h->group_pair = kind;
     return LMOE_OK;
 }
 

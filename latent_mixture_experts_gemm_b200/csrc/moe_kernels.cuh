@@ -18,6 +18,7 @@ enum : int {
     HDR_MT = 2,         // entries of the tensor-core M-tile list
     HDR_NSMALL = 3,     // entries of the weight-streaming list
     HDR_EP_BAD = 4,     // 1: the received counts of the expert-parallel experts stage were rejected
+    HDR_PT = 5,         // entries of the CTA-pair tile list (the same experts as the M-tile list, 256-row entries)
     HDR_WORDS = 16,
 };
 
@@ -356,7 +357,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* scratch, int* to
 }
 
 // Offsets (exclusive scan of counts), the tensor-core M-tile list (experts
-// with more than `small_max` rows, split in 128-row tiles) and the
+// with more than `small_max` rows, split in 128-row tiles), the CTA-pair tile
+// list (the same experts in entries of up to 256 rows) and the
 // weight-streaming list (experts with 1..small_max rows).  A negative
 // small_max selects chunk mode instead (block-scaled experts, which only
 // stream): every FFN expert with rows enters the weight-streaming list as
@@ -375,21 +377,30 @@ __device__ __forceinline__ void write_stream_entries(int4* __restrict__ small_li
     const int chunk = small_max < 0 ? -small_max : c;
     for (int i = 0; i < n; ++i) small_list[pos + i] = make_int4(e, off + chunk * i, min(chunk, c - chunk * i), 0);
 }
+// CTA-pair list entries of expert e (c rows from sorted row off): 256 rows each, the rest last.
+__device__ __forceinline__ void write_pair_entries(int4* __restrict__ pt_list, int pos, int n, int e, int off, int c) {
+    for (int i = 0; i < n; ++i) pt_list[pos + i] = make_int4(e, off + 256 * i, min(256, c - 256 * i), 0);
+}
+
 __device__ __forceinline__ int offsets_and_tiles(int c, int n_tot, int n_ffn, int small_max, int* __restrict__ offsets,
                                                  int4* __restrict__ mt_list, int4* __restrict__ small_list,
-                                                 int* __restrict__ hdr, int* scratch) {
+                                                 int4* __restrict__ pt_list, int* __restrict__ hdr, int* scratch) {
     const int e = threadIdx.x;
     int total;
     const int off = block_exclusive_scan(c, scratch, &total);
     if (e < n_tot) offsets[e] = off;
     if (e == 0) offsets[n_tot] = total;
     const bool ffn = e < n_ffn;
-    const int ntile = (ffn && small_max >= 0 && c > small_max) ? (c + 127) / 128 : 0;
+    const bool tc = ffn && small_max >= 0 && c > small_max;
+    const int ntile = tc ? (c + 127) / 128 : 0;
+    const int ptile = tc ? (c + 255) / 256 : 0;
     const int small = stream_entries(ffn, c, small_max);
-    int mt_total, small_total;
+    int mt_total, small_total, pt_total;
     const int mt_pos = block_exclusive_scan(ntile, scratch, &mt_total);
     const int sm_pos = block_exclusive_scan(small, scratch, &small_total);
+    const int pt_pos = block_exclusive_scan(ptile, scratch, &pt_total);
     for (int i = 0; i < ntile; ++i) mt_list[mt_pos + i] = make_int4(e, off + 128 * i, min(128, c - 128 * i), 0);
+    write_pair_entries(pt_list, pt_pos, ptile, e, off, c);
     write_stream_entries(small_list, sm_pos, small, e, off, c, small_max);
     // R = rows of FFN experts = offsets[n_ffn] (FFN ids come first)
     const int ffn_rows_part = ffn ? c : 0;
@@ -399,6 +410,7 @@ __device__ __forceinline__ int offsets_and_tiles(int c, int n_tot, int n_ffn, in
         hdr[HDR_ROWS] = rows_total;
         hdr[HDR_MT] = mt_total;
         hdr[HDR_NSMALL] = small_total;
+        hdr[HDR_PT] = pt_total;
     }
     return off;
 }
@@ -407,11 +419,12 @@ __device__ __forceinline__ int offsets_and_tiles(int c, int n_tot, int n_ffn, in
 static __global__ void __launch_bounds__(1024) dispatch_offsets_kernel(const int* __restrict__ counts, int n_tot, int n_ffn,
                                                                 int small_max, int* __restrict__ offsets,
                                                                 int4* __restrict__ mt_list, int4* __restrict__ small_list,
-                                                                int* __restrict__ hdr) {
+                                                                int4* __restrict__ pt_list, int* __restrict__ hdr) {
     pdl_begin();
     __shared__ int scratch[33];
     const int e = threadIdx.x;
-    offsets_and_tiles(e < n_tot ? counts[e] : 0, n_tot, n_ffn, small_max, offsets, mt_list, small_list, hdr, scratch);
+    offsets_and_tiles(e < n_tot ? counts[e] : 0, n_tot, n_ffn, small_max, offsets, mt_list, small_list, pt_list, hdr,
+                      scratch);
 }
 
 // Small batches (T <= 256): bitmap, per-expert prefix, offsets, tile lists and
@@ -425,9 +438,9 @@ constexpr int SMALL_BATCH_WORDS = 8;
 __device__ __forceinline__ void dispatch_small_body(const int32_t* __restrict__ idx, int T, int K, int n_tot,
                                                     int n_ffn, int small_max, int* __restrict__ counts,
                                                     int* __restrict__ offsets, int4* __restrict__ mt_list,
-                                                    int4* __restrict__ small_list, int32_t* __restrict__ perm,
-                                                    int32_t* __restrict__ inv, int* __restrict__ hdr, uint32_t* sm,
-                                                    int* scratch) {
+                                                    int4* __restrict__ small_list, int4* __restrict__ pt_list,
+                                                    int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                    int* __restrict__ hdr, uint32_t* sm, int* scratch) {
     const int nwords = (T + 31) >> 5;
     uint32_t* bits = sm;
     uint32_t* prefix = sm + nwords * n_tot;
@@ -462,18 +475,23 @@ __device__ __forceinline__ void dispatch_small_body(const int32_t* __restrict__ 
     }
     if (e == 0) offsets[n_tot] = total;
     const bool ffn = e < n_ffn;
-    const int ntile = (ffn && small_max >= 0 && c > small_max) ? (c + 127) / 128 : 0;
+    const bool tc = ffn && small_max >= 0 && c > small_max;
+    const int ntile = tc ? (c + 127) / 128 : 0;
+    const int ptile = tc ? (c + 255) / 256 : 0;
     const int small = stream_entries(ffn, c, small_max);
-    int mt_total, small_total, rows_total;
+    int mt_total, small_total, rows_total, pt_total;
     const int mt_pos = block_exclusive_scan(ntile, scratch, &mt_total);
     const int sm_pos = block_exclusive_scan(small, scratch, &small_total);
+    const int pt_pos = block_exclusive_scan(ptile, scratch, &pt_total);
     block_exclusive_scan(ffn ? c : 0, scratch, &rows_total);
     for (int i = 0; i < ntile; ++i) mt_list[mt_pos + i] = make_int4(e, off + 128 * i, min(128, c - 128 * i), 0);
+    write_pair_entries(pt_list, pt_pos, ptile, e, off, c);
     write_stream_entries(small_list, sm_pos, small, e, off, c, small_max);
     if (e == 0) {
         hdr[HDR_ROWS] = rows_total;
         hdr[HDR_MT] = mt_total;
         hdr[HDR_NSMALL] = small_total;
+        hdr[HDR_PT] = pt_total;
     }
     __syncthreads();  // base[] visible to every thread
     for (int i = threadIdx.x; i < slots; i += blockDim.x) {
@@ -490,13 +508,14 @@ __device__ __forceinline__ void dispatch_small_body(const int32_t* __restrict__ 
 static __global__ void __launch_bounds__(1024) dispatch_small_kernel(const int32_t* __restrict__ idx, int T, int K, int n_tot,
                                                               int n_ffn, int small_max, int* __restrict__ counts,
                                                               int* __restrict__ offsets, int4* __restrict__ mt_list,
-                                                              int4* __restrict__ small_list, int32_t* __restrict__ perm,
-                                                              int32_t* __restrict__ inv, int* __restrict__ hdr) {
+                                                              int4* __restrict__ small_list, int4* __restrict__ pt_list,
+                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                              int* __restrict__ hdr) {
     pdl_begin();
     extern __shared__ uint32_t sm[];
     __shared__ int scratch[33];
-    dispatch_small_body(idx, T, K, n_tot, n_ffn, small_max, counts, offsets, mt_list, small_list, perm, inv, hdr, sm,
-                        scratch);
+    dispatch_small_body(idx, T, K, n_tot, n_ffn, small_max, counts, offsets, mt_list, small_list, pt_list, perm, inv,
+                        hdr, sm, scratch);
 }
 
 // One warp per slot: copy the token's feature row to its sorted row (FFN experts only).

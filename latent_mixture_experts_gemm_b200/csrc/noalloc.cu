@@ -115,7 +115,7 @@ extern "C" int lmoe_dispatch_noalloc(const int32_t* idx, int32_t T, int32_t top_
     lmoe::dispatch_bitmap_kernel<<<(nwords + 7) / 8, 256, 8 * n_total * 4, s>>>(idx, T, top_k, n_total, bitmap, hdr);
     lmoe::dispatch_expert_scan_kernel<<<(n_total + 7) / 8, 256, 0, s>>>(bitmap, T, n_total, prefix, counts);
     // no FFN experts here: no tile lists, only offsets
-    lmoe::dispatch_offsets_kernel<<<1, 1024, 0, s>>>(counts, n_total, 0, 0, offsets, nullptr, nullptr, hdr);
+    lmoe::dispatch_offsets_kernel<<<1, 1024, 0, s>>>(counts, n_total, 0, 0, offsets, nullptr, nullptr, nullptr, hdr);
     lmoe::dispatch_scatter_kernel<<<static_cast<unsigned>((slots + 7) / 8), 256, 0, s>>>(
         idx, T, top_k, n_total, 0, bitmap, prefix, offsets, nullptr, 0, 0, nullptr, 0, perm, inv);
     // the caller's copy of this call's error bits (the scratch header is cleared by the next call)

@@ -328,6 +328,18 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
         : "memory");
 }
 
+// 5-D tiled load of the box at (c0 .. c4) (c0 innermost) into this CTA's shared memory, completion bytes
+// to an mbarrier given by its shared::cluster address (as tma_load_2d_pair).
+__device__ __forceinline__ void tma_load_5d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0, int c1,
+                                                 int c2, int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2),
+          "r"(c3), "r"(c4)
+        : "memory");
+}
+
 // Pair MMA: D[256 x N] (+)= A[256 x 16] B[N x 16]^T, A rows 0..127 and B rows 0..N/2-1 from the first
 // CTA's shared memory, the rest from the second CTA's at the same addresses; each CTA's tensor memory
 // receives its own 128 rows of D.  Issued by one thread of the first CTA.

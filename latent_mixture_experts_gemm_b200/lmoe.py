@@ -81,6 +81,7 @@ def lib() -> ctypes.CDLL:
         L.lmoe_set_small_rows.argtypes = [P, I32]
         L.lmoe_set_wait_timeout.argtypes = [P, ctypes.c_uint64]
         L.lmoe_set_graph_launch.argtypes = [P, ctypes.c_int]
+        L.lmoe_set_grouped_gemm.argtypes = [P, ctypes.c_int]
         L.lmoe_gemm_bf16.argtypes = [P, P, P, I32, I32, I32, P, P]
         L.lmoe_dispatch_noalloc.argtypes = [P, I32, I32, I32, P, P, P, P, P, P]
         L.lmoe_selftest_wait.argtypes = [P, ctypes.c_uint64, P]
@@ -185,6 +186,11 @@ def lmoe_set_wait_timeout(h: int, ns: int) -> None:
 def lmoe_set_graph_launch(h: int, enable: bool) -> None:
     """Launch each forward as one CUDA graph (default) or its kernels one by one."""
     _check("lmoe_set_graph_launch", lib().lmoe_set_graph_launch(h, 1 if enable else 0))
+
+
+def lmoe_set_grouped_gemm(h: int, kind: int) -> None:
+    """Grouped expert GEMM kernel: 1 (default) CTA pairs, transposed; 0 single-CTA 128-row tiles."""
+    _check("lmoe_set_grouped_gemm", lib().lmoe_set_grouped_gemm(h, int(kind)))
 
 
 def lmoe_selftest_wait(h: int, timeout_ns: int, stream=None) -> None:

@@ -88,6 +88,7 @@ def test_null_handle_calls_are_rejected():
     assert L.lmoe_set_graph_launch(None, 1) == -1
     assert lmoe.lmoe_num_phases() == 11
     assert lmoe.lmoe_phase_name(10) == "ep_regroup"
+    assert L.lmoe_set_grouped_gemm(None, 1) == -1
     assert [lmoe.lmoe_phase_name(i) for i in range(3)] == ["router_proj_gemm", "topk_softmax", "dispatch"]
 
 

@@ -19,6 +19,7 @@ from tests import _parity as P
 pytestmark = pytest.mark.gpu
 
 MEDIUM = synth.LayerConfig(name="medium", tokens=300, d=512, latent=128, m=256, n_ffn=64, top_k=6, seed=21)
+PAIR = synth.LayerConfig(name="pair", tokens=1500, d=512, latent=256, m=512, n_ffn=16, top_k=4, seed=50)
 
 CASES = {
     "tiny": synth.WORKLOADS["tiny"],
@@ -45,6 +46,16 @@ CASES = {
                                                            n_zero=1, seed=41),
     "nemotron_decode": synth.WORKLOADS["nemotron_decode"],
     "std_decode": synth.WORKLOADS["std_decode"],
+    # latent and m in 256-row weight tiles, so the grouped GEMMs can also run on CTA pairs (transposed; see
+    # test_pair_grouped_gemm_parity), with experts of a few to a few hundred rows (token tiles of 16..256
+    # rows, ragged ends)
+    "pair_relu2_375_rows": PAIR,
+    "pair_swiglu_bypass_skew": PAIR.with_(m=384, act="swiglu", n_zero=1, n_copy=1, n_const=1, zipf=1.1, tokens=900,
+                                          top_k=3, seed=51),
+    "pair_identity_standard_moe": PAIR.with_(latent=512, has_proj=0, m=256, act="identity", n_ffn=8, top_k=2,
+                                             tokens=700, seed=52),
+    "pair_20_rows_per_expert": PAIR.with_(n_ffn=64, top_k=6, tokens=213, seed=53),
+    "pair_latent_router_swiglu": PAIR.with_(m=256, act="swiglu", latent_router=1, tokens=611, seed=54),
 }
 
 # The layer configurations the contract names (tiny, the Nemotron-like decode and prefill batches, the
@@ -61,7 +72,7 @@ def _layer(name, cfg):
     return _layers[name]
 
 
-def _run_and_check(cfg, layer, small_rows=None, sample=None, label=None):
+def _run_and_check(cfg, layer, small_rows=None, sample=None, label=None, grouped_kind=None):
     """Forward through the C ABI and compare with the oracle.  ``label`` names the case: a name in
     CONTRACT is held to the plain tolerances; any other case may use the bf16-storage allowance, and a
     warning records each case that does, with both errors."""
@@ -71,6 +82,8 @@ def _run_and_check(cfg, layer, small_rows=None, sample=None, label=None):
     try:
         if small_rows is not None:
             lmoe.lmoe_set_small_rows(mod.h, small_rows)
+        if grouped_kind is not None:
+            lmoe.lmoe_set_grouped_gemm(mod.h, grouped_kind)
         x = layer["x"].cuda()
         y, dbg = mod.forward(x, debug=True)
         torch.cuda.synchronize()
@@ -129,6 +142,51 @@ def test_full_size_parity_on_sampled_tokens(name):
     sample = np.sort(rng.choice(cfg.tokens, size=48, replace=False))
     sample[-1] = cfg.tokens - 1  # include the ragged end of the last tile
     _run_and_check(cfg, layer, sample=sample, label=name)
+
+
+PAIR_CASES = [n for n in CASES if n.startswith("pair_")]
+
+
+@pytest.mark.parametrize("small_rows", [8, 0], ids=["mixed_paths", "tensor_core_only"])
+@pytest.mark.parametrize("name", PAIR_CASES)
+def test_pair_grouped_gemm_parity(name, small_rows):
+    """The grouped expert GEMMs on CTA pairs (kind 1) against the oracle."""
+    cfg = CASES[name]
+    _run_and_check(cfg, _layer(name, cfg), small_rows=small_rows, label=name, grouped_kind=1)
+
+
+def test_pair_grouped_gemm_parity_on_the_kimi_like_layer():
+    """Kind 1 on the full-size Kimi-like skewed layer (gated experts, hundreds to thousands of rows per hot
+    expert), compared on sampled tokens."""
+    cfg = synth.WORKLOADS["kimi_skew"]
+    layer = synth.make_layer(cfg)
+    rng = np.random.default_rng(4321)
+    sample = np.sort(rng.choice(cfg.tokens, size=32, replace=False))
+    _run_and_check(cfg, layer, sample=sample, label="kimi_skew", grouped_kind=1)
+
+
+@pytest.mark.parametrize("name", ["pair_relu2_375_rows", "pair_swiglu_bypass_skew", "pair_identity_standard_moe"])
+def test_grouped_gemm_kinds_agree(name):
+    """The CTA-pair (transposed) and the single-CTA grouped GEMMs: each meets the oracle, each is
+    deterministic, and they agree with each other to bf16 rounding of the expert outputs."""
+    cfg = CASES[name]
+    layer = _layer(name, cfg)
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=cfg.tokens)
+    try:
+        lmoe.lmoe_set_small_rows(mod.h, 0)
+        x = layer["x"].cuda()
+        ys = {}
+        for kind in (1, 0):
+            lmoe.lmoe_set_grouped_gemm(mod.h, kind)
+            y1 = mod.forward(x)
+            y2 = mod.forward(x)
+            torch.cuda.synchronize()
+            assert mod.last_error() == 0
+            assert torch.equal(y1, y2)
+            ys[kind] = y1
+        P.assert_close(P.to_np(ys[1]), P.to_np(ys[0]), "pair vs single-CTA", max_vs_rms=1e-2, mean_rel=2e-3)
+    finally:
+        mod.close()
 
 
 def test_deterministic_and_host_entry_point_agree():
