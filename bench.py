@@ -83,7 +83,9 @@ class ClockSampler:
     """SM clock and throttle reasons sampled while the timed region runs (read-only queries).
 
     NVML, the library nvidia-smi reads, is polled every 0.5 ms from a thread, so even the ~6 ms of 20 decode
-    steps get a dozen samples.  Without NVML, nvidia-smi runs every 200 ms instead.
+    steps get a dozen samples.  While it runs, the interpreter hands the GIL over every 0.1 ms instead of its
+    default 5 ms, so the polling thread is not starved by the launching one.  Without NVML, nvidia-smi runs
+    every 200 ms instead.
     """
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -100,6 +102,7 @@ class ClockSampler:
         self.handle = None
         self.samples = []
         self.done = threading.Event()
+        self.switch = None
 
     def start(self):
         try:
@@ -110,6 +113,8 @@ class ClockSampler:
         except Exception:
             self.nvml = None
         if self.nvml is not None:
+            self.switch = sys.getswitchinterval()
+            sys.setswitchinterval(1e-4)
             self.thread = threading.Thread(target=self._poll, daemon=True)
             self.thread.start()
             return
@@ -143,6 +148,8 @@ class ClockSampler:
             self.done.set()
             if self.thread:
                 self.thread.join(timeout=2)
+            if self.switch is not None:
+                sys.setswitchinterval(self.switch)
             try:
                 max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(self.handle, self.nvml.NVML_CLOCK_SM))
             except Exception:
@@ -216,11 +223,13 @@ EXPERT_RATE = {0: 1.0, 1: 2.0, 2: 2.0, 3: 4.0}
 
 
 #: DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of that kernel as it is now:
-#: the expert up stream of the Nemotron-like decode read 817.4 / 792.2 MB and wrote 1.4 / 2.0 MB in two captured
-#: launches; the NVFP4 decode's expert streams read 224.3 / 224.2 MB and wrote 4.2 / 4.5 MB (up / down).  A kernel
-#: that changes drops out of this table until it is captured again.
+#: the expert up stream of the Nemotron-like decode read 796.4 MB and wrote 1.4 MB per launch (mean of 9
+#: launches); the grouped expert up GEMM of the Nemotron-like prefill read 1442.9 MB and wrote 351.3 MB (one
+#: launch at the full 8192 tokens); the NVFP4 decode's expert streams read 224.3 / 224.2 MB and wrote
+#: 4.2 / 4.5 MB (up / down).  A kernel that changes drops out of this table until it is captured again.
 NCU_TRAFFIC = {
-    ("nemotron_decode", "expert_up_stream"): 806.5e6,
+    ("nemotron_decode", "expert_up_stream"): 797.8e6,
+    ("nemotron_prefill", "expert_up_gemm"): 1794.3e6,
     ("nemotron_decode_nvfp4", "expert_up_stream"): 228.5e6,
     ("nemotron_decode_nvfp4", "expert_down_stream"): 228.8e6,
 }
@@ -331,11 +340,13 @@ def setup_layer(cfg, rank, device):
     return layer, xs
 
 
-def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_clocks=True):
+def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_clocks=True, grouped_kind=None):
     torch.cuda.set_device(device)
     layer, xs = setup_layer(cfg, rank, device)
     T = cfg.tokens
     mod = lmoe.LatentMoE(cfg, layer, max_tokens=T, device=f"cuda:{device}")
+    if grouped_kind is not None:
+        lmoe.lmoe_set_grouped_gemm(mod.h, grouped_kind)
     xd = [x.to(f"cuda:{device}") for x in xs]
     yd = torch.empty_like(xd[0])
     stream = torch.cuda.current_stream()
@@ -661,6 +672,8 @@ def main():
                     help="comma-separated workloads measured beside the main one (reported under `secondary`)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
+    ap.add_argument("--grouped-kind", type=int, choices=[0, 1], default=None,
+                    help="kernel of the grouped expert GEMMs (lmoe_set_grouped_gemm) for the main workload")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -689,7 +702,7 @@ def main():
         if args.ep:
             res = run_ep(cfg, args.steps, args.warmup, rank, world, local, peaks)
         else:
-            res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks)
+            res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks, grouped_kind=args.grouped_kind)
         secondary = None
         if not args.ep and not args.no_secondary:
             secondary = []
@@ -718,6 +731,8 @@ def main():
                 "clocks": res["clocks"],
                 "phases_ms_per_step": {k: v[0] / args.steps for k, v in res["phases"].items()},
                 "routing": res["stats"]}
+        if args.grouped_kind is not None:
+            line["config"]["grouped_gemm_kind"] = args.grouped_kind
         if res.get("graph") is not None:
             line["graph_replay"] = res["graph"]
         if secondary is not None:
