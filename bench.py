@@ -479,8 +479,9 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
 def run_ep(cfg, steps, warmup, rank, world, device, peaks):
     """Expert-parallel steps: this rank holds n_ffn / world experts and routes its own tokens.
 
-    Rows cross ranks by NCCL all-to-all; with one rank nothing moves. A step includes the one host wait of the
-    exchange (the counts that size it).
+    Rows cross ranks by NCCL all-to-all; with one rank nothing moves. Decode-size batches take the block
+    exchange (equal blocks per rank pair, no host wait); larger ones the packed exchange, whose step includes
+    one host wait (the counts that size it).
     """
     from latent_mixture_experts_gemm_b200 import expert_parallel as xp
     torch.cuda.set_device(device)
@@ -575,9 +576,14 @@ def run_ep(cfg, steps, warmup, rank, world, device, peaks):
 
     roof, layer_roof, launches = rooflines(cfg, stats, T, phases, peaks, ms_max / steps)
     roof["kernel_timed_ms_per_step"] = ms_profiled / steps
+    blocks = rk.block_exchange
+    moved = (2 * 2 * (world - 1) * rk.block_rows * cfg.latent) if blocks else 2 * 2 * sent_away * cfg.latent
     exchange = {"ranks": world, "rows_sent_to_other_ranks_per_step": sent_away,
-                "bytes_over_nvlink_per_step": 2 * 2 * sent_away * cfg.latent,
-                "collective": "NCCL all_to_all_single (counts, rows, rows back)" if world > 1 else "none (one rank)"}
+                "bytes_over_nvlink_per_step": moved,
+                "mode": (f"blocks of {rk.block_rows} rows per rank pair, equal splits: no count read on the host"
+                         if blocks else "packed rows, split sizes from the counts read on the host"),
+                "collective": ("NCCL all_to_all_single (counts, row blocks, row blocks back)" if blocks else
+                               "NCCL all_to_all_single (counts, rows, rows back)") if world > 1 else "none (one rank)"}
     rk.close()
     return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
             "e2e": e2e, "clocks": clk, "stats": stats, "exchange": exchange}

@@ -490,6 +490,47 @@ LMOE_API int lmoe_ep_experts(lmoe_handle *h, const void *recv_rows, const int32_
  */
 LMOE_API int lmoe_ep_combine(lmoe_handle *h, const void *ret_rows, void *y, void *stream);
 
+/*
+ * The block exchange: the same three stages with fixed-size blocks, so that
+ * no count has to reach the host during a forward.  Every (sending rank,
+ * receiving rank) pair gets a block of block_rows rows, the same on every
+ * rank, for instance lmoe_ep_block_rows(h) (max_tokens * min(top_k,
+ * n_experts / ep_size), the most rows one rank can send one other rank: a
+ * token's K' experts are distinct).  An all-to-all with equal splits of
+ * block_rows rows (known before the forward) then moves every block, and the
+ * counts (send_counts, device) only tell the receiver how many rows of each
+ * block hold rows.  The blocks cost transfer volume (ep_size * block_rows
+ * latent rows each way per rank, used or not), so the block exchange suits
+ * decode-size batches; the packed stages above send only the routed rows but
+ * need the counts on the host to size the exchange.
+ *
+ * lmoe_ep_dispatch_blocks: as lmoe_ep_dispatch, with send_blocks device bf16
+ *   [ep_size * block_rows, latent]: rank r's rows (experts r * n_local ..,
+ *   ordered as in send_rows) at rows r * block_rows ..; the other rows of
+ *   each block are not written.  block_rows must be at least T * min(top_k,
+ *   n_local) and at most lmoe_ep_block_rows(h) (else LMOE_ERR_INVALID_ARG).
+ *   It uses the handle's gathered-row workspace to sort the rows.
+ * lmoe_ep_experts_blocks: as lmoe_ep_experts, with recv_blocks device bf16
+ *   [ep_size * block_rows, latent]: block s holds rank s's rows for this rank
+ *   (its send_blocks block ep_rank), the first sum(recv_counts[s]) rows of it.
+ *   out_blocks has the same layout (the rows past each block's count are not
+ *   written) and may be recv_blocks.  A source whose counts add up to more
+ *   than block_rows, a negative count, or an expert with more than rows_bound
+ *   rows sets LMOE_ERR_BAD_COUNTS, and the stage computes nothing.
+ * lmoe_ep_combine_blocks: as lmoe_ep_combine, with ret_blocks in the layout
+ *   of send_blocks (the reverse exchange's result); it requires a
+ *   lmoe_ep_dispatch_blocks since the last combine, as lmoe_ep_combine
+ *   requires a lmoe_ep_dispatch.
+ * All asynchronous on `stream`; the stages of one forward on one stream.
+ * The result equals the packed stages' result bit for bit.
+ */
+LMOE_API int64_t lmoe_ep_block_rows(lmoe_handle *h);
+LMOE_API int lmoe_ep_dispatch_blocks(lmoe_handle *h, const void *x, int32_t T, void *send_blocks, int32_t block_rows,
+                                     int32_t *send_counts, void *stream);
+LMOE_API int lmoe_ep_experts_blocks(lmoe_handle *h, const void *recv_blocks, int32_t block_rows,
+                                    const int32_t *recv_counts, int32_t rows_bound, void *out_blocks, void *stream);
+LMOE_API int lmoe_ep_combine_blocks(lmoe_handle *h, const void *ret_blocks, void *y, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -22,16 +22,21 @@ namespace lmoe {
 // give an expert more than rows_bound rows are rejected: every count is taken
 // as 0 (empty tile lists), HDR_EP_BAD is set for the regroup kernels and
 // DEVERR_BAD_COUNTS is reported.
+// Block exchange (block_rows > 0): source s's rows start at s * block_rows,
+// src_off holds each segment's first row there, n_recv is the capacity
+// ep * block_rows, and the counts of a source must add up to at most
+// block_rows instead of the totals adding up to n_recv.
 static __global__ void __launch_bounds__(1024) ep_prep_kernel(const int32_t* __restrict__ recv_counts, int ep,
                                                               int n_local, int n_recv, int rows_bound, int small_max,
                                                               int* __restrict__ counts, int* __restrict__ offsets,
                                                               int4* __restrict__ mt_list, int4* __restrict__ small_list,
                                                               int4* __restrict__ pt_list,
                                                               int* __restrict__ src_off, int* __restrict__ dst_base,
-                                                              int* __restrict__ hdr) {
+                                                              int* __restrict__ hdr, int block_rows) {
     pdl_begin();
     __shared__ int s_cnt[1024];
     __shared__ int s_off[1024];
+    __shared__ int s_so[1024];
     __shared__ int scratch[33];
     __shared__ long long s_total;
     const int n_seg = ep * n_local;
@@ -52,8 +57,13 @@ static __global__ void __launch_bounds__(1024) ep_prep_kernel(const int32_t* __r
     if (j < n_local)
         for (int s = 0; s < ep; ++s) c64 += s_cnt[s * n_local + j];
     bad |= c64 > rows_bound;
+    if (block_rows > 0 && j < ep) {  // each source's rows fit its block
+        long long srows = 0;
+        for (int e = 0; e < n_local; ++e) srows += s_cnt[j * n_local + e];
+        bad |= srows > block_rows;
+    }
     __syncthreads();
-    bad |= s_total != static_cast<long long>(n_recv);
+    if (block_rows == 0) bad |= s_total != static_cast<long long>(n_recv);
     const bool reject = __syncthreads_or(bad) != 0;
     if (reject) {
         cj = 0;
@@ -67,11 +77,14 @@ static __global__ void __launch_bounds__(1024) ep_prep_kernel(const int32_t* __r
     s_off[j] = off;
     int total;
     const int so = block_exclusive_scan(cj, scratch, &total);  // synchronises: s_off and s_cnt are visible
+    s_so[j] = so;
+    __syncthreads();
     if (j < n_seg) {
         const int s = j / n_local, e = j - s * n_local;
         int base = s_off[e];
         for (int q = 0; q < s; ++q) base += s_cnt[q * n_local + e];
-        src_off[j] = so;
+        // block exchange: the segment's first row in source s's block
+        src_off[j] = block_rows > 0 ? s * block_rows + (so - s_so[s * n_local]) : so;
         dst_base[j] = base;
     }
     if (j == 0) {
@@ -130,6 +143,96 @@ static __global__ void __launch_bounds__(256) ep_unregroup_kernel(const __nv_bfl
     const int stride = gridDim.x * EP_ROWS_PER_PASS;
     for (int i = blockIdx.x * EP_ROWS_PER_PASS + (threadIdx.x >> 5); i < n_recv; i += stride) {
         const uint4* src = reinterpret_cast<const uint4*>(rows + static_cast<size_t>(map[i]) * L);
+        uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(i) * L);
+        for (int c = lane; c < L / 8; c += 32) dst[c] = src[c];
+    }
+}
+
+// ---------------------------------------------------------------------------- block exchange
+// The same exchange with every (source rank, destination rank) pair given a fixed block of block_rows rows:
+// the sender's rows for rank r sit at rows r * block_rows .., and rank s's rows arrive at s * block_rows ..
+// (the rest of each block is unused).  The split sizes of the all-to-all are then the same for every pair
+// and known before the forward, so no count has to reach the host.
+
+// Rank of packed send row i: the largest r with offsets[r * n_local] <= i (the rows are sorted by expert id,
+// so rank r's rows are those of experts r * n_local ..).
+__device__ __forceinline__ int ep_rank_of_row(const int* __restrict__ offsets, int n_local, int ep, int i) {
+    int lo = 0, hi = ep - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid * n_local] <= i) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Packed rows (the counting sort's order) <-> rank blocks, one warp per packed row; to_blocks selects the
+// direction.  n_rows is an upper bound on the host; offsets[ep * n_local] is the count on the device.
+static __global__ void __launch_bounds__(256) ep_block_copy_kernel(const __nv_bfloat16* __restrict__ src,
+                                                                   __nv_bfloat16* __restrict__ dst,
+                                                                   const int* __restrict__ offsets, int n_local,
+                                                                   int ep, int block_rows, int n_rows, int L,
+                                                                   int to_blocks) {
+    pdl_begin();
+    const int lane = threadIdx.x & 31;
+    const int n = min(n_rows, offsets[ep * n_local]);
+    const int stride = gridDim.x * EP_ROWS_PER_PASS;
+    for (int i = blockIdx.x * EP_ROWS_PER_PASS + (threadIdx.x >> 5); i < n; i += stride) {
+        const int r = ep_rank_of_row(offsets, n_local, ep, i);
+        const size_t b = static_cast<size_t>(r) * block_rows + (i - offsets[r * n_local]);
+        const uint4* s4 = reinterpret_cast<const uint4*>(src + (to_blocks ? static_cast<size_t>(i) : b) * L);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + (to_blocks ? b : static_cast<size_t>(i)) * L);
+        for (int c = lane; c < L / 8; c += 32) d4[c] = s4[c];
+    }
+}
+
+// Received rank blocks -> expert-major rows (as ep_regroup_kernel), and back.  Row i of the received buffer
+// is row i - s * block_rows of source s's block; it holds a row when that is below source s's count.
+// map[i] = its expert-major row, or -1.
+static __global__ void __launch_bounds__(256) ep_regroup_blocks_kernel(const __nv_bfloat16* __restrict__ recv,
+                                                                       int block_rows, int L,
+                                                                       const int32_t* __restrict__ recv_counts,
+                                                                       const int* __restrict__ src_off,
+                                                                       const int* __restrict__ dst_base, int ep,
+                                                                       int n_local, const int* __restrict__ hdr,
+                                                                       __nv_bfloat16* __restrict__ rows,
+                                                                       int32_t* __restrict__ map) {
+    pdl_begin();
+    if (hdr[HDR_EP_BAD] != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int n = ep * block_rows;
+    const int stride = gridDim.x * EP_ROWS_PER_PASS;
+    for (int i = blockIdx.x * EP_ROWS_PER_PASS + (threadIdx.x >> 5); i < n; i += stride) {
+        // the segment of source s holding row i: the last of s's segments that starts at or before i
+        const int s = i / block_rows;
+        int lo = s * n_local, hi = lo + n_local - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (src_off[mid] <= i) lo = mid;
+            else hi = mid - 1;
+        }
+        const int j = i - src_off[lo];
+        const int dest = j < recv_counts[lo] ? dst_base[lo] + j : -1;
+        if (lane == 0) map[i] = dest;
+        if (dest < 0) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(recv + static_cast<size_t>(i) * L);
+        uint4* dst = reinterpret_cast<uint4*>(rows + static_cast<size_t>(dest) * L);
+        for (int c = lane; c < L / 8; c += 32) dst[c] = src[c];
+    }
+}
+
+static __global__ void __launch_bounds__(256) ep_unregroup_blocks_kernel(const __nv_bfloat16* __restrict__ rows,
+                                                                         const int32_t* __restrict__ map, int n,
+                                                                         int L, const int* __restrict__ hdr,
+                                                                         __nv_bfloat16* __restrict__ out) {
+    pdl_begin();
+    if (hdr[HDR_EP_BAD] != 0) return;
+    const int lane = threadIdx.x & 31;
+    const int stride = gridDim.x * EP_ROWS_PER_PASS;
+    for (int i = blockIdx.x * EP_ROWS_PER_PASS + (threadIdx.x >> 5); i < n; i += stride) {
+        const int m = map[i];
+        if (m < 0) continue;
+        const uint4* src = reinterpret_cast<const uint4*>(rows + static_cast<size_t>(m) * L);
         uint4* dst = reinterpret_cast<uint4*>(out + static_cast<size_t>(i) * L);
         for (int c = lane; c < L / 8; c += 32) dst[c] = src[c];
     }

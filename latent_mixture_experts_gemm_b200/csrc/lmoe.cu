@@ -601,6 +601,7 @@ struct lmoe_handle {
     // expert-parallel forward in progress: the dispatch's x and T (ep_T < 0: none)
     const void* ep_x = nullptr;
     int ep_T = -1;
+    int64_t ep_block_rows = 0;  // the forward in progress exchanges rank blocks of this many rows (0: packed)
     bool stats_ep = false;  // the header's row / tile counts are those of the last experts stage
     unsigned long long timeout_ns = 1000000000ull;
     // weight descriptors: router/projection operands for both column tiles, expert weights, workspace operands
@@ -1511,6 +1512,7 @@ int lmoe_ep_dispatch(lmoe_handle* h, const void* x, int32_t T, void* send_rows, 
             return LMOE_ERR_CUDA;
         h->ep_x = nullptr;
         h->ep_T = 0;
+        h->ep_block_rows = 0;
         return LMOE_OK;
     }
     if (x == nullptr || send_rows == nullptr || !aligned16(x) || !aligned16(send_rows)) return LMOE_ERR_INVALID_ARG;
@@ -1522,6 +1524,7 @@ int lmoe_ep_dispatch(lmoe_handle* h, const void* x, int32_t T, void* send_rows, 
         return LMOE_ERR_CUDA;
     h->ep_x = x;
     h->ep_T = T;
+    h->ep_block_rows = 0;
     return LMOE_OK;
 }
 
@@ -1561,7 +1564,7 @@ int lmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const int32_t* recv_c
         PhaseScope ps(h, PH_EP_REGROUP, s, 2);
         launch(ep_prep_kernel, 1, 1024, 0, s, recv_counts, ep, nl, static_cast<int>(n_recv),
                static_cast<int>(rows_bound), small, h->at<int>(p.ep_counts), h->at<int>(p.ep_offsets),
-               h->at<int4>(p.mt_list), h->at<int4>(p.small_list), h->at<int4>(p.pt_list), src_off, dst_base, hdr);
+               h->at<int4>(p.mt_list), h->at<int4>(p.small_list), h->at<int4>(p.pt_list), src_off, dst_base, hdr, 0);
         launch(ep_regroup_kernel, grid, 32 * EP_ROWS_PER_PASS, static_cast<size_t>(2 * n_seg + 1) * 4, s,
                static_cast<const __nv_bfloat16*>(recv_rows), static_cast<int>(n_recv), L,
                static_cast<const int*>(src_off), static_cast<const int*>(dst_base), n_seg,
@@ -1578,8 +1581,138 @@ int lmoe_ep_experts(lmoe_handle* h, const void* recv_rows, const int32_t* recv_c
     return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- the block exchange
+namespace {
+// The most rows one rank can send to one other rank in a forward of up to max_tokens tokens: each token has
+// at most min(top_k, n_local) slots on a rank's experts (a token's experts are distinct).
+int64_t ep_block_cap(const lmoe_handle* h) {
+    return static_cast<int64_t>(h->c.max_tokens) * std::min(h->c.top_k, h->n_local);
+}
+}  // namespace
+
+int64_t lmoe_ep_block_rows(lmoe_handle* h) {
+    return h == nullptr ? 0 : ep_block_cap(h);
+}
+
+int lmoe_ep_dispatch_blocks(lmoe_handle* h, const void* x, int32_t T, void* send_blocks, int32_t block_rows,
+                            int32_t* send_counts, void* stream) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    if (h->c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
+    if (block_rows < 1 || block_rows < static_cast<int64_t>(T) * std::min(h->c.top_k, h->n_local) ||
+        block_rows > ep_block_cap(h))
+        return LMOE_ERR_INVALID_ARG;
+    if (send_counts == nullptr || !aligned16(send_counts)) return LMOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(send_counts, 0, static_cast<size_t>(h->c.n_experts) * 4, s) != cudaSuccess)
+            return LMOE_ERR_CUDA;
+        h->ep_x = nullptr;
+        h->ep_T = 0;
+        h->ep_block_rows = block_rows;
+        return LMOE_OK;
+    }
+    if (x == nullptr || send_blocks == nullptr || !aligned16(x) || !aligned16(send_blocks)) return LMOE_ERR_INVALID_ARG;
+    const Plan& p = h->p;
+    __nv_bfloat16* packed = h->at<__nv_bfloat16>(p.rows);
+    const int st = run_front(h, x, T, s, packed, h->small_max);
+    if (st != LMOE_OK) return st;
+    const int ep = ep_ranks(h->c), nl = h->n_local, L = h->c.latent;
+    const int n_rows = T * h->c.top_k;
+    {
+        PhaseScope ps(h, PH_EP_REGROUP, s, 1);
+        launch(ep_block_copy_kernel, static_cast<unsigned>(std::min<long>((n_rows + EP_ROWS_PER_PASS - 1) / EP_ROWS_PER_PASS,
+                                                                          8L * h->num_sms)),
+               32 * EP_ROWS_PER_PASS, 0, s, static_cast<const __nv_bfloat16*>(packed),
+               static_cast<__nv_bfloat16*>(send_blocks), static_cast<const int*>(h->at<int>(p.offsets)), nl, ep,
+               static_cast<int>(block_rows), n_rows, L, 1);
+    }
+    if (cudaMemcpyAsync(send_counts, h->at<int>(p.counts), static_cast<size_t>(h->c.n_experts) * 4,
+                        cudaMemcpyDeviceToDevice, s) != cudaSuccess)
+        return LMOE_ERR_CUDA;
+    h->ep_x = x;
+    h->ep_T = T;
+    h->ep_block_rows = block_rows;
+    return LMOE_OK;
+}
+
+int lmoe_ep_experts_blocks(lmoe_handle* h, const void* recv_blocks, int32_t block_rows, const int32_t* recv_counts,
+                           int32_t rows_bound, void* out_blocks, void* stream) {
+    if (h == nullptr) return LMOE_ERR_INVALID_ARG;
+    const lmoe_config& c = h->c;
+    if (c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    if (block_rows < 1 || block_rows > ep_block_cap(h) || rows_bound < 1) return LMOE_ERR_INVALID_ARG;
+    if (recv_blocks == nullptr || recv_counts == nullptr || out_blocks == nullptr || !aligned16(recv_blocks) ||
+        !aligned16(recv_counts) || !aligned16(out_blocks))
+        return LMOE_ERR_INVALID_ARG;
+    const Plan& p = h->p;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int ep = ep_ranks(c), nl = h->n_local, L = c.latent;
+    const int n = ep * block_rows;  // the received buffer's rows, used or not
+    const int small = choose_small(h, rows_bound);
+    h->last_small = small;
+    h->stats_ep = true;
+    int* hdr = h->at<int>(p.hdr);
+    int* src_off = h->at<int>(p.ep_src);
+    int* dst_base = h->at<int>(p.ep_dst);
+    int32_t* map = h->at<int32_t>(p.ep_map);
+    __nv_bfloat16* rows = h->at<__nv_bfloat16>(p.rows);
+    const unsigned grid =
+        static_cast<unsigned>(std::min<long>((n + EP_ROWS_PER_PASS - 1) / EP_ROWS_PER_PASS, 8L * h->num_sms));
+    {
+        PhaseScope ps(h, PH_EP_REGROUP, s, 2);
+        launch(ep_prep_kernel, 1, 1024, 0, s, recv_counts, ep, nl, n, static_cast<int>(rows_bound), small,
+               h->at<int>(p.ep_counts), h->at<int>(p.ep_offsets), h->at<int4>(p.mt_list), h->at<int4>(p.small_list),
+               h->at<int4>(p.pt_list), src_off, dst_base, hdr, static_cast<int>(block_rows));
+        launch(ep_regroup_blocks_kernel, grid, 32 * EP_ROWS_PER_PASS, 0, s,
+               static_cast<const __nv_bfloat16*>(recv_blocks), static_cast<int>(block_rows), L, recv_counts,
+               static_cast<const int*>(src_off), static_cast<const int*>(dst_base), ep, nl,
+               static_cast<const int*>(hdr), rows, map);
+    }
+    const int st = run_experts(h, small, rows_bound > small, s);
+    if (st != LMOE_OK) return st;
+    {
+        PhaseScope ps(h, PH_EP_REGROUP, s, 1);
+        launch(ep_unregroup_blocks_kernel, grid, 32 * EP_ROWS_PER_PASS, 0, s, static_cast<const __nv_bfloat16*>(rows),
+               static_cast<const int32_t*>(map), n, L, static_cast<const int*>(hdr),
+               static_cast<__nv_bfloat16*>(out_blocks));
+    }
+    return cudaGetLastError() == cudaSuccess ? LMOE_OK : LMOE_ERR_CUDA;
+}
+
+int lmoe_ep_combine_blocks(lmoe_handle* h, const void* ret_blocks, void* y, void* stream) {
+    if (h == nullptr || h->ep_T < 0 || h->ep_block_rows < 1) return LMOE_ERR_INVALID_ARG;
+    if (h->c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
+    const int T = h->ep_T;
+    const void* x = h->ep_x;
+    if (T == 0) {
+        h->ep_T = -1;
+        h->ep_block_rows = 0;
+        return LMOE_OK;
+    }
+    if (ret_blocks == nullptr || y == nullptr || !aligned16(ret_blocks) || !aligned16(y)) return LMOE_ERR_INVALID_ARG;
+    const size_t bytes = static_cast<size_t>(T) * h->c.d * 2;
+    const uintptr_t xa = reinterpret_cast<uintptr_t>(x), ya = reinterpret_cast<uintptr_t>(y);
+    if (xa < ya + bytes && ya < xa + bytes) return LMOE_ERR_INVALID_ARG;
+    const Plan& p = h->p;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int n_rows = T * h->c.top_k;
+    __nv_bfloat16* packed = h->at<__nv_bfloat16>(p.rows);
+    {
+        PhaseScope ps(h, PH_EP_REGROUP, s, 1);
+        launch(ep_block_copy_kernel, static_cast<unsigned>(std::min<long>((n_rows + EP_ROWS_PER_PASS - 1) / EP_ROWS_PER_PASS,
+                                                                          8L * h->num_sms)),
+               32 * EP_ROWS_PER_PASS, 0, s, static_cast<const __nv_bfloat16*>(ret_blocks), packed,
+               static_cast<const int*>(h->at<int>(p.offsets)), h->n_local, ep_ranks(h->c),
+               static_cast<int>(h->ep_block_rows), n_rows, h->c.latent, 0);
+    }
+    h->ep_T = -1;
+    h->ep_block_rows = 0;
+    return run_back(h, packed, x, y, T, s);
+}
+
 int lmoe_ep_combine(lmoe_handle* h, const void* ret_rows, void* y, void* stream) {
-    if (h == nullptr || h->ep_T < 0) return LMOE_ERR_INVALID_ARG;
+    if (h == nullptr || h->ep_T < 0 || h->ep_block_rows != 0) return LMOE_ERR_INVALID_ARG;
     if (h->c.expert_fmt != LMOE_FMT_BF16) return LMOE_ERR_UNSUPPORTED_SHAPE;
     const int T = h->ep_T;
     const void* x = h->ep_x;

@@ -23,6 +23,13 @@ NVLink on GPUs, gloo on CPU in the tests. One forward on one rank:
 5. experts;
 6. the reverse all-to-all of the expert outputs;
 7. combine.
+
+The block exchange (``ep_forward_blocks``, the ``*_blocks`` stages) gives every
+pair of ranks a fixed block of rows, so the all-to-alls have equal splits known
+before the forward and step 3 disappears: no forward waits on the device. The
+blocks carry unused rows, so it is the exchange for decode-size batches;
+``ExpertParallelLatentMoE`` takes it when the blocks of one forward are small
+(``block_limit_bytes``).
 """
 from __future__ import annotations
 
@@ -73,6 +80,14 @@ class AllToAll:
         dist.all_to_all_single(out, send_counts, group=self.group)
         return out
 
+    def blocks(self, out: torch.Tensor, inp: torch.Tensor) -> torch.Tensor:
+        """All-to-all of equal blocks: block r of ``inp`` goes to rank r, and block s of ``out`` comes from
+        rank s.  No split sizes: nothing has to be known on the host."""
+        if self.world == 1:
+            return inp
+        dist.all_to_all_single(out, inp, group=self.group)
+        return out
+
     def rows(self, out: torch.Tensor, inp: torch.Tensor, out_splits: List[int], in_splits: List[int]) -> torch.Tensor:
         """All-to-all of rows. ``in_splits[r]`` rows of ``inp`` go to rank r. ``out[...]`` receives
         ``out_splits[s]`` rows from each rank s, in rank order."""
@@ -105,6 +120,22 @@ def ep_forward(stages, exchange, x: torch.Tensor, y: Optional[torch.Tensor] = No
     return stages.combine(ret, y)
 
 
+def ep_forward_blocks(stages, exchange, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """One expert-parallel forward of ``x`` on this rank with the block exchange: the same steps as
+    ``ep_forward``, every rank pair moving a fixed block of rows, and no device-to-host copy.
+
+    ``stages`` provides ``dispatch_blocks(x) -> (send_blocks, send_counts)``, ``recv_blocks()``,
+    ``ret_blocks()``, ``experts_blocks(recv_blocks, recv_counts) -> out_blocks`` and
+    ``combine_blocks(ret_blocks, y) -> y``.
+    """
+    send_blocks, send_counts = stages.dispatch_blocks(x)
+    recv_counts = exchange.counts(send_counts)
+    recv = exchange.blocks(stages.recv_blocks(), send_blocks)
+    out = stages.experts_blocks(recv, recv_counts)
+    ret = exchange.blocks(stages.ret_blocks(), out)
+    return stages.combine_blocks(ret, y)
+
+
 def local_experts(layer: Dict[str, torch.Tensor], n_ffn: int, ep_size: int, ep_rank: int) -> Dict[str, torch.Tensor]:
     """The layer's tensors as rank ``ep_rank`` holds them.
 
@@ -131,10 +162,15 @@ class ExpertParallelLatentMoE:
       the most rows this rank's experts can receive.
 
     The experts stage writes its outputs over the received rows.
+
+    With the block exchange (taken when ``ep_size * block_rows`` latent rows are at most
+    ``block_limit_bytes``, block_rows = ``max_tokens * min(top_k, n_local)``) there are also
+    ``send_blocks`` and ``ret_blocks`` of ``[ep_size * block_rows, latent]``; ``recv_rows`` has that size
+    already.
     """
 
     def __init__(self, cfg, layer: Dict[str, torch.Tensor], max_tokens: int, ep_size: int, ep_rank: int,
-                 device: str = "cuda", group=None, exchange=None):
+                 device: str = "cuda", group=None, exchange=None, block_limit_bytes: int = 64 << 20):
         self.cfg = cfg
         self.ep_size, self.ep_rank = int(ep_size), int(ep_rank)
         self.mod = lmoe.LatentMoE(cfg, local_experts(layer, cfg.n_ffn, self.ep_size, self.ep_rank), max_tokens,
@@ -150,6 +186,12 @@ class ExpertParallelLatentMoE:
         self.send_counts = torch.empty(cfg.n_ffn, dtype=torch.int32, device=self.device)
         self.exchange = exchange if exchange is not None else AllToAll(group)
         self._x = None
+        self.block_rows = lmoe.lmoe_ep_block_rows(self.mod.h)
+        self.rows_bound = self.ep_size * int(max_tokens)  # an expert gets at most one row per token of any rank
+        self.block_exchange = self.ep_size * self.block_rows * L * 2 <= block_limit_bytes
+        if self.block_exchange:
+            self.send_blocks = torch.empty((self.ep_size * self.block_rows, L), **bf)
+            self.ret_blocks_buf = torch.empty((self.ep_size * self.block_rows, L), **bf)
 
     # ---- the stages (the interface ep_forward drives)
     def dispatch(self, x: torch.Tensor):
@@ -176,8 +218,34 @@ class ExpertParallelLatentMoE:
         self._x = None
         return y
 
+    # ---- the block-exchange stages (the interface ep_forward_blocks drives)
+    def dispatch_blocks(self, x: torch.Tensor):
+        self._x = x
+        lmoe.lmoe_ep_dispatch_blocks(self.mod.h, x, self.send_blocks, self.block_rows, self.send_counts)
+        return self.send_blocks, self.send_counts
+
+    def recv_blocks(self) -> torch.Tensor:
+        return self.recv_rows
+
+    def ret_blocks(self) -> torch.Tensor:
+        return self.ret_blocks_buf
+
+    def experts_blocks(self, recv_blocks: torch.Tensor, recv_counts: torch.Tensor) -> torch.Tensor:
+        lmoe.lmoe_ep_experts_blocks(self.mod.h, recv_blocks, self.block_rows, recv_counts, self.rows_bound,
+                                    recv_blocks)
+        return recv_blocks
+
+    def combine_blocks(self, ret_blocks: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if y is None:
+            y = torch.empty_like(self._x)
+        lmoe.lmoe_ep_combine_blocks(self.mod.h, ret_blocks, y)
+        self._x = None
+        return y
+
     # ---- a whole forward
     def forward(self, x: torch.Tensor, y: Optional[torch.Tensor] = None) -> torch.Tensor:
+        if self.block_exchange:
+            return ep_forward_blocks(self, self.exchange, x, y)
         return ep_forward(self, self.exchange, x, y)
 
     def last_error(self) -> int:

@@ -90,6 +90,11 @@ def lib() -> ctypes.CDLL:
         L.lmoe_ep_dispatch.argtypes = [P, P, I32, P, P, P]
         L.lmoe_ep_experts.argtypes = [P, P, P, I32, I32, P, P]
         L.lmoe_ep_combine.argtypes = [P, P, P, P]
+        L.lmoe_ep_block_rows.argtypes = [P]
+        L.lmoe_ep_block_rows.restype = ctypes.c_int64
+        L.lmoe_ep_dispatch_blocks.argtypes = [P, P, I32, P, I32, P, P]
+        L.lmoe_ep_experts_blocks.argtypes = [P, P, I32, P, I32, P, P]
+        L.lmoe_ep_combine_blocks.argtypes = [P, P, P, P]
         _lib = L
     return _lib
 
@@ -266,6 +271,33 @@ def lmoe_ep_experts(h: int, recv_rows: torch.Tensor, recv_counts: torch.Tensor, 
 def lmoe_ep_combine(h: int, ret_rows: torch.Tensor, y: torch.Tensor, stream=None) -> None:
     """Expert-parallel stage 3: aggregation, W_up and residual into ``y``."""
     _check("lmoe_ep_combine", lib().lmoe_ep_combine(h, ret_rows.data_ptr(), y.data_ptr(), _stream(stream)))
+
+
+def lmoe_ep_block_rows(h: int) -> int:
+    """Rows of one rank-pair block of the block exchange (the most one rank can send one other rank)."""
+    return int(lib().lmoe_ep_block_rows(h))
+
+
+def lmoe_ep_dispatch_blocks(h: int, x: torch.Tensor, send_blocks: torch.Tensor, block_rows: int,
+                            send_counts: torch.Tensor, stream=None) -> None:
+    """Expert-parallel stage 1, block exchange: rank r's rows at rows r * block_rows of ``send_blocks``."""
+    _check("lmoe_ep_dispatch_blocks", lib().lmoe_ep_dispatch_blocks(
+        h, x.data_ptr(), int(x.shape[0]), send_blocks.data_ptr(), int(block_rows), send_counts.data_ptr(),
+        _stream(stream)))
+
+
+def lmoe_ep_experts_blocks(h: int, recv_blocks: torch.Tensor, block_rows: int, recv_counts: torch.Tensor,
+                           rows_bound: int, out_blocks: torch.Tensor, stream=None) -> None:
+    """Expert-parallel stage 2, block exchange: block s of ``recv_blocks`` holds rank s's rows."""
+    _check("lmoe_ep_experts_blocks", lib().lmoe_ep_experts_blocks(
+        h, recv_blocks.data_ptr(), int(block_rows), recv_counts.data_ptr(), int(rows_bound), out_blocks.data_ptr(),
+        _stream(stream)))
+
+
+def lmoe_ep_combine_blocks(h: int, ret_blocks: torch.Tensor, y: torch.Tensor, stream=None) -> None:
+    """Expert-parallel stage 3, block exchange: the expert outputs in the layout of the send blocks."""
+    _check("lmoe_ep_combine_blocks", lib().lmoe_ep_combine_blocks(h, ret_blocks.data_ptr(), y.data_ptr(),
+                                                                  _stream(stream)))
 
 
 def lmoe_nvfp4_encode_weights(w: torch.Tensor, stream=None):

@@ -10,7 +10,10 @@ Every rank's output must equal the oracle's whole-layer output for its tokens
 to fp64 rounding. A row sent to the wrong rank or expert, or returned to the
 wrong slot, fails this by a wide margin. Rank counts 2 and 3; uneven token
 counts; a rank with no tokens; skewed routing; MoE++ bypass experts and a
-shared expert.
+shared expert.  Both exchanges: the packed one (split sizes from the counts on
+the host) and the block one (equal blocks, nothing read on the host; the
+stand-in fills the unused rows of every block with NaN, so a row read from
+outside a block's count poisons the output).
 """
 import datetime
 import os
@@ -47,9 +50,10 @@ def _act(cfg, u: torch.Tensor) -> torch.Tensor:
 class OracleStages:
     """fp64 stand-in for the library's three stages on one rank (test only)."""
 
-    def __init__(self, cfg, layer, ep, rank):
+    def __init__(self, cfg, layer, ep, rank, max_tokens=0):
         self.cfg, self.layer, self.ep, self.rank = cfg, layer, ep, rank
         self.nl = cfg.n_ffn // ep
+        self.block_rows = max_tokens * min(cfg.top_k, self.nl)  # block exchange: rows per rank pair
         f = lambda t: None if t is None else t.to(torch.float64)  # noqa: E731
         loc = xp.local_experts(layer, cfg.n_ffn, ep, rank)
         self.w1, self.w2 = f(loc["w1"]), f(loc["w2"])
@@ -119,12 +123,50 @@ class OracleStages:
         return out
 
 
+    # ---- block exchange: the same arithmetic on rank blocks of block_rows rows
+    def _blank(self):
+        return torch.full((self.ep * self.block_rows, self.cfg.latent), float("nan"), dtype=torch.float64)
+
+    def dispatch_blocks(self, x):
+        send_rows, counts = self.dispatch(x)
+        per = counts.view(self.ep, self.nl).sum(1).tolist()
+        self.send_per = per
+        blocks, off = self._blank(), 0
+        for r, n in enumerate(per):
+            assert n <= self.block_rows
+            blocks[r * self.block_rows:r * self.block_rows + n] = send_rows[off:off + n]
+            off += n
+        return blocks, counts
+
+    def recv_blocks(self):
+        return self._blank()
+
+    ret_blocks = recv_blocks
+
+    def experts_blocks(self, recv_blocks, recv_counts):
+        B = self.block_rows
+        per = recv_counts.view(self.ep, self.nl).sum(1).tolist()
+        rows = torch.cat([recv_blocks[s * B:s * B + n] for s, n in enumerate(per)])
+        bound = int(recv_counts.view(self.ep, self.nl).sum(0).max())
+        out_rows = self.experts(rows, recv_counts, int(sum(per)), bound)
+        out, off = self._blank(), 0
+        for s, n in enumerate(per):
+            out[s * B:s * B + n] = out_rows[off:off + n]
+            off += n
+        return out
+
+    def combine_blocks(self, ret_blocks, y):
+        B = self.block_rows
+        ret = torch.cat([ret_blocks[r * B:r * B + n] for r, n in enumerate(self.send_per)])
+        return self.combine(ret, y)
+
+
 def _tokens(cfg, ep):
     """Per-rank token counts: uneven, and with three ranks one rank has none."""
     return [13, 21] if ep == 2 else [17, 0, 9]
 
 
-def _rank_main(rank, world, port, name, q):
+def _rank_main(rank, world, port, name, q, blocks=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     tdist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
     try:
@@ -133,8 +175,8 @@ def _rank_main(rank, world, port, name, q):
         T = _tokens(cfg, world)
         t0 = sum(T[:rank])
         x = layer["x"][t0:t0 + T[rank]]
-        st = OracleStages(cfg, layer, world, rank)
-        y = xp.ep_forward(st, xp.AllToAll(), x)
+        st = OracleStages(cfg, layer, world, rank, max_tokens=max(T))
+        y = (xp.ep_forward_blocks if blocks else xp.ep_forward)(st, xp.AllToAll(), x)
         ref = oracle.forward(cfg, layer, x)["y"] if T[rank] else np.zeros((0, cfg.d))
         err = float(np.max(np.abs(y.numpy() - ref))) if T[rank] else 0.0
         q.put((rank, err, float(np.max(np.abs(ref))) if T[rank] else 1.0, st.seen_bounds))
@@ -149,13 +191,15 @@ def _free_port():
         return s.getsockname()[1]
 
 
+@pytest.mark.parametrize("exchange", ["packed", "blocks"])
 @pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("name", list(CASES))
-def test_exchange_over_gloo_ranks_matches_the_oracle(name, world):
+def test_exchange_over_gloo_ranks_matches_the_oracle(name, world, exchange):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, name, q)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, name, q, exchange == "blocks"))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:
@@ -167,13 +211,14 @@ def test_exchange_over_gloo_ranks_matches_the_oracle(name, world):
         assert len(bounds) == 1
 
 
-def test_one_rank_needs_no_process_group():
+@pytest.mark.parametrize("exchange", ["packed", "blocks"])
+def test_one_rank_needs_no_process_group(exchange):
     cfg = CASES["swiglu_bypass_shared_skew"]
     layer = synth.make_layer(cfg, tokens=19)
-    st = OracleStages(cfg, layer, 1, 0)
+    st = OracleStages(cfg, layer, 1, 0, max_tokens=19)
     ex = xp.AllToAll()
     assert ex.world == 1
-    y = xp.ep_forward(st, ex, layer["x"])
+    y = (xp.ep_forward_blocks if exchange == "blocks" else xp.ep_forward)(st, ex, layer["x"])
     ref = oracle.forward(cfg, layer)["y"]
     assert np.max(np.abs(y.numpy() - ref)) <= 1e-10 * np.max(np.abs(ref))
 

@@ -12,6 +12,9 @@
     result does not depend on which other rows share its tile.
 * Counts that do not match the rows are reported as LMOE_ERR_BAD_COUNTS, and
   the stage then computes nothing; bad calls are rejected.
+* The block exchange (every rank pair a fixed block of rows, the stages'
+  ``*_blocks`` forms) gives the packed exchange's outputs bit for bit, on the
+  same emulated ranks; with one rank it equals ``lmoe_forward``.
 """
 import warnings
 
@@ -74,6 +77,29 @@ def _emulated_forward(ranks, xs):
         if n_send:
             torch.cat([outs[r][int(per[:s, r].sum()):int(per[:s + 1, r].sum())] for r in range(N)], out=ret)
         ys.append(ranks[s].combine(ret))
+    return ys
+
+
+def _emulated_forward_blocks(ranks, xs):
+    """The same forward with the block exchange: block r of rank s's send blocks becomes block s of rank r's
+    receive blocks, and back; no count is read on the host."""
+    N = len(ranks)
+    nl = ranks[0].cfg.n_ffn // N
+    B = ranks[0].block_rows
+    sends = [r.dispatch_blocks(x.cuda()) for r, x in zip(ranks, xs)]
+    outs = []
+    for r in range(N):
+        recv = ranks[r].recv_blocks()
+        for s in range(N):
+            recv[s * B:(s + 1) * B].copy_(sends[s][0][r * B:(r + 1) * B])
+        rc = torch.stack([sends[s][1][r * nl:(r + 1) * nl] for s in range(N)]).contiguous()
+        outs.append(ranks[r].experts_blocks(recv, rc))
+    ys = []
+    for s in range(N):
+        ret = ranks[s].ret_blocks()
+        for r in range(N):
+            ret[r * B:(r + 1) * B].copy_(outs[r][s * B:(s + 1) * B])
+        ys.append(ranks[s].combine_blocks(ret))
     return ys
 
 
@@ -184,6 +210,81 @@ def test_one_rank_stages_bit_identical_to_forward(name, T):
             one.close()
     finally:
         mod.close()
+
+
+@pytest.mark.parametrize("name", ["medium_4_ranks_ragged_empty", "medium_2_ranks_swiglu_bypass_shared_skew",
+                                  "standard_moe_2_ranks", "latent_router_2_ranks", "decode_8_ranks_nemotron_shape",
+                                  "decode_2_ranks_one_token"])
+def test_block_exchange_equals_the_packed_exchange(name):
+    cfg, tokens = CASES[name]
+    layer = synth.make_layer(cfg, tokens=sum(tokens))
+    xs = _split(layer, tokens)
+    ranks = _make_ranks(cfg, layer, tokens)
+    try:
+        assert all(r.block_exchange for r in ranks)
+        packed = _emulated_forward(ranks, xs)
+        blocks = _emulated_forward_blocks(ranks, xs)
+        torch.cuda.synchronize()
+        for r, (a, b) in enumerate(zip(packed, blocks)):
+            assert torch.equal(a, b), f"rank {r}: {(a.float() - b.float()).abs().max().item()}"
+        assert all(rk.last_error() == 0 for rk in ranks)
+    finally:
+        _close(ranks)
+
+
+@pytest.mark.parametrize("T", [32, 5])
+def test_one_rank_block_exchange_equals_forward(T):
+    """One rank, the decode shape: the block stages (no host read of any count) give lmoe_forward's output
+    bit for bit when the expert-path threshold matches (rows_bound = T)."""
+    cfg = DECODE.with_(seed=99)
+    layer = synth.make_layer(cfg, tokens=T)
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=T)
+    try:
+        x = layer["x"].cuda()
+        ref = mod.forward(x)
+        B = lmoe.lmoe_ep_block_rows(mod.h)
+        assert B == T * cfg.top_k
+        blocks = torch.empty((B, cfg.latent), dtype=torch.bfloat16, device="cuda")
+        counts = torch.empty(cfg.n_ffn, dtype=torch.int32, device="cuda")
+        lmoe.lmoe_ep_dispatch_blocks(mod.h, x, blocks, B, counts)
+        lmoe.lmoe_ep_experts_blocks(mod.h, blocks, B, counts, T, blocks)
+        y = torch.empty_like(x)
+        lmoe.lmoe_ep_combine_blocks(mod.h, blocks, y)
+        torch.cuda.synchronize()
+        assert mod.last_error() == 0
+        assert torch.equal(y, ref)
+        # the stages of the two exchanges do not mix within a forward
+        lmoe.lmoe_ep_dispatch_blocks(mod.h, x, blocks, B, counts)
+        with pytest.raises(lmoe.LmoeError):
+            lmoe.lmoe_ep_combine(mod.h, blocks, y)
+        lmoe.lmoe_ep_combine_blocks(mod.h, blocks, y)
+        with pytest.raises(lmoe.LmoeError):  # a block smaller than T * min(K', n_local)
+            lmoe.lmoe_ep_dispatch_blocks(mod.h, x, blocks, B - 1, counts)
+        torch.cuda.synchronize()
+    finally:
+        mod.close()
+
+
+def test_block_counts_over_the_block_are_reported():
+    cfg = MEDIUM
+    layer = synth.make_layer(cfg, tokens=4)
+    rk = xp.ExpertParallelLatentMoE(cfg, layer, max_tokens=4, ep_size=2, ep_rank=1)  # 32 local experts
+    try:
+        B = rk.block_rows                         # 4 tokens x min(6, 32) = 24
+        assert B == 24
+        blocks = torch.zeros((2 * B, cfg.latent), dtype=torch.bfloat16, device="cuda")
+        counts = torch.zeros(64, dtype=torch.int32)  # [2 sources][32 local experts]; rows_bound 2 x 4 = 8
+        counts[0:3] = 8
+        counts[3] = 1                             # source 0 sends 25 rows: more than its block
+        rk.experts_blocks(blocks, counts.cuda())
+        torch.cuda.synchronize()
+        assert rk.last_error() == -8               # LMOE_ERR_BAD_COUNTS
+        counts[3] = 0                             # 24 rows: fits
+        rk.experts_blocks(blocks, counts.cuda())
+        torch.cuda.synchronize()
+        assert rk.last_error() == 0
+    finally:
+        rk.close()
 
 
 def test_inconsistent_counts_are_reported_and_compute_nothing():
