@@ -109,6 +109,9 @@ class ClockSampler:
             import pynvml
             pynvml.nvmlInit()
             self.handle = pynvml.nvmlDeviceGetHandleByUUID(self.uuid)
+            # the first queries after initialisation are slow (milliseconds): make them before the timed region
+            pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+            pynvml.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
             self.nvml = pynvml
         except Exception:
             self.nvml = None
@@ -476,7 +479,7 @@ def run_gpu(cfg, steps, warmup, rank, world, device, peaks, with_e2e=True, with_
             "e2e": e2e, "clocks": clk, "stats": stats, "graph": graph}
 
 
-def run_ep(cfg, steps, warmup, rank, world, device, peaks):
+def run_ep(cfg, steps, warmup, rank, world, device, peaks, exchange_mode="auto"):
     """Expert-parallel steps: this rank holds n_ffn / world experts and routes its own tokens.
 
     Rows cross ranks by NCCL all-to-all; with one rank nothing moves. Decode-size batches take the block
@@ -487,7 +490,9 @@ def run_ep(cfg, steps, warmup, rank, world, device, peaks):
     torch.cuda.set_device(device)
     layer, xs = setup_layer(cfg, rank, device)
     T = cfg.tokens
-    rk = xp.ExpertParallelLatentMoE(cfg, layer, max_tokens=T, ep_size=world, ep_rank=rank, device=f"cuda:{device}")
+    limit = {"auto": 64 << 20, "packed": -1, "blocks": 1 << 62}[exchange_mode]
+    rk = xp.ExpertParallelLatentMoE(cfg, layer, max_tokens=T, ep_size=world, ep_rank=rank, device=f"cuda:{device}",
+                                    block_limit_bytes=limit)
     xd = [x.to(f"cuda:{device}") for x in xs]
     yd = torch.empty_like(xd[0])
     stream = torch.cuda.current_stream()
@@ -574,6 +579,36 @@ def run_ep(cfg, steps, warmup, rank, world, device, peaks):
            "h2d_bytes_per_step": int(xh[0].numel() * xh[0].element_size()),
            "d2h_bytes_per_step": int(yh.numel() * yh.element_size()), "ms_per_step": e2e_ms / steps}
 
+    # With the block exchange a step has no host wait, so one rank's step can be captured in a CUDA graph and
+    # replayed (with several ranks the graph would hold the NCCL exchanges: not measured here).
+    graph = None
+    if rk.block_exchange and world == 1:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            rk.forward(xd[0], yd)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graphs = []
+        for i in range(N_INPUT_BATCHES):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                rk.forward(xd[i], yd)
+            graphs.append(gr)
+        for i in range(warmup):
+            graphs[i % N_INPUT_BATCHES].replay()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for i in range(steps):
+            graphs[i % N_INPUT_BATCHES].replay()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        g_ms = ev0.elapsed_time(ev1)
+        check("in the graph-replay region")
+        graph = {"value": T * steps / (g_ms / 1e3), "unit": "tokens/s", "ms_per_step": g_ms / steps,
+                 "launch": "one CUDA graph per expert-parallel step (block exchange, one rank), replayed"}
+        del graphs
+
     roof, layer_roof, launches = rooflines(cfg, stats, T, phases, peaks, ms_max / steps)
     roof["kernel_timed_ms_per_step"] = ms_profiled / steps
     blocks = rk.block_exchange
@@ -586,7 +621,7 @@ def run_ep(cfg, steps, warmup, rank, world, device, peaks):
                                "NCCL all_to_all_single (counts, rows, rows back)") if world > 1 else "none (one rank)"}
     rk.close()
     return {"ms": ms_max, "phases": phases, "launches": launches, "roofline": roof, "layer_roofline": layer_roof,
-            "e2e": e2e, "clocks": clk, "stats": stats, "exchange": exchange}
+            "e2e": e2e, "clocks": clk, "stats": stats, "exchange": exchange, "graph": graph}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU) arm
@@ -678,6 +713,8 @@ def main():
                     help="comma-separated workloads measured beside the main one (reported under `secondary`)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ep", action="store_true", help="expert parallelism over the ranks instead of replicas")
+    ap.add_argument("--ep-exchange", default="auto", choices=["auto", "packed", "blocks"],
+                    help="--ep: the block exchange for small batches (auto), or one of the two always")
     ap.add_argument("--grouped-kind", type=int, choices=[0, 1], default=None,
                     help="kernel of the grouped expert GEMMs (lmoe_set_grouped_gemm) for the main workload")
     args = ap.parse_args()
@@ -706,7 +743,7 @@ def main():
     peaks = load_peaks()
     try:
         if args.ep:
-            res = run_ep(cfg, args.steps, args.warmup, rank, world, local, peaks)
+            res = run_ep(cfg, args.steps, args.warmup, rank, world, local, peaks, args.ep_exchange)
         else:
             res = run_gpu(cfg, args.steps, args.warmup, rank, world, local, peaks, grouped_kind=args.grouped_kind)
         secondary = None
