@@ -124,15 +124,17 @@ bool make_map_e2m1(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) 
     return r == CUDA_SUCCESS;
 }
 
-// NVFP4 token scale chunks, planar [chunks][rows][16] bytes; a box is 4 chunks x 32 rows x 16 bytes (the
-// four 512-byte scale atoms of one 256-element stage, first 32 rows).
+// NVFP4 token scale chunks, planar [chunks][rows][16] bytes, seen as 8-byte elements [chunks][2 * rows]: a
+// box is 4 chunks x 64 elements, the four 512-byte scale atoms of one 256-element stage (32 rows from the x
+// coordinate 2 * first row).  The copy engine's cost grows with the rows of a box: 4 rows of 512 bytes here
+// against 128 rows of 16 bytes for a [chunks][rows][16] box of the same bytes.
 bool make_map_nv_sf(CUtensorMap* m, const void* base, uint64_t rows, uint64_t chunks) {
     if (!load_encode() || rows == 0) return false;
-    cuuint64_t dims[3] = {16, rows, chunks};
-    cuuint64_t strides[2] = {16, rows * 16};
-    cuuint32_t box[3] = {16, 32, 4};
-    cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+    cuuint64_t dims[2] = {2 * rows, chunks};
+    cuuint64_t strides[1] = {rows * 16};
+    cuuint32_t box[2] = {64, 4};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 2, const_cast<void*>(base), dims, strides, box, estr,
                                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -561,7 +563,7 @@ void launch_mx(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xs
 template <int EPI, bool QOUT>
 void launch_nv(const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf, const NvArgs& a, int grid,
                cudaStream_t s) {
-    launch(tc_swap_nv_kernel<EPI, QOUT>, grid, 192, NvCfg<EPI>::SMEM_BYTES, s, w, x, xsf, a);
+    launch(tc_swap_nv_kernel<EPI, QOUT>, grid, NvCfg<EPI>::THREADS, NvCfg<EPI>::SMEM_BYTES, s, w, x, xsf, a);
 }
 void launch_nv_phase(bool up, int epi, const CUtensorMap& w, const CUtensorMap& x, const CUtensorMap& xsf,
                      const NvArgs& a, int grid, cudaStream_t s) {

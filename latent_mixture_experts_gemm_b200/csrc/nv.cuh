@@ -25,8 +25,9 @@
 // Token-operand layout (workspace): codes [rows, K/2] bytes; scales planar
 // [K/64][rows][16] bytes: chunk c of row r holds, in its first four bytes, the
 // scales of the row's elements 64c .. 64c+63 (the other twelve are not read).
-// A 3-D copy of 4 chunks x 32 rows lands as the four 512-byte atoms of one
-// 256-element stage (the first 32 rows of each 128-row atom).
+// Seen as 8-byte elements [K/64][2 * rows], one copy of 4 chunks x 64 elements
+// (four 512-byte rows) lands as the four 512-byte atoms of one 256-element
+// stage (the first 32 rows of each 128-row atom).
 #pragma once
 #include "mx.cuh"
 
@@ -199,29 +200,35 @@ struct NvCfg {
     // tile a at column (c * NA + a) * NT
     static constexpr int CHAINS = 2;
     static constexpr int ACC_COLS = CHAINS * NA * NT;
-    // TMEM scale columns: a ring of SF_SLOTS slots after the two accumulator sets; a slot holds a stage's
-    // scales, 4 columns per MMA: weight tile 0's MMAs, then tile 1's (gated), then the token rows'
+    // TMEM scale columns: one slot per shared-memory stage after the two accumulator sets; a slot holds a
+    // stage's scales, 4 columns per MMA: weight tile 0's MMAs, then tile 1's (gated), then the token rows'
+    // (the order of the atoms in the stage's shared memory)
     static constexpr int SF_COL = 2 * ACC_COLS;
     static constexpr int SF_SLOT = 4 * MMAS * (NA + 1);
-    static constexpr int SF_SLOTS = 4;
+    static constexpr int SF_SLOTS = STAGES;
     static constexpr int TMEM_COLS = SF_COL + SF_SLOTS * SF_SLOT <= 256 ? 256 : 512;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+    // warps: 0 TMA, 1 MMA, 2-5 epilogue, 6-9 scales (one per TMEM lane quadrant)
+    static constexpr int THREADS = 320;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 512;
     static_assert(SF_COL % 4 == 0 && SF_SLOT % 4 == 0 && SF_COL + SF_SLOTS * SF_SLOT <= TMEM_COLS, "scale columns");
     static_assert(STAGE_BYTES % 1024 == 0 && SMEM_BYTES <= 232448, "shared memory");
+    static_assert(MMAS == 4, "the scale warps store four atoms (16 columns) at a time");
 };
 
 // Weight-streaming GEMM with NVFP4 operands for experts that received <= 32
 // rows (D^T[128 x 32] = W_tile * X^T, the weight rows as the M = 128 operand).
 // Per stage of 256 K elements: the weight tile(s) and the token tile by TMA,
 // the weight scale atoms (one per MMA) by a bulk copy, and the token scale
-// atoms by one 3-D TMA copy.  The MMA thread moves each stage's atoms into a
-// ring of TMEM slots with tcgen05.cp and issues four K = 64 MMAs, alternating
-// between two accumulators.  The epilogue multiplies by the expert matrix's g;
-// with QOUT it applies the activation, stores it in bf16 precision and
-// re-encodes it in NVFP4 (g = 1): a 16-column block of a token row is held by
-// 16 lanes of a warp.  Otherwise it writes bf16.
+// atoms by one TMA copy of four 512-byte rows.  Four scale warps, one per TMEM
+// lane quadrant, store each stage's atoms into the stage's TMEM slot
+// (tcgen05.st, outside the tensor-core pipe: eight tcgen05.cp per stage in
+// that pipe measured 12 us slower per launch); the MMA thread issues four
+// K = 64 MMAs, alternating between two accumulators.  The epilogue multiplies
+// by the expert matrix's g; with QOUT it applies the activation, stores it in
+// bf16 precision and re-encodes it in NVFP4 (g = 1): a 16-column block of a
+// token row is held by 16 lanes of a warp.  Otherwise it writes bf16.
 template <int EPI, bool QOUT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(NvCfg<EPI>::THREADS, 1)
     tc_swap_nv_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmXsf, const NvArgs args) {
     pdl_begin();
@@ -234,7 +241,8 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* tfull = empty + C::STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* mma_done = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+    uint64_t* sfull = mma_done + 1;  // a stage's scales are in its TMEM slot (one arrival per scale warp)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sfull + C::STAGES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -245,6 +253,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&sfull[s], 4);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull[b], 1);
@@ -299,7 +308,7 @@ __global__ void __launch_bounds__(192, 1)
                     if (C::NA == 2)
                         bulk_load(st + C::OFF_SFA + STAGE_SF, sfa1 + static_cast<size_t>(kb) * STAGE_SF, STAGE_SF,
                                   &full[s]);
-                    tma_load_3d(st + C::OFF_SFB, &tmXsf, &full[s], 0, e.y, kb * C::MMAS);
+                    tma_load_2d(st + C::OFF_SFB, &tmXsf, &full[s], 2 * e.y, kb * C::MMAS);
                     issued[s] = true;
                     last_parity[s] = ph;
                 }
@@ -331,18 +340,14 @@ __global__ void __launch_bounds__(192, 1)
                         ok = false;
                         break;
                     }
+                    if (!mbar_wait_bounded(&sfull[s], ph, abort_flag, args.err, args.timeout_ns)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
                     const uint32_t st = smem_u32(smem + s * C::STAGE_BYTES);
-                    const uint32_t slot = tmem_base + C::SF_COL + (kc % C::SF_SLOTS) * C::SF_SLOT;
+                    const uint32_t slot = tmem_base + C::SF_COL + s * C::SF_SLOT;
                     const uint32_t sf_a1 = slot + 4 * C::MMAS, sf_b = slot + 4 * C::MMAS * C::NA;
-#pragma unroll
-                    for (int kk = 0; kk < C::MMAS; ++kk) {
-                        tmem_cp_32x128b_x4(slot + 4 * kk, umma_desc_plain(st + C::OFF_SFA + kk * C::ATOM, 128));
-                        if (C::NA == 2)
-                            tmem_cp_32x128b_x4(sf_a1 + 4 * kk,
-                                               umma_desc_plain(st + C::OFF_SFA + STAGE_SF + kk * C::ATOM, 128));
-                        tmem_cp_32x128b_x4(sf_b + 4 * kk, umma_desc_plain(st + C::OFF_SFB + kk * C::ATOM, 128));
-                    }
                     const uint64_t a0 = umma_desc_sw128(st);
                     const uint64_t a1 = umma_desc_sw128(st + C::A_BYTES);
                     const uint64_t bx = umma_desc_sw128(st + C::OFF_B);
@@ -363,6 +368,39 @@ __global__ void __launch_bounds__(192, 1)
             int no_abort = 0;
             const uint64_t drain = args.timeout_ns > 200000000ull ? args.timeout_ns : 200000000ull;
             mbar_wait_bounded(mma_done, 0, &no_abort, args.err, drain);
+        }
+    } else if (warp >= 6) {
+        // ---------------------------------------------------- scale warps
+        // The stage's (NA + 1) * MMAS atoms lie in shared memory in the order of the slot's columns (weight
+        // tile 0's, tile 1's, the token rows'), 4 columns each: each lane stores its row of every atom, in
+        // its warp's lane quadrant, four atoms per store.
+        const uint32_t quadrant = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        uint32_t kc = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+            for (int kb = 0; kb < nkb; ++kb, ++kc) {
+                const int s = kc % C::STAGES;
+                const uint32_t ph = (kc / C::STAGES) & 1;
+                // every lane observes the copy's completion before it reads the stage's shared memory
+                const bool got = mbar_wait_bounded(&full[s], ph, abort_flag, args.err, args.timeout_ns);
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* atoms = smem + s * C::STAGE_BYTES + C::OFF_SFA;
+                const uint32_t taddr = tmem_base + quadrant + C::SF_COL + s * C::SF_SLOT;
+#pragma unroll
+                for (int g = 0; g < C::NA + 1; ++g) {
+                    uint32_t r[16];
+#pragma unroll
+                    for (int kk = 0; kk < C::MMAS; ++kk) atom_row(atoms + (g * C::MMAS + kk) * C::ATOM, lane, r + 4 * kk);
+                    tmem_st_32x32b_x16(taddr + 16 * g, r);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sfull[s]);
+            }
         }
     } else {
         // ---------------------------------------------------- epilogue: thread = output column

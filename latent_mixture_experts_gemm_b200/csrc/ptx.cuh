@@ -293,6 +293,39 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Stores from registers: thread i of the warp writes lane (quadrant base + i), consecutive 32-bit columns
+// from taddr.  Complete (visible to the tensor cores after a thread sync) once tmem_st_wait returns.
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, const uint32_t (&r)[4]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// One 512-byte scale atom (32 rows x 16 bytes in shared memory) into 4 TMEM columns of this warp's 32 lanes:
+// lane i gets row i, bytes 4j..4j+3 in column j.  Run by the four warps of the four lane quadrants, it leaves
+// the layout tcgen05.cp.32x128b.warpx4 leaves, without passing through the tensor-core pipe.
+__device__ __forceinline__ void atom_row(const uint8_t* atom, int lane, uint32_t* dst4) {
+    const uint4 v = *reinterpret_cast<const uint4*>(atom + lane * 16);
+    dst4[0] = v.x;
+    dst4[1] = v.y;
+    dst4[2] = v.z;
+    dst4[3] = v.w;
+}
+
 // ---------------------------------------------------------------- CTA pairs (cluster of 2, cta_group::2)
 // Rank of this CTA in its cluster.
 __device__ __forceinline__ uint32_t cluster_ctarank() {
