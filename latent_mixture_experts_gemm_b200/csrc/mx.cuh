@@ -220,7 +220,8 @@ template <int EPI, bool W4, bool QOUT>
 __global__ void __launch_bounds__(192, 1)
     tc_swap_mx_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                       const __grid_constant__ CUtensorMap tmXsf, const MxArgs args) {
-    pdl_begin();
+    // The work list and the weights (codes and scales) are read before the wait for the previous kernel (see
+    // pdl_wait); the token tiles, token scales and every output after it.
     using C = MxCfg<EPI, W4>;
     constexpr int NT = C::NT;
     extern __shared__ uint8_t smem_raw[];
@@ -235,7 +236,10 @@ __global__ void __launch_bounds__(192, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = *args.count * args.n_wtiles;
-    if (static_cast<int>(blockIdx.x) >= ntiles) return;
+    if (static_cast<int>(blockIdx.x) >= ntiles) {
+        pdl_begin();
+        return;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -262,10 +266,31 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int nkb = args.K / C::BK;
+    if (!(warp == 0 && lane == 0)) pdl_begin();
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
+            // The first STAGES stages' weight tiles and weight scales are requested before the wait for the
+            // previous kernel (every slot is free then), their token tiles and token scales after it.
+            uint32_t pre = 0;
+            for (int t = blockIdx.x; t < ntiles && pre < C::STAGES; t += gridDim.x) {
+                const int4 e = args.list[t / args.n_wtiles];
+                const int wrow = e.x * args.w_rows_per_expert + (t % args.n_wtiles) * 128;
+                const uint8_t* sfa0 = args.w_sf + static_cast<size_t>(wrow / 128) * nkb * C::SF_BYTES;
+                const uint8_t* sfa1 = args.w_sf + static_cast<size_t>((wrow + args.up_offset) / 128) * nkb * C::SF_BYTES;
+                for (int kb = 0; kb < nkb && pre < C::STAGES; ++kb, ++pre) {
+                    uint8_t* st = smem + pre * C::STAGE_BYTES;
+                    mbar_arrive_expect_tx(&full[pre], C::TX_BYTES);
+                    tma_load_2d(st, &tmW, &full[pre], kb * C::BK, wrow);
+                    if (C::NA == 2) tma_load_2d(st + C::A_BYTES, &tmW, &full[pre], kb * C::BK, wrow + args.up_offset);
+                    bulk_load(st + C::OFF_SFA, sfa0 + static_cast<size_t>(kb) * C::SF_BYTES, C::SF_BYTES, &full[pre]);
+                    if (C::NA == 2)
+                        bulk_load(st + C::OFF_SFA + C::SF_BYTES, sfa1 + static_cast<size_t>(kb) * C::SF_BYTES,
+                                  C::SF_BYTES, &full[pre]);
+                }
+            }
+            pdl_begin();
             uint32_t kc = 0;
             uint32_t last_parity[C::STAGES];
             bool issued[C::STAGES];
@@ -279,19 +304,23 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kb = 0; kb < nkb; ++kb, ++kc) {
                     const int s = kc % C::STAGES;
                     const uint32_t ph = (kc / C::STAGES) & 1;
-                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.err, args.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
                     uint8_t* st = smem + s * C::STAGE_BYTES;
-                    mbar_arrive_expect_tx(&full[s], C::TX_BYTES);
-                    tma_load_2d(st, &tmW, &full[s], kb * C::BK, wrow);
-                    if (C::NA == 2) tma_load_2d(st + C::A_BYTES, &tmW, &full[s], kb * C::BK, wrow + args.up_offset);
+                    if (kc >= pre) {
+                        if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.err, args.timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[s], C::TX_BYTES);
+                        tma_load_2d(st, &tmW, &full[s], kb * C::BK, wrow);
+                        if (C::NA == 2)
+                            tma_load_2d(st + C::A_BYTES, &tmW, &full[s], kb * C::BK, wrow + args.up_offset);
+                        bulk_load(st + C::OFF_SFA, sfa0 + static_cast<size_t>(kb) * C::SF_BYTES, C::SF_BYTES,
+                                  &full[s]);
+                        if (C::NA == 2)
+                            bulk_load(st + C::OFF_SFA + C::SF_BYTES, sfa1 + static_cast<size_t>(kb) * C::SF_BYTES,
+                                      C::SF_BYTES, &full[s]);
+                    }
                     tma_load_2d(st + C::OFF_B, &tmX, &full[s], kb * C::BK, e.y);
-                    bulk_load(st + C::OFF_SFA, sfa0 + static_cast<size_t>(kb) * C::SF_BYTES, C::SF_BYTES, &full[s]);
-                    if (C::NA == 2)
-                        bulk_load(st + C::OFF_SFA + C::SF_BYTES, sfa1 + static_cast<size_t>(kb) * C::SF_BYTES,
-                                  C::SF_BYTES, &full[s]);
                     tma_load_2d(st + C::OFF_SFB, &tmXsf, &full[s], kb * 16, e.y);
                     issued[s] = true;
                     last_parity[s] = ph;

@@ -19,15 +19,24 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// Programmatic dependent launch.  Every kernel of the layer starts with
-// pdl_begin(): it lets the next kernel in the stream be launched now (its CTAs
-// are placed as SMs free up and run up to their own wait), then waits until the
-// previous kernel has completed and its memory is visible.  Every CTA waits
-// before it can exit, so completion stays ordered along the stream.  Without
-// the launch attribute both instructions are no-ops.
+// Programmatic dependent launch.  pdl_wait() waits until the previous kernel in
+// the stream has completed and its memory is visible; pdl_trigger() lets the
+// next kernel be launched (its CTAs are placed as SMs free up and run up to
+// their own wait).  Every CTA of every kernel of the layer waits before it
+// triggers and before it exits, so:
+//  * completion stays ordered along the stream;
+//  * while a kernel runs, the kernel two places before it has completed, so
+//    its outputs may be read before the wait.  The weight-streaming kernels use
+//    this: their work lists come from the dispatch, always two or more launches
+//    earlier, and their weights from no kernel, so they request their first
+//    weight tiles while the previous kernel drains.
+// Without the launch attribute both instructions are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// The common case: wait, then trigger, first thing in the kernel.
 __device__ __forceinline__ void pdl_begin() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    pdl_wait();
+    pdl_trigger();
 }
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {

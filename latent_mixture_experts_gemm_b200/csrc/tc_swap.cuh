@@ -115,7 +115,8 @@ __global__ void __launch_bounds__(192, 1)
     tc_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                    const __grid_constant__ CUtensorMap tmW2, const __grid_constant__ CUtensorMap tmX2,
                    const SwapArgs args) {
-    pdl_begin();
+    // No pdl_begin() here: the work list (from the dispatch, two or more launches back) and the weights are
+    // read before the wait for the previous kernel; the token tiles and every output after it.
     using C = SwapCfg<NT, EPI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -129,7 +130,10 @@ __global__ void __launch_bounds__(192, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ntiles = swap_total(args);
-    if (static_cast<int>(blockIdx.x) >= ntiles) return;
+    if (static_cast<int>(blockIdx.x) >= ntiles) {
+        pdl_begin();
+        return;
+    }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
@@ -157,10 +161,28 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int nkb = args.K / C::BK;
+    if (!(warp == 0 && lane == 0)) pdl_begin();
 
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------ TMA producer
+            // The first STAGES stages' weight tiles are requested before the wait for the previous kernel
+            // (every slot is free then), their token tiles after it; each stage's barrier expects both.
+            uint32_t pre = 0;
+            for (int t = blockIdx.x; t < ntiles && pre < C::STAGES; t += gridDim.x) {
+                SwapJob j;
+                swap_job(args, t, nkb, j);
+                const CUtensorMap* wmap = j.second ? &tmW2 : &tmW;
+                for (int kb = j.kb0; kb < j.kb1 && pre < C::STAGES; ++kb, ++pre) {
+                    uint8_t* st = smem + pre * C::STAGE_BYTES;
+                    const bool x2 = args.k_wrap > 0 && kb * C::BK >= args.k_wrap;
+                    const int kx = x2 ? kb * C::BK - args.k_wrap : kb * C::BK;
+                    mbar_arrive_expect_tx(&full[pre], C::STAGE_BYTES);
+                    tma_load_2d(st, wmap, &full[pre], kx, j.wrow);
+                    if (C::NA == 2) tma_load_2d(st + C::A_BYTES, wmap, &full[pre], kx, j.wrow + args.up_offset);
+                }
+            }
+            pdl_begin();
             uint32_t kc = 0;
             uint32_t last_parity[C::STAGES];
             bool issued[C::STAGES];
@@ -173,16 +195,18 @@ __global__ void __launch_bounds__(192, 1)
                 for (int kb = j.kb0; kb < j.kb1; ++kb, ++kc) {
                     const int s = kc % C::STAGES;
                     const uint32_t ph = (kc / C::STAGES) & 1;
-                    if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.err, args.timeout_ns)) {
-                        ok = false;
-                        break;
-                    }
                     uint8_t* st = smem + s * C::STAGE_BYTES;
                     const bool x2 = args.k_wrap > 0 && kb * C::BK >= args.k_wrap;
                     const int kx = x2 ? kb * C::BK - args.k_wrap : kb * C::BK;
-                    mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
-                    tma_load_2d(st, wmap, &full[s], kx, j.wrow);
-                    if (C::NA == 2) tma_load_2d(st + C::A_BYTES, wmap, &full[s], kx, j.wrow + args.up_offset);
+                    if (kc >= pre) {
+                        if (!mbar_wait_bounded(&empty[s], ph ^ 1, abort_flag, args.err, args.timeout_ns)) {
+                            ok = false;
+                            break;
+                        }
+                        mbar_arrive_expect_tx(&full[s], C::STAGE_BYTES);
+                        tma_load_2d(st, wmap, &full[s], kx, j.wrow);
+                        if (C::NA == 2) tma_load_2d(st + C::A_BYTES, wmap, &full[s], kx, j.wrow + args.up_offset);
+                    }
                     tma_load_2d(st + C::NA * C::A_BYTES, x2 ? &tmX2 : &tmX, &full[s], kx, j.e.y);
                     issued[s] = true;
                     last_parity[s] = ph;
