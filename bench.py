@@ -232,9 +232,9 @@ EXPERT_RATE = {0: 1.0, 1: 2.0, 2: 2.0, 3: 4.0}
 #: 4.2 / 4.5 MB (up / down).  A kernel that changes drops out of this table until it is captured again.
 NCU_TRAFFIC = {
     ("nemotron_decode", "expert_up_stream"): 797.8e6,
-    ("nemotron_prefill", "expert_up_gemm"): 1794.3e6,
-    ("nemotron_decode_nvfp4", "expert_up_stream"): 229.6e6,
-    ("nemotron_decode_nvfp4", "expert_down_stream"): 230.1e6,
+    ("nemotron_prefill", "expert_up_gemm"): 1792.0e6,
+    ("nemotron_decode_nvfp4", "expert_up_stream"): 229.7e6,
+    ("nemotron_decode_nvfp4", "expert_down_stream"): 230.0e6,
 }
 
 
