@@ -225,16 +225,25 @@ ACT_BYTES = {0: 2.0, 1: 1.0 + 1.0 / 32, 2: 1.0 + 1.0 / 32, 3: 0.5 + 1.0 / 16}
 EXPERT_RATE = {0: 1.0, 1: 2.0, 2: 2.0, 3: 4.0}
 
 
-#: DRAM bytes (read + write) per launch of a dominant kernel, from one ncu capture of that kernel as it is now:
-#: the expert up stream of the Nemotron-like decode read 796.4 MB and wrote 1.4 MB per launch (mean of 9
-#: launches); the grouped expert up GEMM of the Nemotron-like prefill read 1442.9 MB and wrote 351.3 MB (one
-#: launch at the full 8192 tokens); the NVFP4 decode's expert streams read 224.3 / 224.2 MB and wrote
-#: 4.2 / 4.5 MB (up / down).  A kernel that changes drops out of this table until it is captured again.
+#: DRAM bytes (read + write) per launch of each workload's expert phases, from ncu captures of the kernels as
+#: they are now (dram__bytes_read.sum + dram__bytes_write.sum): decode streams as the mean over the captured
+#: steps' launches, prefill grouped GEMMs from one launch each at the full token count.  A kernel that changes
+#: drops out of this table until it is captured again.
 NCU_TRAFFIC = {
     ("nemotron_decode", "expert_up_stream"): 797.8e6,
-    ("nemotron_prefill", "expert_up_gemm"): 1792.0e6,
+    ("nemotron_decode", "expert_down_stream"): 797.8e6,
+    ("nemotron_prefill", "expert_up_gemm"): 1792.1e6,
+    ("nemotron_prefill", "expert_down_gemm"): 1788.5e6,
+    ("std_decode", "expert_up_stream"): 836.5e6,
+    ("std_decode", "expert_down_stream"): 839.2e6,
+    ("std_prefill", "expert_up_gemm"): 1662.7e6,
+    ("std_prefill", "expert_down_gemm"): 1554.5e6,
+    ("kimi_skew", "expert_up_gemm"): 1237.9e6,
+    ("kimi_skew", "expert_down_gemm"): 772.3e6,
     ("nemotron_decode_nvfp4", "expert_up_stream"): 229.7e6,
     ("nemotron_decode_nvfp4", "expert_down_stream"): 230.0e6,
+    ("nemotron_decode_mxfp4", "expert_up_stream"): 214.2e6,
+    ("nemotron_decode_mxfp4", "expert_down_stream"): 214.4e6,
 }
 
 
