@@ -712,7 +712,7 @@ def workload_config(cfg):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0, help="override the workload's token count (profiling runs)")
@@ -760,8 +760,9 @@ def main():
             secondary = []
             for name in [w for w in args.secondary.split(",") if w and w != args.workload]:
                 sc = synth.WORKLOADS[name]
-                # at least 20 steps for every workload: decode batches take well under a millisecond each
-                s_steps = max(20, min(args.steps, 50)) if sc.tokens <= 32 else max(3, min(args.steps, 20))
+                # decode batches take well under a millisecond each: at least 100 timed steps, so that the
+                # clock sampler sees the region and a single slow step moves the mean little
+                s_steps = max(100, min(args.steps, 400)) if sc.tokens <= 32 else max(3, min(args.steps, 20))
                 r2 = run_gpu(sc, s_steps, args.warmup, rank, world, local, peaks, with_e2e=False)
                 secondary.append({"workload": sc.name, "config": workload_config(sc), "dtype": compute_dtype(sc),
                                   "steps": s_steps,
