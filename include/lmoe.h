@@ -198,9 +198,14 @@ LMOE_API int lmoe_forward(lmoe_handle *h, const void *x, void *y, int32_t T, voi
 
 /*
  * The same forward on HOST buffers: copies x_host [T, d] into the workspace,
- * runs the layer and copies y back to y_host [T, d], all on `stream`.  The
- * host buffers should be pinned for the copies to be asynchronous; the caller
- * synchronises the stream before reading y_host.
+ * runs the layer and copies y back to y_host [T, d].  The input copy runs on a
+ * stream of the handle's own, into one of two workspace input buffers taken in
+ * turn, and `stream` waits for it; the forward and the output copy run on
+ * `stream`.  So calls issued back to back overlap each call's input copy with
+ * the previous call's forward.  While `stream` is being captured, everything
+ * runs on `stream`.  The host buffers should be pinned for the copies to be
+ * asynchronous; the caller synchronises `stream` before reading y_host or
+ * reusing x_host (that covers the input copy too).
  */
 LMOE_API int lmoe_forward_host(lmoe_handle *h, const void *x_host, void *y_host, int32_t T, void *stream);
 

@@ -190,7 +190,7 @@ int n_local_experts(const lmoe_config& c) { return c.n_experts / ep_ranks(c); }
 struct Plan {
     size_t hdr, logits, z, zlo, idx, w, bitmap, prefix, counts, offsets, perm, inv, mt_list, pt_list, small_list, rows,
         hbuf, yl,
-        partial, hs, s2, partial2, rows4, rows_sf4, h4, h_sf4, rows8, rows_sf, h8, h_sf, xin, yout, ep_map, ep_src,
+        partial, hs, s2, partial2, rows4, rows_sf4, h4, h_sf4, rows8, rows_sf, h8, h_sf, xin, xin2, yout, ep_map, ep_src,
         ep_dst, ep_counts,
         ep_offsets, total;
     size_t rows_cap;  // rows of the expert-side buffers: a forward's slots, or the most an experts stage receives
@@ -260,6 +260,7 @@ Plan make_plan(const lmoe_config& c) {
         p.h_sf = take(R * mx_ld_sf(static_cast<int>(m)));
     }
     p.xin = take(T * d * 2);
+    p.xin2 = take(T * d * 2);  // the host-buffer forward alternates between two input buffers
     p.yout = take(T * d * 2);
     // expert-parallel experts stage: received row -> expert-major row, segment tables, local counts / offsets
     p.ep_map = take(p.ep_cap * 4);
@@ -621,7 +622,7 @@ struct lmoe_handle {
     // block-scaled experts: weight codes (128 x 128 boxes) and the MXFP8 token operands with their scales
     CUtensorMap w1q{}, w2q{}, rows8{}, rows_sf{}, h8{}, h_sf{};
     // NVFP4 experts: packed weight codes (128 x 128-byte boxes), token codes (32 x 128-byte boxes) and the
-    // token scale chunks (4 chunks x 32 rows x 16 bytes)
+    // token scale chunks (4 rows of 512 bytes: one stage's four atoms)
     CUtensorMap w1n{}, w2n{}, rows4{}, rows_sf4{}, h4{}, h_sf4{};
     // TMA store maps of bf16 GEMM outputs (32-row x 64-column boxes): hidden rows, expert outputs, z
     CUtensorMap o_h{}, o_rows{}, o_z{};
@@ -631,6 +632,12 @@ struct lmoe_handle {
     bool group_pair_ok = false;  // the shapes allow it: m (gated: m / 2 per pair tile) and latent in 256-row tiles
     int group_pair = 0;          // 1: grouped expert GEMMs on CTA pairs; 0 (default): single-CTA 128-row tiles
     cudaStream_t side = nullptr;     // the shared expert runs here, concurrently with the routed path
+    // lmoe_forward_host: the input copy runs on `hcopy` into one of two input buffers, so that the copy of
+    // one call overlaps the forward of the one before; ev_in[b] marks buffer b's copy done, ev_used[b] the
+    // forward that read it done
+    cudaStream_t hcopy = nullptr;
+    cudaEvent_t ev_in[2] = {nullptr, nullptr}, ev_used[2] = {nullptr, nullptr};
+    uint64_t host_calls = 0;
     // Forwards launched as a CUDA graph: each call captures its launches on `cap` and replays them on the
     // caller's stream from an executable graph, updated in place.  A few executable graphs are kept, one per
     // launch sequence (token counts that change the kernels used), least recently used first out.
@@ -1487,6 +1494,21 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, void* stream
     return run_forward(h, x, y, T, s, dbg);
 }
 
+// The copy stream and events of the host-buffer forward, made on its first use.
+bool host_copy_ready(lmoe_handle* h) {
+    if (h->hcopy != nullptr) return true;
+    cudaStream_t cs = nullptr;
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return false;
+    for (int b = 0; b < 2; ++b)
+        if (cudaEventCreateWithFlags(&h->ev_in[b], cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&h->ev_used[b], cudaEventDisableTiming) != cudaSuccess) {
+            cudaStreamDestroy(cs);
+            return false;
+        }
+    h->hcopy = cs;
+    return true;
+}
+
 int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t T, void* stream) {
     if (h == nullptr || h->c.ep_size > 1) return LMOE_ERR_INVALID_ARG;
     if (T < 0 || T > h->c.max_tokens) return LMOE_ERR_TOO_MANY_TOKENS;
@@ -1494,9 +1516,31 @@ int lmoe_forward_host(lmoe_handle* h, const void* x_host, void* y_host, int32_t 
     if (x_host == nullptr || y_host == nullptr) return LMOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const size_t bytes = static_cast<size_t>(T) * h->c.d * 2;
-    void* xin = h->at<void>(h->p.xin);
     void* yout = h->at<void>(h->p.yout);
-    if (cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return LMOE_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(s, &cap) != cudaSuccess) return LMOE_ERR_CUDA;
+    void* xin = h->at<void>(h->p.xin);
+    if (cap != cudaStreamCaptureStatusNone || !host_copy_ready(h)) {
+        // captured by the caller (or no copy stream): everything in order on `stream`
+        if (cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) return LMOE_ERR_CUDA;
+    } else {
+        // The input copy goes on the handle's copy stream, into the buffer the forward before last read (its
+        // forward has finished with it once ev_used fires); `stream` waits for the copy.  A caller that issues
+        // calls back to back thus has each call's copy overlap the previous call's forward.
+        const int b = static_cast<int>(h->host_calls & 1);
+        xin = h->at<void>(b ? h->p.xin2 : h->p.xin);
+        if (cudaStreamWaitEvent(h->hcopy, h->ev_used[b], 0) != cudaSuccess ||
+            cudaMemcpyAsync(xin, x_host, bytes, cudaMemcpyHostToDevice, h->hcopy) != cudaSuccess ||
+            cudaEventRecord(h->ev_in[b], h->hcopy) != cudaSuccess || cudaStreamWaitEvent(s, h->ev_in[b], 0) != cudaSuccess)
+            return LMOE_ERR_CUDA;
+        const int rc = graph_forward_ok(h, s, nullptr) ? forward_graph(h, xin, yout, T, s)
+                                                       : run_forward(h, xin, yout, T, s, nullptr);
+        if (rc != LMOE_OK) return rc;
+        if (cudaEventRecord(h->ev_used[b], s) != cudaSuccess) return LMOE_ERR_CUDA;
+        ++h->host_calls;
+        if (cudaMemcpyAsync(y_host, yout, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return LMOE_ERR_CUDA;
+        return LMOE_OK;
+    }
     const int rc = graph_forward_ok(h, s, nullptr) ? forward_graph(h, xin, yout, T, s) : run_forward(h, xin, yout, T, s, nullptr);
     if (rc != LMOE_OK) return rc;
     if (cudaMemcpyAsync(y_host, yout, bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess) return LMOE_ERR_CUDA;
@@ -1748,6 +1792,11 @@ void lmoe_destroy(lmoe_handle* h) {
     if (h->ev_fork) cudaEventDestroy(h->ev_fork);
     if (h->ev_join) cudaEventDestroy(h->ev_join);
     if (h->side) cudaStreamDestroy(h->side);
+    for (int b = 0; b < 2; ++b) {
+        if (h->ev_in[b]) cudaEventDestroy(h->ev_in[b]);
+        if (h->ev_used[b]) cudaEventDestroy(h->ev_used[b]);
+    }
+    if (h->hcopy) cudaStreamDestroy(h->hcopy);
     for (auto& ge : h->graphs)
         if (ge.exec) cudaGraphExecDestroy(ge.exec);  // one still in flight is freed when it completes
     if (h->cap) cudaStreamDestroy(h->cap);

@@ -209,6 +209,31 @@ def test_deterministic_and_host_entry_point_agree():
         mod.close()
 
 
+@pytest.mark.parametrize("cfg", [MEDIUM, synth.WORKLOADS["tiny"].with_(tokens=32, seed=12)], ids=["medium", "tiny_decode"])
+def test_host_entry_point_back_to_back(cfg):
+    """Host-buffer forwards issued back to back, with no wait between them: each call's input copy runs on the
+    handle's copy stream into one of two buffers while the previous call's forward may still run.  Every
+    output must equal the device forward of its own input, bit for bit."""
+    layer = synth.make_layer(cfg)
+    mod = lmoe.LatentMoE(cfg, layer, max_tokens=cfg.tokens)
+    try:
+        sizes = [cfg.tokens, 7, cfg.tokens, 1, cfg.tokens // 2 + 1, cfg.tokens]
+        xs = [synth.make_tokens(cfg, T, seed=500 + i) for i, T in enumerate(sizes)]
+        want = [mod.forward(x.cuda()).cpu() for x in xs]
+        torch.cuda.synchronize()
+        xh = [x.pin_memory() for x in xs]
+        yh = [torch.full_like(x, float("nan")).pin_memory() for x in xs]
+        for rep in range(2):
+            for i in range(len(xs)):
+                mod.forward_host(xh[i], yh[i])
+            torch.cuda.synchronize()
+            for i in range(len(xs)):
+                assert torch.equal(yh[i], want[i]), f"call {i} of round {rep}"
+        assert mod.last_error() == 0
+    finally:
+        mod.close()
+
+
 def test_smaller_batches_on_one_handle():
     """A handle sized for many tokens serves smaller (ragged, single, empty) batches."""
     cfg = MEDIUM
