@@ -567,6 +567,41 @@ static __global__ void __launch_bounds__(256) dispatch_scatter_kernel(const int3
     }
 }
 
+// One warp per token (SCATTER_WARPS per block): the token's feature row is read once into shared memory, and
+// each of its slots is placed (perm / inv) and, for FFN experts, receives the row at its sorted position by
+// one bulk copy from shared memory, so the row is read from memory once instead of once per slot.  The same
+// positions as dispatch_scatter_kernel.  Dynamic shared memory: SCATTER_WARPS * fdim * 2 bytes.
+constexpr int SCATTER_WARPS = 4;
+static __global__ void __launch_bounds__(32 * SCATTER_WARPS) dispatch_scatter_rows_kernel(
+    const int32_t* __restrict__ idx, int T, int K, int n_tot, int n_ffn, const uint32_t* __restrict__ bitmap,
+    const uint32_t* __restrict__ prefix, const int* __restrict__ offsets, const __nv_bfloat16* __restrict__ feat,
+    int ld_feat, int fdim, __nv_bfloat16* __restrict__ rows_out, int ld_rows, int32_t* __restrict__ perm,
+    int32_t* __restrict__ inv) {
+    pdl_begin();
+    extern __shared__ uint4 srow[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int t = blockIdx.x * SCATTER_WARPS + warp;
+    if (t >= T) return;
+    uint4* row = srow + static_cast<size_t>(warp) * (fdim / 8);
+    const uint4* src = reinterpret_cast<const uint4*>(feat + static_cast<size_t>(t) * ld_feat);
+    for (int c = lane; c < fdim / 8; c += 32) row[c] = src[c];
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the row, visible to the bulk copies
+    __syncwarp();
+    const int w = t >> 5, b = t & 31;
+    for (int k = lane; k < K; k += 32) {
+        const long i = static_cast<long>(t) * K + k;
+        const int e = idx[i];
+        if (e < 0 || e >= n_tot) continue;  // flagged by the bitmap kernel
+        const size_t cell = static_cast<size_t>(w) * n_tot + e;
+        const int pos = offsets[e] + static_cast<int>(prefix[cell]) + __popc(bitmap[cell] & ((1u << b) - 1u));
+        perm[pos] = static_cast<int32_t>(i);
+        inv[i] = pos;
+        if (e < n_ffn) bulk_store(rows_out + static_cast<size_t>(pos) * ld_rows, row, static_cast<uint32_t>(fdim) * 2);
+    }
+    bulk_commit();
+    bulk_wait_all();  // the copies have read the shared row and written the rows before the warp exits
+}
+
 // Experts with at most this many rows take the weight-streaming (swap-AB) GEMM.
 constexpr int SMALL_MAX = 32;
 
