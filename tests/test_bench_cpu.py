@@ -73,3 +73,18 @@ def test_block_scaled_expert_gemm_takes_its_own_dtype_peak():
     peaks = {"hbm_gbs": 6540.2, "bf16_tflops": 1645.9, "source": "measured"}
     roof, _, _ = bench.rooflines(cfg, stats, cfg.tokens, {"expert_up_stream": (0.2, 1)}, peaks, 1.0)
     assert roof["bound"] == "tensor" and roof["peak"] == pytest.approx(4 * 1645.9)
+
+
+def test_every_benchmarked_workload_has_traffic_for_its_expert_phases():
+    """Each workload of the default benchmark run carries the ncu traffic of its dominant kernel: the expert
+    phases (weight streams at decode, grouped GEMMs at prefill; the Kimi-like layer runs both) all have an
+    entry, so a bench line never reports a null traffic for them."""
+    names = [bench.DEFAULT_WORKLOAD] + list(bench.SECONDARY_WORKLOADS)
+    for name in names:
+        cfg = synth.WORKLOADS[name]
+        phases = ["expert_up_stream", "expert_down_stream"] if cfg.tokens <= 32 else ["expert_up_gemm",
+                                                                                       "expert_down_gemm"]
+        for ph in phases:
+            assert (name, ph) in bench.NCU_TRAFFIC, (name, ph)
+            assert bench.NCU_TRAFFIC[(name, ph)] > 0
+
