@@ -1511,13 +1511,16 @@ int lmoe_forward(lmoe_handle* h, const void* x, void* y, int32_t T, void* stream
 bool host_copy_ready(lmoe_handle* h) {
     if (h->hcopy != nullptr) return true;
     cudaStream_t cs = nullptr;
-    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return false;
-    for (int b = 0; b < 2; ++b)
-        if (cudaEventCreateWithFlags(&h->ev_in[b], cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&h->ev_used[b], cudaEventDisableTiming) != cudaSuccess) {
-            cudaStreamDestroy(cs);
-            return false;
-        }
+    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};
+    bool ok = cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) == cudaSuccess;
+    for (int i = 0; i < 4 && ok; ++i) ok = cudaEventCreateWithFlags(&ev[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {  // nothing half made stays behind
+        for (cudaEvent_t e : ev)
+            if (e != nullptr) cudaEventDestroy(e);
+        if (cs != nullptr) cudaStreamDestroy(cs);
+        return false;
+    }
+    h->ev_in[0] = ev[0], h->ev_in[1] = ev[1], h->ev_used[0] = ev[2], h->ev_used[1] = ev[3];
     h->hcopy = cs;
     return true;
 }
